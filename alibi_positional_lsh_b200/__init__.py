@@ -1,0 +1,128 @@
+"""Python binding of libplsh (Positional-LSH approximate ALiBi attention, B200).
+
+Argument marshalling only: each function here has the name of the C entry
+point it calls (include/plsh.h), checks that tensors sit where the C side
+expects them, passes raw pointers and the current CUDA stream, and turns a
+nonzero status into PlshError. Every step of the computation runs in the
+library's CUDA kernels; importing this package fails loudly if libplsh.so
+is missing, and there is no other code path.
+
+PyTorch is used for device memory and streams only.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libplsh.so")
+
+PLSH_OK = 0
+PLSH_BF16 = 0
+PLSH_F32 = 1
+PLSH_TILE = 128
+PLSH_MAX_S = 64
+DEVERR_BITS = {1: "RANGE", 2: "TABLE", 4: "WINDOW", 8: "TIMEOUT", 16: "SIGMA"}
+
+
+class PlshError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"libplsh error {code}: {msg}")
+        self.code = code
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built: run `python -m alibi_positional_lsh_b200.build` "
+                          "(or __graft_entry__.build()) first")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, u64, dp = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64, ctypes.c_void_p
+    lib.plsh_last_error.restype = ctypes.c_char_p
+    lib.plsh_last_error.argtypes = []
+    lib.plsh_version.restype = i32
+    lib.plsh_version.argtypes = []
+    lib.plsh_draw_table.restype = i32
+    lib.plsh_draw_table.argtypes = [u64, i32, i32, dp, dp]
+    lib.plsh_sample_bins.restype = i32
+    lib.plsh_sample_bins.argtypes = [vp, i32, i32, i32, vp, vp, vp]
+    lib.plsh_window.restype = i32
+    lib.plsh_window.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp]
+    lib.plsh_attention_fwd.restype = i32
+    lib.plsh_attention_fwd.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, i32, vp, vp, vp, i32,
+                                       vp, vp, vp, vp]
+    return lib
+
+
+_lib = _load()
+
+
+def _check(rc: int) -> None:
+    if rc != PLSH_OK:
+        raise PlshError(rc, _lib.plsh_last_error().decode(errors="replace"))
+
+
+def _dev_ptr(t, name: str):
+    """Pointer of a contiguous CUDA tensor (None passes NULL)."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def plsh_last_error() -> str:
+    return _lib.plsh_last_error().decode(errors="replace")
+
+
+def plsh_version() -> int:
+    return _lib.plsh_version()
+
+
+def plsh_draw_table(seed: int, H: int, s: int, sigma_host: np.ndarray, table_host: np.ndarray) -> None:
+    """Host call: fills table_host float64 [H][s][2] with (delta, u)."""
+    sig = np.ascontiguousarray(sigma_host, dtype=np.float64)
+    if sig.shape != (H,):
+        raise ValueError("sigma_host must have shape [H]")
+    if table_host.dtype != np.float64 or table_host.shape != (H, s, 2) or not table_host.flags.c_contiguous:
+        raise ValueError("table_host must be a contiguous float64 array [H][s][2]")
+    _check(_lib.plsh_draw_table(ctypes.c_uint64(seed & (2 ** 64 - 1)), H, s,
+                                sig.ctypes.data_as(ctypes.c_void_p), table_host.ctypes.data_as(ctypes.c_void_p)))
+
+
+def plsh_sample_bins(table_dev, H: int, s: int, n: int, ids_dev, err_dev, stream=None) -> None:
+    _check(_lib.plsh_sample_bins(_dev_ptr(table_dev, "table_dev"), H, s, n, _dev_ptr(ids_dev, "ids_dev"),
+                                 _dev_ptr(err_dev, "err_dev"), _stream_ptr(stream)))
+
+
+def plsh_window(ids_dev, H: int, s: int, n: int, causal: int, bmax_dev, tile_span_dev, bmask_dev, err_dev,
+                stream=None) -> None:
+    _check(_lib.plsh_window(_dev_ptr(ids_dev, "ids_dev"), H, s, n, int(causal), _dev_ptr(bmax_dev, "bmax_dev"),
+                            _dev_ptr(tile_span_dev, "tile_span_dev"), _dev_ptr(bmask_dev, "bmask_dev"),
+                            _dev_ptr(err_dev, "err_dev"), _stream_ptr(stream)))
+
+
+def plsh_attention_fwd(Q, K, V, dtype: int, B: int, H: int, H_kv: int, n: int, d: int, sigma_dev, s: int,
+                       table_dev, tile_span_dev, bmask_dev, causal: int, O, row_sum, err_dev,
+                       stream=None) -> None:
+    _check(_lib.plsh_attention_fwd(_dev_ptr(Q, "Q"), _dev_ptr(K, "K"), _dev_ptr(V, "V"), dtype, B, H, H_kv, n, d,
+                                   _dev_ptr(sigma_dev, "sigma_dev"), s, _dev_ptr(table_dev, "table_dev"),
+                                   _dev_ptr(tile_span_dev, "tile_span_dev"), _dev_ptr(bmask_dev, "bmask_dev"),
+                                   int(causal), _dev_ptr(O, "O"), _dev_ptr(row_sum, "row_sum"),
+                                   _dev_ptr(err_dev, "err_dev"), _stream_ptr(stream)))
+
+
+def decode_device_error(word: int) -> list:
+    return [name for bit, name in DEVERR_BITS.items() if word & bit]
+
+
+from .api import PlshForward, forward  # noqa: E402,F401

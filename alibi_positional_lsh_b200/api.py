@@ -1,0 +1,129 @@
+"""User-facing forward pass built on the C entry points.
+
+PlshForward owns the device buffers of one problem shape (allocated once
+with torch) and runs the whole path:
+  a1 plsh_draw_table   (host)   -> (delta, u) table, copied to the device
+  a2 plsh_sample_bins  (K1)     -> bin ids
+  a3 plsh_window       (K2)     -> b_max, tile windows, boundary masks
+  a4 plsh_attention_fwd (K3)    -> O, row_sum
+All arithmetic of a2..a4 runs in libplsh's CUDA kernels.
+"""
+from __future__ import annotations
+
+from typing import Optional, Sequence, Tuple
+
+import numpy as np
+import torch
+
+from . import (PLSH_BF16, PLSH_F32, PLSH_TILE, PlshError, decode_device_error, plsh_attention_fwd,
+               plsh_draw_table, plsh_sample_bins, plsh_window)
+
+
+class PlshForward:
+    """Positional-LSH approximate ALiBi attention for one (B, H, H_kv, n, d, s) shape."""
+
+    def __init__(self, B: int, H: int, H_kv: int, n: int, d: int, s: int, causal: bool,
+                 sigma: Sequence[float], seed: int, dtype: torch.dtype = torch.bfloat16,
+                 device: str = "cuda"):
+        if dtype not in (torch.bfloat16, torch.float32):
+            raise ValueError("dtype must be torch.bfloat16 or torch.float32")
+        self.B, self.H, self.H_kv, self.n, self.d, self.s = B, H, H_kv, n, d, s
+        self.causal = bool(causal)
+        self.seed = int(seed)
+        self.dtype = dtype
+        self.dtype_code = PLSH_BF16 if dtype == torch.bfloat16 else PLSH_F32
+        self.device = torch.device(device)
+        self.sigma_host = np.ascontiguousarray(sigma, dtype=np.float64)
+        if self.sigma_host.shape != (H,):
+            raise ValueError("sigma must hold one value per query head")
+        T = (n + PLSH_TILE - 1) // PLSH_TILE
+        dev = self.device
+        self.table_host = torch.empty((H, s, 2), dtype=torch.float64).pin_memory()
+        self._table_copied = None  # event after the last host->device table copy
+        self.table_dev = torch.empty((H, s, 2), dtype=torch.float64, device=dev)
+        self.sigma_dev = torch.from_numpy(self.sigma_host.copy()).to(dev)
+        self.ids = torch.empty((H, s, n), dtype=torch.int32, device=dev)
+        self.bmax = torch.empty((H,), dtype=torch.int32, device=dev)
+        self.spans = torch.empty((H, T, 2), dtype=torch.int32, device=dev)
+        self.bmask = torch.empty((H, n), dtype=torch.int32 if s <= 32 else torch.int64, device=dev)
+        self.err = torch.zeros((4,), dtype=torch.int32, device=dev)
+        self.O = torch.empty((B, H, n, d), dtype=dtype, device=dev)
+        self.row_sum = torch.empty((B, H, n), dtype=torch.float32, device=dev)
+
+    # a1 + a2 + a3
+    def prepare(self, stream: Optional[torch.cuda.Stream] = None, table: Optional[np.ndarray] = None) -> None:
+        """Draws the table (or takes `table`, float64 [H][s][2]) and builds ids, windows and masks."""
+        if self._table_copied is not None:
+            self._table_copied.synchronize()   # the pinned buffer may still be in flight
+        if table is None:
+            plsh_draw_table(self.seed, self.H, self.s, self.sigma_host, self.table_host.numpy())
+        else:
+            t = np.ascontiguousarray(table, dtype=np.float64)
+            if t.shape != (self.H, self.s, 2):
+                raise ValueError("table must be float64 [H][s][2]")
+            self.table_host.numpy()[...] = t
+        st = torch.cuda.current_stream() if stream is None else stream
+        with torch.cuda.stream(st):
+            self.table_dev.copy_(self.table_host, non_blocking=True)
+            self._table_copied = torch.cuda.Event()
+            self._table_copied.record(st)
+        plsh_sample_bins(self.table_dev, self.H, self.s, self.n, self.ids, self.err, st)
+        plsh_window(self.ids, self.H, self.s, self.n, int(self.causal), self.bmax, self.spans, self.bmask,
+                    self.err, st)
+
+    # a4
+    def attend(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+               stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+        B, H, H_kv, n, d = self.B, self.H, self.H_kv, self.n, self.d
+        if q.shape != (B, H, n, d) or k.shape != (B, H_kv, n, d) or v.shape != (B, H_kv, n, d):
+            raise ValueError("q/k/v shapes do not match the plan")
+        for t, nm in ((q, "q"), (k, "k"), (v, "v")):
+            if t.dtype != self.dtype or t.device != self.O.device:
+                raise ValueError(f"{nm} must be {self.dtype} on {self.O.device}")
+        st = torch.cuda.current_stream() if stream is None else stream
+        plsh_attention_fwd(q, k, v, self.dtype_code, B, H, H_kv, n, d, self.sigma_dev, self.s, self.table_dev,
+                           self.spans, self.bmask, int(self.causal), self.O, self.row_sum, self.err, st)
+        return self.O, self.row_sum
+
+    def __call__(self, q, k, v, stream=None, table=None):
+        self.prepare(stream, table)
+        return self.attend(q, k, v, stream)
+
+    def run_host(self, q_host: torch.Tensor, k_host: torch.Tensor, v_host: torch.Tensor,
+                 q_dev: torch.Tensor, k_dev: torch.Tensor, v_dev: torch.Tensor,
+                 o_host: torch.Tensor, rs_host: Optional[torch.Tensor] = None,
+                 stream=None) -> None:
+        """End to end from (pinned) host inputs to host outputs on one stream."""
+        st = torch.cuda.current_stream() if stream is None else stream
+        with torch.cuda.stream(st):
+            q_dev.copy_(q_host, non_blocking=True)
+            k_dev.copy_(k_host, non_blocking=True)
+            v_dev.copy_(v_host, non_blocking=True)
+            self.prepare(st)
+            self.attend(q_dev, k_dev, v_dev, st)
+            o_host.copy_(self.O, non_blocking=True)
+            if rs_host is not None:
+                rs_host.copy_(self.row_sum, non_blocking=True)
+
+    def reset_errors(self) -> None:
+        self.err.zero_()
+
+    def device_errors(self) -> list:
+        """Synchronises and decodes the device error word."""
+        torch.cuda.synchronize(self.O.device)
+        return decode_device_error(int(self.err[0].item()) & 0xFFFFFFFF)
+
+    def check(self) -> None:
+        errs = self.device_errors()
+        if errs:
+            raise PlshError(-1, "device reported " + ",".join(errs))
+
+
+def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, sigma: Sequence[float], s: int, seed: int,
+            causal: bool) -> Tuple[torch.Tensor, torch.Tensor]:
+    """One-shot T~ and row_sum for CUDA tensors q [B,H,n,d], k, v [B,H_kv,n,d]."""
+    B, H, n, d = q.shape
+    plan = PlshForward(B, H, k.shape[1], n, d, s, causal, sigma, seed, q.dtype, str(q.device))
+    O, R = plan(q.contiguous(), k.contiguous(), v.contiguous())
+    plan.check()
+    return O.clone(), R.clone()

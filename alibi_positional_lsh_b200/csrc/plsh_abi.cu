@@ -1,0 +1,89 @@
+// Entry points of libplsh (declared in include/plsh.h): argument checks,
+// then the launch. Every check that can be made on the host is made here,
+// before anything is enqueued.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "plsh_internal.h"
+
+namespace plsh {
+
+namespace {
+thread_local char g_last_error[512] = "";
+}
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(PLSH_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_sizes(const char* fn, int H, int s, int n) {
+  if (H < 1 || n < 1) return fail(PLSH_ERR_INVALID_ARG, "%s: need H >= 1 and n >= 1 (H=%d n=%d)", fn, H, n);
+  if (s < 1 || s > PLSH_MAX_S)
+    return fail(PLSH_ERR_INVALID_ARG, "%s: need 1 <= s <= %d (s=%d)", fn, PLSH_MAX_S, s);
+  if (H > 65535) return fail(PLSH_ERR_RANGE, "%s: H=%d exceeds 65535", fn, H);
+  if (n > (1 << 30)) return fail(PLSH_ERR_RANGE, "%s: n=%d exceeds 2^30", fn, n);
+  return PLSH_OK;
+}
+
+}  // namespace
+}  // namespace plsh
+
+using plsh::fail;
+
+extern "C" const char* plsh_last_error(void) { return plsh::g_last_error; }
+
+extern "C" int plsh_version(void) { return 100; }
+
+extern "C" int plsh_sample_bins(const double* table_dev, int H, int s, int n, int32_t* ids_dev,
+                                uint32_t* err_dev, void* stream) {
+  if (int rc = plsh::check_sizes("plsh_sample_bins", H, s, n)) return rc;
+  if (!table_dev || !ids_dev || !err_dev) return fail(PLSH_ERR_INVALID_ARG, "plsh_sample_bins: null pointer");
+  return plsh::launch_sample_bins(table_dev, H, s, n, ids_dev, err_dev, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int plsh_window(const int32_t* ids_dev, int H, int s, int n, int causal, int32_t* bmax_dev,
+                           int32_t* tile_span_dev, void* bmask_dev, uint32_t* err_dev, void* stream) {
+  if (int rc = plsh::check_sizes("plsh_window", H, s, n)) return rc;
+  if (!ids_dev || !bmax_dev || !tile_span_dev || !bmask_dev || !err_dev)
+    return fail(PLSH_ERR_INVALID_ARG, "plsh_window: null pointer");
+  if (causal != 0 && causal != 1) return fail(PLSH_ERR_INVALID_ARG, "plsh_window: causal must be 0 or 1");
+  return plsh::launch_window(ids_dev, H, s, n, causal, bmax_dev, tile_span_dev, bmask_dev, err_dev,
+                             static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int plsh_attention_fwd(const void* Q, const void* K, const void* V, int dtype, int B, int H,
+                                  int H_kv, int n, int d, const double* sigma_dev, int s,
+                                  const double* table_dev, const int32_t* tile_span_dev,
+                                  const void* bmask_dev, int causal, void* O, float* row_sum,
+                                  uint32_t* err_dev, void* stream) {
+  const char* fn = "plsh_attention_fwd";
+  if (int rc = plsh::check_sizes(fn, H, s, n)) return rc;
+  if (B < 1 || B > 65535) return fail(PLSH_ERR_INVALID_ARG, "%s: need 1 <= B <= 65535 (B=%d)", fn, B);
+  if (H_kv < 1 || H % H_kv != 0)
+    return fail(PLSH_ERR_INVALID_ARG, "%s: H_kv must divide H (H=%d H_kv=%d)", fn, H, H_kv);
+  if (causal != 0 && causal != 1) return fail(PLSH_ERR_INVALID_ARG, "%s: causal must be 0 or 1", fn);
+  if (dtype != PLSH_BF16 && dtype != PLSH_F32) return fail(PLSH_ERR_UNSUPPORTED, "%s: dtype %d", fn, dtype);
+  if (d != 64 && d != 128) return fail(PLSH_ERR_UNSUPPORTED, "%s: head dim %d (64 or 128 supported)", fn, d);
+  if (!Q || !K || !V || !O || !row_sum || !tile_span_dev || !bmask_dev || !err_dev)
+    return fail(PLSH_ERR_INVALID_ARG, "%s: null pointer", fn);
+  if (!plsh::aligned16(Q) || !plsh::aligned16(K) || !plsh::aligned16(V) || !plsh::aligned16(O))
+    return fail(PLSH_ERR_INVALID_ARG, "%s: Q, K, V and O must be 16-byte aligned", fn);
+  plsh::AttnArgs a{Q, K, V, dtype, B, H, H_kv, n, d, s, causal, sigma_dev, table_dev,
+                   tile_span_dev, bmask_dev, O, row_sum, err_dev};
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == PLSH_BF16 && d == 128) return plsh::launch_attention_tc(a, st);
+  return plsh::launch_attention_simt(a, st);
+}

@@ -1,0 +1,36 @@
+// Internal declarations shared by the libplsh translation units.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "plsh.h"
+
+namespace plsh {
+
+// Records a message for plsh_last_error() and returns `code`.
+int fail(int code, const char* fmt, ...);
+// Maps a CUDA error to PLSH_ERR_CUDA with the call site in the message.
+int cuda_fail(cudaError_t e, const char* what);
+
+inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Kernel launchers (each returns PLSH_OK or an error code; arguments are
+// already validated by the entry point).
+int launch_sample_bins(const double* table, int H, int s, int n, int32_t* ids, uint32_t* err,
+                       cudaStream_t st);
+int launch_window(const int32_t* ids, int H, int s, int n, int causal, int32_t* bmax,
+                  int32_t* spans, void* bmask, uint32_t* err, cudaStream_t st);
+
+struct AttnArgs {
+  const void* Q; const void* K; const void* V;
+  int dtype, B, H, H_kv, n, d, s, causal;
+  const double* sigma; const double* table;
+  const int32_t* spans; const void* bmask;
+  void* O; float* row_sum; uint32_t* err;
+};
+int launch_attention_simt(const AttnArgs& a, cudaStream_t st);
+int launch_attention_tc(const AttnArgs& a, cudaStream_t st);
+
+}  // namespace plsh

@@ -1,0 +1,175 @@
+/*
+ * plsh.h -- C ABI of libplsh: Positional-LSH approximate ALiBi attention on
+ * NVIDIA B200 (sm_100a).
+ *
+ * Method: "Positional LSH: Binary Block Matrix Approximation for Attention
+ * with Linear Biases" (Wolfson & Wagner, arXiv 2605.09472), as summarised by
+ * the gist.science explainer pages (nl/zh/ja). ALiBi's bias matrix
+ * L*_ij = e^{-|i-j|/sigma} is the expectation of the binary block masks M(h)
+ * of random binnings of the token positions (technical summary, Methodology
+ * 1, "mechanism" and "expectation"); the mean M~ of s such masks approximates
+ * it (Methodology 2, Theorem 2.1), and attention weighted by M~ approximates
+ * ALiBi attention (Methodology 3, Theorem 2.2; Results, convergence of
+ * ||T* - T~||). This library computes
+ *
+ *     T~ = D~^{-1} (exp(Q K^T / sqrt d) o M~) V,   M~ = (1/s) sum_k M(h_k),
+ *
+ * optionally with the causal mask j <= i, for grouped-query attention.
+ *
+ * Conventions for every entry point:
+ *   - Returns PLSH_OK (0) or a PLSH_ERR_* code; on error nothing was
+ *     launched and plsh_last_error() (thread-local) says why.
+ *   - "_dev" pointers are device memory owned by the caller; "_host"
+ *     pointers are host memory owned by the caller. The library allocates
+ *     no device memory and keeps no state between calls except the
+ *     thread-local error string and a cached driver entry point.
+ *   - Device work is enqueued on `stream` (a cudaStream_t passed as void*,
+ *     NULL = legacy default stream) and is asynchronous: no entry point
+ *     synchronises the device.
+ *   - err_dev is a caller-zeroed device uint32 word. Kernels OR PLSH_DEVERR_*
+ *     bits into it when they meet bad data that only the device can see
+ *     (a bin id overflowing int32, a window outside [0, n), a bounded wait
+ *     that gave up). Read it after the stream has finished. A kernel that
+ *     sets a bit still ends normally; its outputs are then unspecified.
+ *   - Positions are 0-based. Tensors are dense row-major (C order).
+ */
+#ifndef PLSH_H_
+#define PLSH_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PLSH_API __attribute__((visibility("default")))
+#else
+#define PLSH_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes. */
+#define PLSH_OK               0
+#define PLSH_ERR_INVALID_ARG  1  /* a null pointer, a negative size, s out of range, H % H_kv != 0 */
+#define PLSH_ERR_UNSUPPORTED  2  /* head dim / dtype combination without a kernel */
+#define PLSH_ERR_RANGE        3  /* a size whose index arithmetic would overflow */
+#define PLSH_ERR_CUDA         4  /* a CUDA runtime or driver call failed */
+
+/* Bits a kernel ORs into *err_dev. */
+#define PLSH_DEVERR_RANGE    1u  /* a relative bin id did not fit in int32 */
+#define PLSH_DEVERR_TABLE    2u  /* a table entry with delta not finite and > 0, or u not finite */
+#define PLSH_DEVERR_WINDOW   4u  /* a tile window outside [0, n) or not covering the tile's own rows */
+#define PLSH_DEVERR_TIMEOUT  8u  /* a bounded wait on a barrier gave up (the kernel returned early) */
+#define PLSH_DEVERR_SIGMA   16u  /* a per-head sigma not finite and > 0 */
+
+#define PLSH_TILE   128   /* query/key tile height of the windows */
+#define PLSH_MAX_S  64    /* most hashes per head (one bit each in a 64-bit boundary mask) */
+
+/* dtype codes for Q, K, V and O. */
+#define PLSH_BF16 0
+#define PLSH_F32  1
+
+/* Thread-local description of the last error returned on this thread. */
+PLSH_API const char* plsh_last_error(void);
+
+/* ABI version (major * 100 + minor). */
+PLSH_API int plsh_version(void);
+
+/*
+ * plsh_draw_table -- the (delta, u) table of s random binnings per head, on
+ * the host.
+ *
+ * Cites: Methodology 1 (random binning of the integer positions, after
+ * Rahimi & Recht's Random Binning Features for the Laplace kernel) and
+ * Methodology 2 (s i.i.d. hashes; the Gamma law behind the binning).
+ * For head h and hash k: delta = -sigma_h (ln U1 + ln U2) ~ Gamma(shape 2,
+ * scale sigma_h) and u = U3 * delta ~ U[0, delta), with U1, U2 in (0,1) and
+ * U3 in [0,1) taken from SplitMix64(seed) outputs ((h << 16) | k) * 3 + 0,1,2
+ * (U_open = ((z >> 12) + 1/2) 2^-52, U3 = (z >> 11) 2^-53). A table with s
+ * hashes is a prefix of one with more.
+ *
+ *   seed        64-bit seed.
+ *   H           heads, >= 1.
+ *   s           hashes per head, 1..PLSH_MAX_S.
+ *   sigma_host  [H] doubles, each finite and > 0 (else PLSH_ERR_INVALID_ARG).
+ *   table_host  [H][s][2] doubles written as (delta, u).
+ * Pure host code; needs no GPU.
+ */
+PLSH_API int plsh_draw_table(uint64_t seed, int H, int s, const double* sigma_host, double* table_host);
+
+/*
+ * plsh_sample_bins (K1) -- bin ids of every (head, hash, position).
+ *
+ * Cites: Methodology 1, mechanism (h splits the positions into contiguous
+ * bins). id_{h,k}(i) = floor((i + u)/delta) - floor(u/delta) with IEEE
+ * float64 add and divide, round to nearest, so ids are bit-exact with any
+ * IEEE float64 evaluation of the same formula.
+ *
+ *   table_dev  [H][s][2] doubles (delta, u).
+ *   H, s, n    heads, hashes (1..PLSH_MAX_S), positions (>= 1).
+ *   ids_dev    [H][s][n] int32 out.
+ *   err_dev    device error word (PLSH_DEVERR_RANGE, PLSH_DEVERR_TABLE).
+ */
+PLSH_API int plsh_sample_bins(const double* table_dev, int H, int s, int n, int32_t* ids_dev,
+                     uint32_t* err_dev, void* stream);
+
+/*
+ * plsh_window (K2) -- b_max, per-tile key windows and boundary masks.
+ *
+ * Cites: Methodology 1, structure (blocks are contiguous and do not
+ * overlap) and Methodology 2, block-size control (b_max ~ sigma log log n).
+ *
+ *   ids_dev        [H][s][n] int32 from plsh_sample_bins.
+ *   causal         0 or 1.
+ *   bmax_dev       [H] int32 out: longest run of equal ids over the s hashes.
+ *   tile_span_dev  [H][ceil(n/128)][2] int32 out: for query rows
+ *                  [128t, min(n,128t+128)), the inclusive key range [lo, hi]
+ *                  holding every key with a nonzero M~ weight for some row of
+ *                  the tile (and key <= row when causal).
+ *   bmask_dev      [H][n] boundary masks out: bit k of entry p is set iff
+ *                  hash k starts a block at p (entry 0 has all s bits).
+ *                  uint32 entries when s <= 32, uint64 entries when s > 32.
+ *   err_dev        device error word.
+ */
+PLSH_API int plsh_window(const int32_t* ids_dev, int H, int s, int n, int causal, int32_t* bmax_dev,
+                int32_t* tile_span_dev, void* bmask_dev, uint32_t* err_dev, void* stream);
+
+/*
+ * plsh_attention_fwd (K3) -- the fused banded Positional-LSH attention.
+ *
+ * Cites: Methodology 2 (M~ = (1/s) sum_k M(h_k)), Methodology 3 (ALiBi
+ * attention reduced to attention restricted to short random blocks) and the
+ * Results' convergence bullet (T~ as the approximation of T*). Per query
+ * head h with KV head h / (H/H_kv):
+ *   O_i       = sum_j c_ij e^{S_ij} V_j / sum_j c_ij e^{S_ij},  S = Q K^T / sqrt d,
+ *   row_sum_i = ln( sum_j (c_ij / s) e^{S_ij} )   (natural log, float32),
+ * with c_ij = number of hashes putting i and j in one bin, restricted to
+ * j <= i when causal. c_ij is read from the boundary masks:
+ * c_ij = s - popcount(OR of bmask over (min(i,j), max(i,j)]).
+ *
+ *   Q              [B][H][n][d]; K, V [B][H_kv][n][d]; O like Q.
+ *   dtype          PLSH_BF16 (bf16 in and out, fp32 accumulation, tcgen05
+ *                  tensor cores when d == 128) or PLSH_F32 (fp32 in and out,
+ *                  fp32 CUDA-core arithmetic).
+ *   d              64 or 128.
+ *   sigma_dev      [H] doubles, the ALiBi length scales the table was drawn
+ *                  for; checked finite and > 0 (PLSH_DEVERR_SIGMA). May be NULL.
+ *   s              hashes per head, as given to plsh_window.
+ *   table_dev      [H][s][2] the table the masks were built from; its pitches
+ *                  are checked (PLSH_DEVERR_TABLE). May be NULL.
+ *   tile_span_dev, bmask_dev   from plsh_window with the same causal flag.
+ *   row_sum        [B][H][n] float32 out.
+ * Every pointer must be 16-byte aligned.
+ */
+PLSH_API int plsh_attention_fwd(const void* Q, const void* K, const void* V, int dtype, int B, int H,
+                       int H_kv, int n, int d, const double* sigma_dev, int s,
+                       const double* table_dev, const int32_t* tile_span_dev,
+                       const void* bmask_dev, int causal, void* O, float* row_sum,
+                       uint32_t* err_dev, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PLSH_H_ */

@@ -1,0 +1,104 @@
+"""The C-ABI library without a GPU: it loads, exports every symbol the header
+declares, its host-side table sampler matches the oracle bit for bit, and
+its host-side argument checks return the documented codes before any
+device work."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "plsh.h")
+
+
+def _declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(plsh_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def plsh():
+    import alibi_positional_lsh_b200 as m
+    return m
+
+
+def test_header_declares_the_path():
+    syms = _declared_symbols()
+    for want in ("plsh_draw_table", "plsh_sample_bins", "plsh_window", "plsh_attention_fwd", "plsh_last_error"):
+        assert want in syms, syms
+
+
+def test_library_exports_every_declared_symbol(plsh):
+    lib = ctypes.CDLL(plsh.LIB_PATH)
+    for name in _declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_version(plsh):
+    assert plsh.plsh_version() >= 100
+
+
+@pytest.mark.parametrize("seed,sigma,s", [
+    (0, [16.0], 8),
+    (1, [2.0 ** (h + 1) for h in range(8)], 10),
+    (2, [2.0 ** ((h + 1) / 2) for h in range(16)], 20),
+    (3, [2.0 ** ((h + 1) / 4) for h in range(32)], 40),
+    (4, [2.0 ** (8 * (h + 1) / 40) for h in range(40)], 16),
+    (2 ** 64 - 1, [1e-3, 1e6], 64),
+])
+def test_draw_table_bit_exact_with_oracle(plsh, seed, sigma, s):
+    H = len(sigma)
+    got = np.empty((H, s, 2), dtype=np.float64)
+    plsh.plsh_draw_table(seed, H, s, np.asarray(sigma), got)
+    want = oracle.draw_table(seed, sigma, s)
+    assert got.tobytes() == want.tobytes()
+
+
+def test_draw_table_for_every_workload(plsh):
+    for w in workloads.WORKLOADS.values():
+        got = np.empty((w.H, w.s, 2))
+        plsh.plsh_draw_table(w.seed, w.H, w.s, np.asarray(w.sigmas()), got)
+        assert got.tobytes() == oracle.draw_table(w.seed, w.sigmas(), w.s).tobytes()
+
+
+def test_draw_table_rejects_bad_arguments(plsh):
+    t = np.empty((1, 4, 2))
+    for sigma in ([0.0], [-1.0], [float("nan")], [float("inf")]):
+        with pytest.raises(plsh.PlshError) as e:
+            plsh.plsh_draw_table(1, 1, 4, np.asarray(sigma), t)
+        assert e.value.code == 1
+    with pytest.raises(plsh.PlshError):
+        plsh.plsh_draw_table(1, 1, 65, np.asarray([1.0]), np.empty((1, 65, 2)))
+
+
+def test_entry_points_reject_bad_sizes_before_any_launch(plsh):
+    lib = plsh._lib
+    null = None
+    # invalid sizes or null pointers: INVALID_ARG (1), returned by host checks
+    assert lib.plsh_sample_bins(null, 1, 0, 10, null, null, null) == 1
+    assert lib.plsh_sample_bins(null, 1, 4, 10, null, null, null) == 1
+    assert lib.plsh_window(null, 1, 4, 10, 2, null, null, null, null, null) == 1
+    assert lib.plsh_window(null, 0, 4, 10, 0, null, null, null, null, null) == 1
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the checks fail first
+    # head dim without a kernel: UNSUPPORTED (2)
+    rc = lib.plsh_attention_fwd(fake, fake, fake, 0, 1, 1, 1, 128, 96, null, 4, null, fake, fake, 0, fake, fake,
+                                fake, null)
+    assert rc == 2 and "head dim" in plsh.plsh_last_error()
+    # H_kv not dividing H
+    rc = lib.plsh_attention_fwd(fake, fake, fake, 0, 1, 6, 4, 128, 128, null, 4, null, fake, fake, 0, fake, fake,
+                                fake, null)
+    assert rc == 1
+    # misaligned Q
+    rc = lib.plsh_attention_fwd(ctypes.c_void_p((1 << 20) + 8), fake, fake, 0, 1, 1, 1, 128, 128, null, 4, null,
+                                fake, fake, 0, fake, fake, fake, null)
+    assert rc == 1 and "aligned" in plsh.plsh_last_error()
+    # unknown dtype
+    rc = lib.plsh_attention_fwd(fake, fake, fake, 7, 1, 1, 1, 128, 128, null, 4, null, fake, fake, 0, fake, fake,
+                                fake, null)
+    assert rc == 2
