@@ -1,0 +1,440 @@
+"""Throughput of Positional-LSH approximate ALiBi attention on B200.
+
+One step = the whole forward path on one batch of synthetic inputs already in
+HBM: table draw (host) + its copy, bin ids (K1), windows and boundary masks
+(K2), fused attention (K3). Metric: query tokens per second (B * n per step,
+summed over ranks), plus the roofline fraction of the attention kernel.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   (the CPU oracle on a bounded sample)
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own independent
+problem of the same shape (the path has no exchange step), so per-GPU work is
+fixed and scaling is weak; the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+TILE = 128
+ATTN_KERNEL_SRC = os.path.join(ROOT, "alibi_positional_lsh_b200", "csrc", "plsh_attn_tc.cu")
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "attn_tc_qwen3_0p6b_n32k.md")
+
+
+# ---------------------------------------------------------------- helpers
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in PEAKS_FALLBACK}, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def kernel_source_hash() -> str:
+    with open(ATTN_KERNEL_SRC, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch of the attention kernel from the committed ncu summary,
+    or None when absent or taken on a different kernel source."""
+    if not os.path.exists(PROFILE_SUMMARY):
+        return None
+    text = open(PROFILE_SUMMARY).read()
+    mh = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
+    mt = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not mh or not mt or mh.group(1) != kernel_source_hash():
+        return None
+    return float(mt.group(1))
+
+
+class ClockSampler:
+    """SM clock and clock-event reasons sampled through NVML every ~2 ms while the timed region runs."""
+
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, local_index: int, period_s: float = 0.002):
+        self.local_index = local_index
+        self.period = period_s
+        self.samples = []
+        self.error = None
+        self._stop = None
+        self._thread = None
+
+    def _handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.local_index)
+        bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+        return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+
+    def __enter__(self):
+        import threading
+        try:
+            self.nvml, self.h = self._handle()
+            self.max_mhz = self.nvml.nvmlDeviceGetMaxClockInfo(self.h, self.nvml.NVML_CLOCK_SM)
+        except Exception as e:  # pragma: no cover - no NVML on this host
+            self.error = f"nvml unavailable: {e}"
+            return self
+        self._stop = threading.Event()
+
+        def loop():
+            while not self._stop.is_set():
+                try:
+                    mhz = self.nvml.nvmlDeviceGetClockInfo(self.h, self.nvml.NVML_CLOCK_SM)
+                    rs = self.nvml.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                    self.samples.append((mhz, rs))
+                except Exception as e:  # pragma: no cover
+                    self.error = str(e)
+                    return
+                time.sleep(self.period)
+
+        self._thread = threading.Thread(target=loop, daemon=True)
+        self._thread.start()
+        time.sleep(0.02)
+        return self
+
+    def __exit__(self, *a):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=2)
+
+    def summary(self):
+        if self.error or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.error or "no samples"], "samples": 0,
+                    "source": "nvml"}
+        mhz = [m for m, _ in self.samples]
+        reasons = sorted({name for _, rs in self.samples for name, bit in self.REASONS.items() if rs & bit})
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.samples), "source": "nvml, every 2 ms during the timed region"}
+
+
+def issued_tiles(spans: np.ndarray, causal: bool) -> int:
+    """Key tiles of 128 the fused kernel's window covers, summed over heads and query tiles:
+    ceil((hi - lo + 1) / 128) per query tile (the span rounded to the MMA N granularity)."""
+    lo = spans[..., 0].astype(np.int64)
+    hi = spans[..., 1].astype(np.int64)
+    return int(np.sum((hi - lo + 1 + TILE - 1) // TILE))
+
+
+def kernel_tiles(spans: np.ndarray, causal: bool) -> int:
+    """Key tiles the fused kernel actually visits (128-aligned around the diagonal)."""
+    T = spans.shape[1]
+    i0 = (np.arange(T) * TILE)[None, :]
+    lo = spans[..., 0].astype(np.int64)
+    hi = spans[..., 1].astype(np.int64)
+    below = (i0 - lo + TILE - 1) // TILE
+    above = 0 if causal else (hi - i0) // TILE
+    return int(np.sum(1 + below + above))
+
+
+# ---------------------------------------------------------------- distributed plumbing
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def dist_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+# ---------------------------------------------------------------- CPU oracle (baseline and reference arm)
+
+class OracleSampler:
+    """The CPU oracle on query rows of batch element 0, all heads, of one workload.
+
+    Inputs, table and bin ids are prepared once; run(budget_s) then computes
+    rows (8 at a time, every head) until the budget is spent and returns the
+    equivalent query-tokens/s = (row, head) units / time / H.
+    """
+
+    def __init__(self, w: workloads.Workload):
+        import oracle
+        self.oracle = oracle
+        self.w = w
+        g = torch.Generator().manual_seed(w.seed)
+        self.q = torch.randn(1, w.H, w.n, w.d, generator=g).to(w.torch_dtype).double().numpy()
+        self.k = torch.randn(1, w.H_kv, w.n, w.d, generator=g).to(w.torch_dtype).double().numpy()
+        self.v = torch.randn(1, w.H_kv, w.n, w.d, generator=g).to(w.torch_dtype).double().numpy()
+        self.table = oracle.draw_table(w.seed, w.sigmas(), w.s)
+        self.ids = oracle.bin_ids(self.table, w.n)
+        self.rows = workloads.sample_rows(w.n, min(w.n, 4096), w.seed)
+        self.next = 0
+        self.cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+
+    def run(self, budget_s: float):
+        from threadpoolctl import threadpool_limits
+        w = self.w
+        group = w.H // w.H_kv
+        units = 0
+        with threadpool_limits(limits=self.cores):
+            t0 = time.perf_counter()
+            while True:
+                rows = self.rows[self.next:self.next + 8]
+                self.next = (self.next + 8) % len(self.rows)
+                for h in range(w.H):
+                    self.oracle.approx_attention(self.q[0, h], self.k[0, h // group], self.v[0, h // group],
+                                                 self.ids[h], w.causal, rows)
+                    units += len(rows)
+                if time.perf_counter() - t0 >= budget_s:
+                    break
+            dt = time.perf_counter() - t0
+        rate = units / dt / w.H
+        desc = (f"{units // w.H} query rows x all {w.H} heads of batch element 0 of {w.name} "
+                f"({units} row-head units in {dt:.1f} s, float64 numpy on {self.cores} cores); "
+                f"query-tokens/s = units / time / H")
+        return rate, desc
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, local):
+    from alibi_positional_lsh_b200 import PlshForward
+    import alibi_positional_lsh_b200 as plsh_mod  # noqa: F401
+
+    w = workloads.WORKLOADS[args.workload]
+    if args.batch:
+        w = w.with_(B=args.batch)
+    dev = f"cuda:{local}"
+    torch.cuda.set_device(local)
+    wr = w.with_(seed=w.seed + 1000 * rank)          # independent problem per rank
+    q, k, v = workloads.make_qkv_device(wr, dev)
+    plan = PlshForward(w.B, w.H, w.H_kv, w.n, w.d, w.s, w.causal, w.sigmas(), wr.seed, w.torch_dtype, dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        plan.prepare(stream)
+        if ev is not None:
+            ev[0].record(stream)
+        plan.attend(q, k, v, stream)
+        if ev is not None:
+            ev[1].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    errs = plan.device_errors()
+    if errs:
+        raise RuntimeError(f"device errors during warm-up: {errs}")
+    spans = plan.spans.cpu().numpy()
+    tiles_min = issued_tiles(spans, w.causal)
+    tiles_run = kernel_tiles(spans, w.causal)
+
+    # timed region: K steps, device-timed, inputs (Q+K+V > L2) already resident
+    K = args.steps
+    ev_k = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        start.record(stream)
+        for i in range(K):
+            step(ev_k[i])
+        end.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    ms_total = start.elapsed_time(end)
+    attn_ms = [a.elapsed_time(b) for a, b in ev_k]
+    ms_total = dist_max(ms_total, world)
+    ms_step = ms_total / K
+    attn_avg = dist_max(sum(attn_ms) / K, world)
+    clocks = clk.summary()
+    errs = plan.device_errors()
+    if errs:
+        raise RuntimeError(f"device errors during the timed region: {errs}")
+
+    # end to end through the public API: pinned host Q/K/V in, host O and row_sum out
+    qh = q.cpu().pin_memory()
+    kh = k.cpu().pin_memory()
+    vh = v.cpu().pin_memory()
+    oh = torch.empty_like(plan.O, device="cpu").pin_memory()
+    rh = torch.empty_like(plan.row_sum, device="cpu").pin_memory()
+    qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    for _ in range(3):
+        plan.run_host(qh, kh, vh, qd, kd, vd, oh, rh, stream)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    Ke = max(3, min(K, 20))
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(Ke):
+        plan.run_host(qh, kh, vh, qd, kd, vd, oh, rh, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = dist_max(e0.elapsed_time(e1) / Ke, world)
+    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh)) + plan.table_host.numel() * 8
+    d2h = oh.numel() * oh.element_size() + rh.numel() * 4
+
+    tokens = w.B * w.n * world
+    value = tokens / (ms_step * 1e-3)
+    peaks, peak_src = load_peaks()
+    elt = 2 if w.dtype == "bf16" else 4
+    qkvo_bytes = (w.B * w.H * w.n * w.d * 2 + 2 * w.B * w.H_kv * w.n * w.d) * elt
+    flops = 4.0 * w.d * TILE * TILE * tiles_min * w.B
+    t_mem = qkvo_bytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    attn_s = attn_avg * 1e-3
+    if t_mem >= t_tc:
+        roof = {"bound": "hbm", "achieved": qkvo_bytes / attn_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": flops / attn_s / 1e12, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = profiled_traffic()
+    roof.update({
+        "peak_source": f"{peak_src} (burst figures of MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback",
+        "kernel": "attn_tc_kernel" if (w.dtype == "bf16" and w.d == 128) else "attn_simt_kernel",
+        "kernel_ms": attn_avg,
+        "algorithmic_bytes": qkvo_bytes,
+        "issued_tensor_flops": flops,
+        "roofline_ms": max(t_mem, t_tc) * 1e3,
+        "t_mem_ms": t_mem * 1e3,
+        "t_tensor_ms": t_tc * 1e3,
+        "frac_vs_sustained_tensor": (max(t_mem, flops / (peaks["bf16_tflops_sustained"] * 1e12)) / attn_s),
+        "key_tiles_per_batch": tiles_min,
+        "key_tiles_visited_per_batch": tiles_run,
+    })
+
+    line = {
+        "metric": "PLSH-ALiBi fwd query-tokens/s at n=32k, s=20; achieved % of roofline",
+        "value": value,
+        "unit": "query-tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": max(3, args.warmup),
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": w.dtype,
+        "data": "synthetic (iid N(0,1) Q/K/V drawn on the device, seeded per rank)",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.H_kv, "n": w.n, "d": w.d, "s": w.s,
+                   "causal": w.causal, "global_batch": w.B * world, "seq_len": w.n,
+                   "parallelism": f"independent problem per GPU x{world}",
+                   "l2": f"no flush: Q+K+V = {(qkvo_bytes * 3 // 4) / 1e6:.0f} MB per step, larger than the 126 MB L2"},
+        "roofline": roof,
+        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "query-tokens/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "path": "PlshForward.run_host: pinned host Q/K/V -> device -> table, K1, K2, K3 -> host O, row_sum"},
+        "gpu_launches": 4 * K,
+        "gpu_launches_per_step": {"sample_bins_kernel": 1, "mask_bmax_kernel": 1, "spans_kernel": 1,
+                                  roof["kernel"]: 1},
+        "step_breakdown_ms": {"attention": attn_avg, "table+bins+window": ms_step - attn_avg},
+        "clocks": clocks,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        sampler = OracleSampler(w)
+        rate, desc = sampler.run(args.cpu_seconds)
+        line["cpu_baseline"] = {"value": rate, "unit": "query-tokens/s", "cores": sampler.cores, "kind": "oracle",
+                                "sample": desc}
+    return line
+
+
+def run_reference(args, rank, world):
+    """The CPU oracle as the reference arm: rank 0 only, a bounded sample per step."""
+    w = workloads.WORKLOADS[args.workload]
+    if rank != 0:
+        return None
+    sampler = OracleSampler(w)
+    per_step = min(5.0, max(0.5, args.cpu_seconds / max(1, args.steps)))
+    for _ in range(args.warmup):
+        sampler.run(0.2)
+    rates = []
+    t0 = time.perf_counter()
+    desc = ""
+    for _ in range(args.steps):
+        r, desc = sampler.run(per_step)
+        rates.append(r)
+    dt = time.perf_counter() - t0
+    value = statistics.mean(rates)
+    return {
+        "impl": "reference",
+        "metric": "PLSH-ALiBi fwd query-tokens/s at n=32k, s=20; achieved % of roofline",
+        "value": value,
+        "unit": "query-tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": dt * 1e3 / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (iid N(0,1) Q/K/V, seeded)",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.H_kv, "n": w.n, "d": w.d, "s": w.s,
+                   "causal": w.causal},
+        "cpu_baseline": {"value": value, "unit": "query-tokens/s", "cores": sampler.cores, "kind": "oracle",
+                         "sample": f"each step: {desc}"},
+        "e2e": {"value": value, "unit": "query-tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=workloads.HEADLINE, choices=list(workloads.WORKLOADS))
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (smaller cases for profiling)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    rank, world, local = dist_setup(args.gpus) if args.impl == "ours" else (
+        int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), 0)
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, rank, world)
+        else:
+            line = run_ours(args, rank, world, local)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if args.impl == "ours" and world > 1 and torch.distributed.is_initialized():
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
