@@ -11,31 +11,41 @@
 // visited (Methodology 3: attention restricted to short random blocks).
 //
 // Persistent CTAs (one per SM) walk a static list of work items, heads with
-// the widest windows first. Warp roles (256 threads):
-//   warp 0      TMA producer: Q per item (2 buffers), K and V per key tile (2-stage rings)
-//   warp 1      TMEM owner and single-thread tcgen05.mma issuer
-//   warp 2      mask producer: the key tile's boundary masks into shared memory
-//   warps 4-7   softmax: one query row per thread (TMEM lane = row)
+// the widest windows first. Warp roles (352 threads):
+//   warps 0-7    softmax: warps 0-3 own key columns 0-63 and warps 4-7 key
+//                columns 64-127 of query row (warp % 4) * 32 + lane
+//   warp 8       TMA producer: Q per item (2 buffers), K and V per key tile (2-stage rings)
+//   warp 9       TMEM owner and single-thread tcgen05.mma issuer
+//   warp 10      mask warp: the key tile's boundary masks and their in-tile
+//                prefix / suffix ORs; for 32-bit masks also the tile's table
+//                of log2 weights (below)
 // Per key tile g (counted across items): S_g = Q K_g^T (SS MMA into TMEM,
-// double-buffered); the softmax warps turn S_g into bf16 P_g in TMEM; then
-// O += P_g V_g (TS MMA: P from TMEM, fp32 O in TMEM). S_{g+1} is issued
-// before PV_g so the tensor core works while the softmax runs.
+// double-buffered); the softmax warps turn S_g into bf16 P_g written over
+// the first 64 columns of S_g; then O += P_g V_g (TS MMA, P from TMEM, fp32 O
+// in TMEM, one O buffer per item parity). S_{g+1} is issued before PV_g so
+// the tensor core works while the softmax runs. An item's epilogue (O / l)
+// runs after the next item's first tile, when its last PV has long finished.
 //
-// Weights: a row keeps a running OR R of the boundary masks between itself
-// and the current key while it walks the tile's columns away from itself;
-// log2(s - popcount(R)) is only recomputed where some hash opens a block
-// (checked four keys at a time, the same for the whole warp). The logit is
-// x = S * log2(e)/sqrt(d) + log2(c_ij) (-inf where c_ij = 0), so
-// P = 2^(x - m) = c_ij 2^(S log2(e)/sqrt(d) - m). Key tiles are visited
-// diagonal first, then downward, then upward, so the OR passed so far carries
-// from tile to tile. The reference maximum m moves only when a tile's
-// maximum exceeds it by more than 8 (then O and the row sum are rescaled),
-// which keeps every P <= 256.
+// Weights. The logit is x = S * log2(e)/sqrt(d) + log2(c_ij) (-inf where
+// c_ij = 0), so P = 2^(x - m) = c_ij 2^(S log2(e)/sqrt(d) - m). Key tiles are
+// visited diagonal first, then downward, then upward. Below the diagonal
+// the OR over (j, i] splits into SUF[c] (inside the key tile) and the row's
+// carry Y = OR over [j0 + 128, i]; above it into the row's carry
+// Z = OR over (i, j0] and PRE[c]. The carries of a query tile's rows form a
+// chain of nested sets, so a tile has few distinct carries; the mask warp
+// writes one row of log2 weights per distinct carry (indexed by its
+// popcount) and each softmax thread reads its row: one shared load and one
+// FMA per key. On the diagonal tile (and for 64-bit masks everywhere) a row
+// scans its keys away from itself with a running OR instead, recomputing
+// log2(s - popcount) only where some hash opens a block.
+// The reference maximum m moves only when a tile's maximum exceeds it by
+// more than 8 (then O and the row sum are rescaled), so every P <= 256.
 //
 // Every barrier wait is bounded in time (PLSH_DEVERR_TIMEOUT); on timeout all
 // roles leave their loops, in-flight copies and MMAs are drained and TMEM is
 // freed before the CTA returns.
 #include <cmath>
+#include <type_traits>
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -51,22 +61,39 @@ using namespace sm100;
 
 constexpr int kTile = PLSH_TILE;
 constexpr int kD = 128;
-constexpr int kThreads = 256;
+constexpr int kThreads = 352;         // 11 warps
+constexpr int kSoftmaxWarps = 8;      // warps 0-7
+constexpr int kWarpTma = 8, kWarpMma = 9, kWarpMask = 10;
+constexpr int kHalf = 64;             // key columns per softmax thread
 constexpr int kStages = 2;
 constexpr int kChunkBytes = kTile * 64 * 2;         // 128 rows x 64 bf16 = 16 KB (one SW128 box)
 constexpr int kTileBytes = 2 * kChunkBytes;         // 128 x 128 bf16 = 32 KB
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;      // S buffers at columns 0 and 128
-constexpr uint32_t kColO = 256;    // O accumulator, 128 fp32 columns
-constexpr uint32_t kColP = 384;    // P buffers at 384 and 448 (bf16 pairs)
+constexpr uint32_t kColS = 0;      // S buffers at columns 0 and 128 (P overwrites their first 64 columns)
+constexpr uint32_t kColO = 256;    // O buffers at columns 256 and 384
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kMaxSortedHeads = 256;
+constexpr int kTblRows = 33;       // table rows: popcounts 0..32
+constexpr int kTblStride = 132;    // floats per table row (spreads rows over banks)
 
 template <typename MaskT>
 struct alignas(16) MaskStage {
-  MaskT bm[kTile + 4];   // bm[c]  = boundary mask of key j0 + c, c = 0..128 (all ones outside [0, n))
-  MaskT bmn[kTile];      // bmn[c] = bm[c + 1]
+  MaskT bm[kTile + 4];   // bm[c]   = boundary mask of key j0 + c, c = 0..128 (all ones outside [0, n))
+  MaskT bmn[kTile];      // bmn[c]  = bm[c + 1]
+  MaskT pre[kTile];      // pre[c]  = OR bm[1 .. c]        (pre[0] = 0)
+  MaskT suf[kTile];      // suf[c]  = OR bm[c + 1 .. 127]  (suf[127] = 0)
+  MaskT preh[kHalf];     // preh[q] = OR bm[64 .. 64 + q]
+  MaskT sufl[kHalf];     // sufl[c] = OR bm[c + 1 .. 63]   (sufl[63] = 0)
 };
+
+// Log2-weight table of one key tile (32-bit masks only).
+struct alignas(16) WeightTable {
+  float w[kTblRows][kTblStride];
+};
+struct NoTable {};
+
+template <typename MaskT>
+constexpr bool kUseTable = sizeof(MaskT) == 4;
 
 template <typename MaskT>
 struct __align__(1024) TcSmem {
@@ -74,6 +101,12 @@ struct __align__(1024) TcSmem {
   uint8_t k[kStages][kTileBytes];
   uint8_t v[kStages][kTileBytes];
   MaskStage<MaskT> m[kStages];
+  typename std::conditional<kUseTable<MaskT>, WeightTable, NoTable>::type tbl;
+  MaskT pfxq[kTile];                   // mask warp: OR over [i0, i0 + r] of the current item
+  MaskT sfxq[kTile];                   // mask warp: OR over (i0 + r, i0 + 127]
+  MaskT ykey[kTblRows + 3];            // mask warp: carry set of each popcount present
+  float pmax[2][2][kTile];             // [tile parity][half][row] partial row maxima
+  float psum[2][2][kTile];             // [item parity][half][row] partial row sums
   float lg[PLSH_MAX_S + 4];            // lg[w] = log2(w), lg[0] = -inf
   int16_t order[kMaxSortedHeads];      // heads by decreasing window width
   int32_t width[kMaxSortedHeads];
@@ -81,7 +114,9 @@ struct __align__(1024) TcSmem {
   uint64_t k_full[kStages], k_empty[kStages];
   uint64_t v_full[kStages], v_empty[kStages];
   uint64_t m_full[kStages], m_empty[kStages];
+  uint64_t t_full, t_empty;            // weight table handoff
   uint64_t s_full[2], p_full[2], pv_done[2];
+  uint64_t xmax[2], xsum[2];           // softmax half exchange: row maxima per tile, row sums per item
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -92,31 +127,45 @@ struct Params {
   const int32_t* spans;
 };
 
-// One key tile of one work item, in the order every role walks them.
+// One key tile of one work item, in the order every role walks them. The
+// window of the next item is fetched one item ahead.
 struct TileIter {
   const Params* p;
   const int16_t* order;
   int x;        // work item index
-  int k;        // work items started by this CTA so far (Q buffer = k & 1)
+  int k;        // work items started by this CTA so far (Q and O buffer = k & 1)
   int it;       // key tile within the item
   int total;    // key tiles of the item
   int n_below;
   int b, h, t, i0;
   int g;        // key tile counted across this CTA's items
+  int u;        // table tiles (below / above the diagonal) counted across this CTA's items
   bool valid;
   bool bad_window;  // the window read for this item was out of range (and was clamped)
+  int nx_lo, nx_hi; // window of item x + gridDim.x
 
-  __device__ __forceinline__ void load_item() {
+  __device__ __forceinline__ int head_of(int xx) const {
+    const int hr = xx / (p->B * p->T);
+    return (p->H <= kMaxSortedHeads) ? static_cast<int>(order[hr]) : hr;
+  }
+  __device__ __forceinline__ void fetch(int xx, int& lo, int& hi) const {
+    if (xx < p->items) {
+      const int hh = head_of(xx);
+      const int tt = (xx - (xx / (p->B * p->T)) * (p->B * p->T)) % p->T;
+      lo = p->spans[(static_cast<size_t>(hh) * p->T + tt) * 2];
+      hi = p->spans[(static_cast<size_t>(hh) * p->T + tt) * 2 + 1];
+    }
+  }
+  __device__ __forceinline__ void load_item(int lo, int hi) {
     valid = x < p->items;
     if (!valid) return;
     const int BT = p->B * p->T;
-    const int hr = x / BT, rem = x - hr * BT;
-    h = (p->H <= kMaxSortedHeads) ? static_cast<int>(order[hr]) : hr;
+    const int rem = x - (x / BT) * BT;
+    h = head_of(x);
     b = rem / p->T;
     t = rem - b * p->T;
     i0 = t * kTile;
-    int lo = p->spans[(static_cast<size_t>(h) * p->T + t) * 2];
-    int hi = p->spans[(static_cast<size_t>(h) * p->T + t) * 2 + 1];
+    fetch(x + gridDim.x, nx_lo, nx_hi);
     const int last_row = min(p->n, i0 + kTile) - 1;
     bad_window = lo < 0 || lo > i0 || hi >= p->n || hi < last_row;
     lo = max(0, min(lo, i0));
@@ -131,14 +180,19 @@ struct TileIter {
     x = blockIdx.x;
     k = 0;
     g = 0;
-    load_item();
+    u = 0;
+    nx_lo = nx_hi = 0;
+    int lo = 0, hi = 0;
+    fetch(x, lo, hi);
+    load_item(lo, hi);
   }
   __device__ __forceinline__ void next() {
     ++g;
+    if (it > 0) ++u;
     if (++it >= total) {
       x += gridDim.x;
       ++k;
-      load_item();
+      load_item(nx_lo, nx_hi);
     }
   }
   __device__ __forceinline__ int kind() const { return it == 0 ? 0 : (it <= n_below ? 1 : 2); }
@@ -168,26 +222,63 @@ __device__ __forceinline__ void load4(const MaskT* p, MaskT (&b)[4]) {
   }
 }
 
-// Logits of one key tile for one row: x[c] <- S[c] * sc + log2(c_ij), with the running OR carried in/out.
-// kind 0: diagonal tile (row r = column r); kind 1: below the diagonal; kind 2: above.
-template <typename MaskT, bool kCausal>
-__device__ __forceinline__ void tile_logits(float (&x)[kTile], const MaskStage<MaskT>& ms, const float* lg, int kind,
-                                            int r, int s, float sc, MaskT& Y, MaskT& Z) {
-  constexpr bool causal = kCausal;
-  if (kind == 1) {
-    // R(127) = Y; R(c) = R(c + 1) | bm[c + 1]
-    MaskT R = Y;
-    float lw = lg[max(0, s - popc_m(R))];
+template <typename MaskT>
+__device__ __forceinline__ MaskT warp_prefix_or(MaskT v, int lane) {   // inclusive over lanes 0..lane
 #pragma unroll
-    for (int g4 = kTile / 4 - 1; g4 >= 0; --g4) {
+  for (int o = 1; o < 32; o <<= 1) {
+    const MaskT y = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v |= y;
+  }
+  return v;
+}
+
+template <typename MaskT>
+__device__ __forceinline__ MaskT warp_suffix_or(MaskT v, int lane) {   // inclusive over lanes lane..31
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const MaskT y = __shfl_down_sync(0xffffffffu, v, o);
+    if (lane + o < 32) v |= y;
+  }
+  return v;
+}
+
+__device__ __forceinline__ int lg_index(int s, int popcount) { return max(0, s - popcount); }
+
+// x[cc] <- x[cc] * sc + table row, for the 64 columns of this half (loads issued four at a time
+// so that at most 16 table values are live next to the 64 logits).
+__device__ __forceinline__ void logits_from_table(float (&x)[kHalf], const float* row, float sc) {
+#pragma unroll
+  for (int g4 = 0; g4 < kHalf / 4; ++g4) {
+    if ((g4 & 3) == 0) asm volatile("" ::: "memory");
+    const float4 t4 = reinterpret_cast<const float4*>(row)[g4];
+    x[4 * g4 + 0] = fmaf(x[4 * g4 + 0], sc, t4.x);
+    x[4 * g4 + 1] = fmaf(x[4 * g4 + 1], sc, t4.y);
+    x[4 * g4 + 2] = fmaf(x[4 * g4 + 2], sc, t4.z);
+    x[4 * g4 + 3] = fmaf(x[4 * g4 + 3], sc, t4.w);
+  }
+}
+
+// Scans for one row's half of a key tile: x[cc] <- S[c] * sc + log2(c_ij) for c = 64*half + cc.
+// kind 0: diagonal tile (row r is column r); kind 1: below the diagonal; kind 2: above.
+// R is the OR over the gap between the row and the current key, carried in from Y / Z.
+template <typename MaskT, bool kCausal>
+__device__ __forceinline__ void logits_by_scan(float (&x)[kHalf], const MaskStage<MaskT>& ms, const float* lg,
+                                               int kind, int r, int half, int s, float sc, MaskT Y, MaskT Z) {
+  const int c0 = kHalf * half;
+  if (kind == 1) {
+    // R(127) = Y, R(63) = Y | OR bm[64..127], R(c) = R(c + 1) | bm[c + 1]
+    MaskT R = half ? Y : static_cast<MaskT>(Y | ms.suf[kHalf - 1]);
+    float lw = lg[lg_index(s, popc_m(R))];
+#pragma unroll
+    for (int g4 = kHalf / 4 - 1; g4 >= 0; --g4) {
       MaskT bb[4];
-      load4(&ms.bmn[4 * g4], bb);
-      if (g4 == kTile / 4 - 1) bb[3] = 0;
+      load4(&ms.bmn[c0 + 4 * g4], bb);
+      if (g4 == kHalf / 4 - 1 && half) bb[3] = 0;
       if ((bb[0] | bb[1] | bb[2] | bb[3]) != 0) {
 #pragma unroll
         for (int e = 3; e >= 0; --e) {
           R |= bb[e];
-          lw = lg[max(0, s - popc_m(R))];
+          lw = lg[lg_index(s, popc_m(R))];
           x[4 * g4 + e] = fmaf(x[4 * g4 + e], sc, lw);
         }
       } else {
@@ -195,21 +286,20 @@ __device__ __forceinline__ void tile_logits(float (&x)[kTile], const MaskStage<M
         for (int e = 3; e >= 0; --e) x[4 * g4 + e] = fmaf(x[4 * g4 + e], sc, lw);
       }
     }
-    Y = R | ms.bm[0];   // OR over [j0, i]
   } else if (!kCausal && kind == 2) {
-    // R(0) = Z (already holds bm[0]); R(c) = R(c - 1) | bm[c]
-    MaskT R = Z;
-    float lw = lg[max(0, s - popc_m(R))];
+    // R(0) = Z (holds bm[0]), R(63) = Z | OR bm[1..63], R(c) = R(c - 1) | bm[c]
+    MaskT R = half ? static_cast<MaskT>(Z | ms.pre[kHalf - 1]) : Z;
+    float lw = lg[lg_index(s, popc_m(R))];
 #pragma unroll
-    for (int g4 = 0; g4 < kTile / 4; ++g4) {
+    for (int g4 = 0; g4 < kHalf / 4; ++g4) {
       MaskT bb[4];
-      load4(&ms.bm[4 * g4], bb);
-      if (g4 == 0) bb[0] = 0;
+      load4(&ms.bm[c0 + 4 * g4], bb);
+      if (g4 == 0 && !half) bb[0] = 0;
       if ((bb[0] | bb[1] | bb[2] | bb[3]) != 0) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           R |= bb[e];
-          lw = lg[max(0, s - popc_m(R))];
+          lw = lg[lg_index(s, popc_m(R))];
           x[4 * g4 + e] = fmaf(x[4 * g4 + e], sc, lw);
         }
       } else {
@@ -217,67 +307,66 @@ __device__ __forceinline__ void tile_logits(float (&x)[kTile], const MaskStage<M
         for (int e = 0; e < 4; ++e) x[4 * g4 + e] = fmaf(x[4 * g4 + e], sc, lw);
       }
     }
-    Z = R;              // OR over (i, j0 + 127]
   } else {
-    // columns c <= r: R(r) = 0; R(c) = R(c + 1) | bm[c + 1] for c < r
-    MaskT R = 0;
-    float lw = lg[s];
+    // columns c <= r: R(c) = OR bm[c+1 .. r]; in the low half a row r >= 64 starts from OR bm[64..r]
+    MaskT R = (!half && r >= kHalf) ? ms.preh[r - kHalf] : static_cast<MaskT>(0);
+    float lw = lg[lg_index(s, popc_m(R))];
 #pragma unroll
-    for (int g4 = kTile / 4 - 1; g4 >= 0; --g4) {
+    for (int g4 = kHalf / 4 - 1; g4 >= 0; --g4) {
       MaskT bb[4];
-      load4(&ms.bmn[4 * g4], bb);
+      load4(&ms.bmn[c0 + 4 * g4], bb);
       if ((bb[0] | bb[1] | bb[2] | bb[3]) != 0) {
 #pragma unroll
         for (int e = 3; e >= 0; --e) {
-          const int c = 4 * g4 + e;
+          const int cc = 4 * g4 + e, c = c0 + cc;
           if (c < r) R |= bb[e];
-          lw = lg[max(0, s - popc_m(R))];
-          x[c] = (c <= r) ? fmaf(x[c], sc, lw) : (causal ? -INFINITY : x[c]);
+          lw = lg[lg_index(s, popc_m(R))];
+          x[cc] = (c <= r) ? fmaf(x[cc], sc, lw) : (kCausal ? -INFINITY : x[cc]);
         }
       } else {
 #pragma unroll
         for (int e = 3; e >= 0; --e) {
-          const int c = 4 * g4 + e;
-          x[c] = (c <= r) ? fmaf(x[c], sc, lw) : (causal ? -INFINITY : x[c]);
+          const int cc = 4 * g4 + e, c = c0 + cc;
+          x[cc] = (c <= r) ? fmaf(x[cc], sc, lw) : (kCausal ? -INFINITY : x[cc]);
         }
       }
     }
-    Y = R | ms.bm[0];   // OR over [i0, i]
-    MaskT R2 = 0;
-    if (!causal) {
-      // columns c > r: R(r) = 0; R(c) = R(c - 1) | bm[c]
-      float lw2 = lg[s];
+    if (!kCausal) {
+      // columns c > r: R(c) = OR bm[r+1 .. c]; in the high half a row r < 64 starts from OR bm[r+1..63]
+      MaskT R2 = (half && r < kHalf) ? ms.sufl[r] : static_cast<MaskT>(0);
+      float lw2 = lg[lg_index(s, popc_m(R2))];
 #pragma unroll
-      for (int g4 = 0; g4 < kTile / 4; ++g4) {
+      for (int g4 = 0; g4 < kHalf / 4; ++g4) {
         MaskT bb[4];
-        load4(&ms.bm[4 * g4], bb);
+        load4(&ms.bm[c0 + 4 * g4], bb);
         if ((bb[0] | bb[1] | bb[2] | bb[3]) != 0) {
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int c = 4 * g4 + e;
+            const int cc = 4 * g4 + e, c = c0 + cc;
             if (c > r) R2 |= bb[e];
-            lw2 = lg[max(0, s - popc_m(R2))];
-            if (c > r) x[c] = fmaf(x[c], sc, lw2);
+            lw2 = lg[lg_index(s, popc_m(R2))];
+            if (c > r) x[cc] = fmaf(x[cc], sc, lw2);
           }
         } else {
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int c = 4 * g4 + e;
-            if (c > r) x[c] = fmaf(x[c], sc, lw2);
+            const int cc = 4 * g4 + e, c = c0 + cc;
+            if (c > r) x[cc] = fmaf(x[cc], sc, lw2);
           }
         }
       }
     }
-    Z = R2;             // OR over (i, i0 + 127]
   }
 }
 
 template <typename MaskT, bool kCausal>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
-               const __grid_constant__ CUtensorMap tmap_v, Params prm, const double* __restrict__ sigma,
+               const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ Params prm,
+               const double* __restrict__ sigma,
                const double* __restrict__ table, const MaskT* __restrict__ bmask, __nv_bfloat16* __restrict__ O,
                float* __restrict__ row_sum, uint32_t* __restrict__ err) {
+  constexpr bool kTable = kUseTable<MaskT>;
   extern __shared__ uint8_t smem_raw[];
   auto& sm = *reinterpret_cast<TcSmem<MaskT>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   volatile int* abort_flag = &sm.abort_flag;
@@ -306,6 +395,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       sm.width[h] = prm.spans[(static_cast<size_t>(h) * prm.T + tm) * 2 + 1] -
                     prm.spans[(static_cast<size_t>(h) * prm.T + tm) * 2];
   }
+  if (threadIdx.x < PLSH_MAX_S + 4)
+    sm.lg[threadIdx.x] = threadIdx.x == 0 ? -INFINITY : log2f(static_cast<float>(threadIdx.x));
   __syncthreads();
   if (H <= kMaxSortedHeads) {
     for (int h = threadIdx.x; h < H; h += kThreads) {
@@ -324,8 +415,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       mbar_init(&sm.q_full[i], 1);
       mbar_init(&sm.q_empty[i], 1);
       mbar_init(&sm.s_full[i], 1);
-      mbar_init(&sm.p_full[i], 4);
+      mbar_init(&sm.p_full[i], kSoftmaxWarps);
       mbar_init(&sm.pv_done[i], 1);
+      mbar_init(&sm.xmax[i], kSoftmaxWarps);
+      mbar_init(&sm.xsum[i], kSoftmaxWarps);
     }
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&sm.k_full[i], 1);
@@ -333,13 +426,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       mbar_init(&sm.v_full[i], 1);
       mbar_init(&sm.v_empty[i], 1);
       mbar_init(&sm.m_full[i], 1);
-      mbar_init(&sm.m_empty[i], 4);
+      mbar_init(&sm.m_empty[i], kSoftmaxWarps);
     }
+    mbar_init(&sm.t_full, 1);
+    mbar_init(&sm.t_empty, kSoftmaxWarps);
     mbar_init(&sm.drain, 1);
     fence_mbarrier_init();
   }
-  if (threadIdx.x < PLSH_MAX_S + 4) sm.lg[threadIdx.x] = threadIdx.x == 0 ? -INFINITY : log2f(static_cast<float>(threadIdx.x));
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     tmem_alloc(&sm.tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -348,7 +442,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
-  if (warp == 0) {
+  if (warp == kWarpTma) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tmap_q);
@@ -396,7 +490,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0);
@@ -427,35 +521,40 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         if (!mbar_wait(&sm.v_full[st], static_cast<uint32_t>(ti.g / kStages) & 1u, abort_flag, err)) return false;
         tc_fence_after();
         const uint32_t v_addr = smem_u32(sm.v[st]);
-        const uint32_t p_tmem = tmem + kColP + 64u * static_cast<uint32_t>(ti.g & 1);
+        const uint32_t p_tmem = tmem + kColS + 128u * static_cast<uint32_t>(ti.g & 1);
+        const uint32_t o_tmem = tmem + kColO + 128u * static_cast<uint32_t>(ti.k & 1);
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk) {
           // 16 keys = two 8-row groups of the MN-major V tile; the two d halves sit kChunkBytes apart
-          mma_ts(tmem + kColO, p_tmem + 8u * kk, smem_desc_sw128(v_addr + kk * 2048, kChunkBytes, 1024), idesc_pv,
+          mma_ts(o_tmem, p_tmem + 8u * kk, smem_desc_sw128(v_addr + kk * 2048, kChunkBytes, 1024), idesc_pv,
                  (ti.it > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(&sm.pv_done[ti.g & 1]);
         mma_commit(&sm.v_empty[st]);
         return true;
       };
+      // `nxt` runs one tile ahead of `cur`: S of the next tile is issued before PV of the current one
       TileIter cur, nxt;
       cur.start(&prm, sm.order);
+      nxt.start(&prm, sm.order);
       bool ok = !cur.valid || issue_s(cur);
+      if (nxt.valid) nxt.next();
       while (ok && cur.valid) {
-        nxt = cur;
-        nxt.next();
         if (nxt.valid) ok = issue_s(nxt);
         if (ok) ok = issue_pv(cur);
-        cur = nxt;
+        cur.next();
+        if (nxt.valid) nxt.next();
       }
       // every MMA issued so far completes before `drain` arrives
       mma_commit(&sm.drain);
       mbar_wait_drain(&sm.drain, 0, 100000000ull);
     }
-  } else if (warp == 2) {
-    // ------------------------------------------------------------ mask producer
+  } else if (warp == kWarpMask) {
+    // ------------------------------------------------------------ mask warp
     TileIter ti;
     ti.start(&prm, sm.order);
+    MaskT mid_b = 0;   // below the diagonal: OR over [j0 + 128, i0)
+    MaskT mid_a = 0;   // above the diagonal: OR over [i0 + 128, j0]
     while (ti.valid) {
       const int st = ti.g % kStages;
       if (ti.g >= kStages &&
@@ -464,71 +563,251 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       const MaskT* bm_h = bmask + static_cast<size_t>(ti.h) * n;
       MaskStage<MaskT>& ms = sm.m[st];
       const int j0 = ti.j0();
+      const int kind = ti.kind();
+      MaskT xv[4];
 #pragma unroll
-      for (int e = 0; e < 5; ++e) {
-        const int c = lane + 32 * e;
-        if (c <= kTile) {
-          const int j = j0 + c;
-          const MaskT v = (j >= 0 && j < n) ? bm_h[j] : FULL;
-          ms.bm[c] = v;
-          if (c >= 1) ms.bmn[c - 1] = v;
+      for (int e = 0; e < 4; ++e) {
+        const int c = 4 * lane + e, j = j0 + c;
+        xv[e] = (j >= 0 && j < n) ? bm_h[j] : FULL;
+        ms.bm[c] = xv[e];
+        if (c >= 1) ms.bmn[c - 1] = xv[e];
+      }
+      if (lane == 0) {
+        const int j = j0 + kTile;
+        const MaskT v = (j >= 0 && j < n) ? bm_h[j] : FULL;
+        ms.bm[kTile] = v;
+        ms.bmn[kTile - 1] = v;
+      }
+      MaskT pre_v[4], suf_v[4];
+      {  // pre[c] = OR bm[1..c]
+        const MaskT p0 = lane == 0 ? static_cast<MaskT>(0) : xv[0];
+        const MaskT p1 = p0 | xv[1], p2 = p1 | xv[2], p3 = p2 | xv[3];
+        MaskT before = __shfl_up_sync(0xffffffffu, warp_prefix_or<MaskT>(p3, lane), 1);
+        if (lane == 0) before = 0;
+        pre_v[0] = before | p0; pre_v[1] = before | p1; pre_v[2] = before | p2; pre_v[3] = before | p3;
+      }
+      {  // suf[c] = OR bm[c+1..127]
+        const MaskT u2 = xv[3], u1 = u2 | xv[2], u0 = u1 | xv[1];
+        MaskT after = __shfl_down_sync(0xffffffffu, warp_suffix_or<MaskT>(u0 | xv[0], lane), 1);
+        if (lane == 31) after = 0;
+        suf_v[0] = after | u0; suf_v[1] = after | u1; suf_v[2] = after | u2; suf_v[3] = after;
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        ms.pre[4 * lane + e] = pre_v[e];
+        ms.suf[4 * lane + e] = suf_v[e];
+      }
+      {  // preh[q] = OR bm[64..64+q] (lanes 16..31 hold columns 64..127)
+        const bool hiL = lane >= 16;
+        const MaskT h0 = xv[0], h1 = h0 | xv[1], h2 = h1 | xv[2], h3 = h2 | xv[3];
+        MaskT before = __shfl_up_sync(0xffffffffu, warp_prefix_or<MaskT>(hiL ? h3 : static_cast<MaskT>(0), lane), 1);
+        if (lane <= 16) before = 0;
+        if (hiL) {
+          const int q = 4 * (lane - 16);
+          ms.preh[q + 0] = before | h0;
+          ms.preh[q + 1] = before | h1;
+          ms.preh[q + 2] = before | h2;
+          ms.preh[q + 3] = before | h3;
+        }
+      }
+      {  // sufl[c] = OR bm[c+1..63] (lanes 0..15 hold columns 0..63)
+        const bool loL = lane < 16;
+        const MaskT u2 = xv[3], u1 = u2 | xv[2], u0 = u1 | xv[1];
+        MaskT after = __shfl_down_sync(0xffffffffu, warp_suffix_or<MaskT>(loL ? static_cast<MaskT>(u0 | xv[0])
+                                                                              : static_cast<MaskT>(0), lane), 1);
+        if (lane >= 15) after = 0;
+        if (loL) {
+          ms.sufl[4 * lane + 0] = after | u0;
+          ms.sufl[4 * lane + 1] = after | u1;
+          ms.sufl[4 * lane + 2] = after | u2;
+          ms.sufl[4 * lane + 3] = after;
+        }
+      }
+      if constexpr (kTable) {
+        if (kind == 0) {
+          // the query tile's own prefix / suffix ORs, for this item's table tiles
+          const MaskT bm0 = __shfl_sync(0xffffffffu, xv[0], 0);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            sm.pfxq[4 * lane + e] = static_cast<MaskT>(bm0 | pre_v[e]);
+            sm.sfxq[4 * lane + e] = suf_v[e];
+          }
+          mid_b = 0;
+          mid_a = 0;
+        } else {
+          // the distinct carries of the tile's rows, then one table row per distinct carry
+          const MaskT bm0 = __shfl_sync(0xffffffffu, xv[0], 0);
+          if (kind == 2) mid_a |= bm0;
+          const MaskT mid = kind == 1 ? mid_b : mid_a;
+          __syncwarp();
+          uint32_t pres_lo = 0, pres_hi = 0;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int r = lane + 32 * e;
+            const MaskT cy = static_cast<MaskT>(mid | (kind == 1 ? sm.pfxq[r] : sm.sfxq[r]));
+            const int key = popc_m(cy);
+            if (key < 32) pres_lo |= 1u << key; else pres_hi |= 1u << (key - 32);
+          }
+          pres_lo = __reduce_or_sync(0xffffffffu, pres_lo);
+          pres_hi = __reduce_or_sync(0xffffffffu, pres_hi);
+          bool ok = true;
+          if (ti.u >= 1) ok = mbar_wait(&sm.t_empty, static_cast<uint32_t>((ti.u - 1) & 1), abort_flag, err);
+          if (!__all_sync(0xffffffffu, ok)) break;
+          // rows with the same popcount hold the same carry (the carries of a tile are nested)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int r = lane + 32 * e;
+            const MaskT cy = static_cast<MaskT>(mid | (kind == 1 ? sm.pfxq[r] : sm.sfxq[r]));
+            sm.ykey[popc_m(cy)] = cy;
+          }
+          __syncwarp();
+          for (int key = 0; key < kTblRows; ++key) {
+            const bool present = key < 32 ? ((pres_lo >> key) & 1u) : ((pres_hi >> (key - 32)) & 1u);
+            if (!present) continue;
+            const MaskT cy = sm.ykey[key];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int c = lane + 32 * e;
+              const MaskT Rc = kind == 1 ? static_cast<MaskT>(ms.suf[c] | cy) : static_cast<MaskT>(cy | ms.pre[c]);
+              sm.tbl.w[key][c] = sm.lg[lg_index(s, popc_m(Rc))];
+            }
+          }
+          if (kind == 1) mid_b |= static_cast<MaskT>(bm0 | __shfl_sync(0xffffffffu, suf_v[0], 0));
+          else mid_a |= __shfl_sync(0xffffffffu, pre_v[3], 31);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.t_full);
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.m_full[st]);
       ti.next();
     }
-  } else if (warp >= 4) {
+  } else if (warp < kSoftmaxWarps) {
     // ------------------------------------------------------------ softmax
-    const int quarter = warp - 4;
+    const int half = warp >= 4 ? 1 : 0;
+    const int quarter = warp & 3;
     const int r = quarter * 32 + lane;   // row within the tile == TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t col_off = static_cast<uint32_t>(kHalf * half);
     const float sc = 1.4426950408889634f / sqrtf(static_cast<float>(kD));
     float m2 = -INFINITY, l = 0.0f;
     MaskT Y = 0, Z = 0;
+    // epilogue still owed for the previous item
+    // (always the item just before the current tile's item: index x - gridDim.x, tile g - 1, count k - 1)
+    bool pend = false;
+    float pend_l = 0.0f, pend_m = 0.0f;
+    auto epilogue = [&](int pend_x, int pend_g, int pend_k) -> bool {
+      const int BT = prm.B * prm.T;
+      const int pend_h = (H <= kMaxSortedHeads) ? static_cast<int>(sm.order[pend_x / BT]) : pend_x / BT;
+      const int rem = pend_x % BT;
+      const int pend_b = rem / prm.T;
+      const int pend_i0 = (rem % prm.T) * kTile;
+      bool okw = mbar_wait(&sm.pv_done[pend_g & 1], static_cast<uint32_t>(pend_g >> 1) & 1u, abort_flag, err);
+      okw = __all_sync(0xffffffffu, okw && mbar_wait(&sm.xsum[pend_k & 1], static_cast<uint32_t>(pend_k >> 1) & 1u,
+                                                     abort_flag, err));
+      if (!okw) return false;
+      tc_fence_after();
+      const float ltot = pend_l + sm.psum[pend_k & 1][half ^ 1][r];
+      const int i = pend_i0 + r;
+      const float inv = 1.0f / ltot;
+      const uint32_t ob = tmem + lane_off + kColO + 128u * static_cast<uint32_t>(pend_k & 1) + col_off;
+      __nv_bfloat16* orow = O + ((static_cast<size_t>(pend_b) * H + pend_h) * n + (i < n ? i : 0)) * kD + col_off;
+#pragma unroll 1
+      for (int q2 = 0; q2 < 2; ++q2) {
+        uint32_t raw[32];
+        tmem_ld32(ob + 32u * q2, raw);
+        tmem_wait_ld();
+        if (i < n) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * q2);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              pk[u] = pack_bf16x2(__uint_as_float(raw[8 * e + 2 * u]) * inv, __uint_as_float(raw[8 * e + 2 * u + 1]) * inv);
+            dst[e] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+        }
+      }
+      tc_fence_before();
+      if (i < n) {
+        if (half == 0)
+          row_sum[(static_cast<size_t>(pend_b) * H + pend_h) * n + i] =
+              (log2f(ltot) + pend_m) * 0.6931471805599453f - logf(static_cast<float>(s));
+      }
+      pend = false;
+      return true;
+    };
     TileIter ti;
     ti.start(&prm, sm.order);
     bool ok = true;
     while (ti.valid) {
       const int g = ti.g;
       const int st = g % kStages;
+      const int kind = ti.kind();
       if (ti.first()) {
         m2 = -INFINITY;
         l = 0.0f;
-        if (ti.bad_window && r == 0) atomicOr(err, PLSH_DEVERR_WINDOW);
+        if (ti.bad_window && r == 0 && half == 0) atomicOr(err, PLSH_DEVERR_WINDOW);
       }
       ok = mbar_wait(&sm.m_full[st], static_cast<uint32_t>(g / kStages) & 1u, abort_flag, err);
-      ok = __all_sync(0xffffffffu, ok && mbar_wait(&sm.s_full[g & 1], static_cast<uint32_t>(g >> 1) & 1u,
-                                                   abort_flag, err));
+      ok = ok && mbar_wait(&sm.s_full[g & 1], static_cast<uint32_t>(g >> 1) & 1u, abort_flag, err);
+      if (kTable && kind != 0) ok = ok && mbar_wait(&sm.t_full, static_cast<uint32_t>(ti.u & 1), abort_flag, err);
+      ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      float x[kTile];
+      float x[kHalf];
       {
-        const uint32_t base = tmem + lane_off + kColS + 128u * static_cast<uint32_t>(g & 1);
-        uint32_t raw[4][32];
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(base + 32u * q4, raw[q4]);
+        const uint32_t base = tmem + lane_off + kColS + 128u * static_cast<uint32_t>(g & 1) + col_off;
+        uint32_t raw[2][32];
+        tmem_ld32(base, raw[0]);
+        tmem_ld32(base + 32u, raw[1]);
         tmem_wait_ld();
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4)
-#pragma unroll
-          for (int e = 0; e < 32; ++e) x[32 * q4 + e] = __uint_as_float(raw[q4][e]);
+        for (int e = 0; e < 32; ++e) {
+          x[e] = __uint_as_float(raw[0][e]);
+          x[32 + e] = __uint_as_float(raw[1][e]);
+        }
       }
       const MaskStage<MaskT>& ms = sm.m[st];
-      const int kind = ti.kind();
       if (kind == 2) Z |= ms.bm[0];   // now OR over (i, j0]
-      tile_logits<MaskT, kCausal>(x, ms, sm.lg, kind, r, s, sc, Y, Z);
+      if constexpr (kTable) {
+        if (kind != 0) {
+          const MaskT cy = kind == 1 ? Y : Z;
+          logits_from_table(x, &sm.tbl.w[popc_m(cy)][col_off], sc);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.t_empty);
+        } else {
+          logits_by_scan<MaskT, kCausal>(x, ms, sm.lg, kind, r, half, s, sc, Y, Z);
+        }
+      } else {
+        logits_by_scan<MaskT, kCausal>(x, ms, sm.lg, kind, r, half, s, sc, Y, Z);
+      }
+      // carries past this tile
+      if (kind == 0) {
+        Y = static_cast<MaskT>(ms.bm[0] | ms.pre[r]);       // OR over [i0, i]
+        Z = kCausal ? static_cast<MaskT>(0) : ms.suf[r];     // OR over (i, i0 + 127]
+      } else if (kind == 1) {
+        Y = static_cast<MaskT>(Y | ms.bm[0] | ms.suf[0]);   // OR over [j0, i]
+      } else {
+        Z = static_cast<MaskT>(Z | ms.pre[kTile - 1]);      // OR over (i, j0 + 127]
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.m_empty[st]);
 
-      // ---- tile maximum and reference update
+      // ---- tile maximum (both halves) and reference update
       float mx[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) mx[u] = x[u];
 #pragma unroll
-      for (int c = 8; c < kTile; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
-      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      for (int c = 8; c < kHalf; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
+      float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      sm.pmax[g & 1][half][r] = mt;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.xmax[g & 1]);
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.xmax[g & 1], static_cast<uint32_t>(g >> 1) & 1u, abort_flag, err));
+      if (!ok) break;
+      mt = fmaxf(mt, sm.pmax[g & 1][half ^ 1][r]);
       float alpha = 1.0f;
       bool need_rescale = false;
       if (mt > m2 + kRescaleThreshold) {
@@ -540,48 +819,42 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       }
       const float neg_m = (m2 == -INFINITY) ? 0.0f : -m2;
 
-      // ---- P buffer g&1 must be free: PV of tile g-2 done
-      if (g >= 2) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&sm.pv_done[g & 1], static_cast<uint32_t>((g - 2) >> 1) & 1u,
-                                               abort_flag, err));
-        if (!ok) break;
-      }
-      // ---- rescale O when some row of the warp moved its reference (never on an item's first tile)
+      // ---- rescale this half of the item's O when some row of the warp moved its reference
       if (__any_sync(0xffffffffu, need_rescale)) {
         ok = __all_sync(0xffffffffu, mbar_wait(&sm.pv_done[(g - 1) & 1], static_cast<uint32_t>((g - 1) >> 1) & 1u,
                                                abort_flag, err));
         if (!ok) break;
         tc_fence_after();
-        uint32_t raw[32];
-#pragma unroll
+#pragma unroll 1
         for (int q4 = 0; q4 < 4; ++q4) {
-          const uint32_t addr = tmem + lane_off + kColO + 32u * q4;
-          tmem_ld32(addr, raw);
+          uint32_t raw[16];
+          const uint32_t addr = tmem + lane_off + kColO + 128u * static_cast<uint32_t>(ti.k & 1) + col_off + 16u * q4;
+          tmem_ld16(addr, raw);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * alpha);
-          tmem_st32(addr, raw);
+          for (int e = 0; e < 16; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * alpha);
+          tmem_st16(addr, raw);
         }
         tmem_wait_st();
       }
 
-      // ---- P = 2^(x - m) as bf16 into TMEM, row sum
-      const uint32_t p_base = tmem + lane_off + kColP + 64u * static_cast<uint32_t>(g & 1);
+      // ---- P = 2^(x - m) as bf16 over the first 64 columns of S_g, partial row sum
+      const uint32_t p_base = tmem + lane_off + kColS + 128u * static_cast<uint32_t>(g & 1) + col_off / 2;
       float ls[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) ls[u] = 0.0f;
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
+      for (int q2 = 0; q2 < 2; ++q2) {
         uint32_t packed[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const float p0 = ex2_approx(x[32 * q4 + e] + neg_m);
-          const float p1 = ex2_approx(x[32 * q4 + e + 1] + neg_m);
+          const float p0 = ex2_approx(x[32 * q2 + e] + neg_m);
+          const float p1 = ex2_approx(x[32 * q2 + e + 1] + neg_m);
           ls[e & 7] += p0;
           ls[(e + 1) & 7] += p1;
           packed[e >> 1] = pack_bf16x2(p0, p1);
         }
-        tmem_st16(p_base + 16u * q4, packed);
+        tmem_st16(p_base + 16u * q2, packed);
       }
       tmem_wait_st();
       l = l * alpha + (((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7])));
@@ -589,45 +862,28 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.p_full[g & 1]);
 
-      // ---- epilogue of the item: O / l and row_sum
+      // ---- the previous item's epilogue, now that its last PV has had a tile's time to finish
+      if (pend && !epilogue(ti.x - static_cast<int>(gridDim.x), g - 1, ti.k - 1)) {
+        ok = false;
+        break;
+      }
       if (ti.last()) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&sm.pv_done[g & 1], static_cast<uint32_t>(g >> 1) & 1u,
-                                               abort_flag, err));
-        if (!ok) break;
-        tc_fence_after();
-        const int i = ti.i0 + r;
-        const float inv = 1.0f / l;
-        __nv_bfloat16* orow = O + ((static_cast<size_t>(ti.b) * H + ti.h) * n + (i < n ? i : 0)) * kD;
-#pragma unroll 1
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint32_t raw[32];
-          tmem_ld32(tmem + lane_off + kColO + 32u * q4, raw);
-          tmem_wait_ld();
-          if (i < n) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * q4);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              uint32_t pk[4];
-#pragma unroll
-              for (int u = 0; u < 4; ++u)
-                pk[u] = pack_bf16x2(__uint_as_float(raw[8 * e + 2 * u]) * inv, __uint_as_float(raw[8 * e + 2 * u + 1]) * inv);
-              dst[e] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            }
-          }
-        }
-        tc_fence_before();
-        if (i < n) {
-          row_sum[(static_cast<size_t>(ti.b) * H + ti.h) * n + i] =
-              (log2f(l) + m2) * 0.6931471805599453f - logf(static_cast<float>(s));
-        }
+        sm.psum[ti.k & 1][half][r] = l;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.xsum[ti.k & 1]);
+        pend = true;
+        pend_l = l;
+        pend_m = m2;
       }
       ti.next();
     }
+    // the CTA's last item: ti has moved past it
+    if (ok && pend) epilogue(ti.x - static_cast<int>(gridDim.x), ti.g - 1, ti.k - 1);
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
