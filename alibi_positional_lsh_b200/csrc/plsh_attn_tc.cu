@@ -10,42 +10,46 @@
 // c_ij > 0 (Methodology 2, block-size control), and only those key tiles are
 // visited (Methodology 3: attention restricted to short random blocks).
 //
-// Persistent CTAs (one per SM) walk a static list of work items, heads with
-// the widest windows first. Warp roles (352 threads):
-//   warps 0-7    softmax: warps 0-3 own key columns 0-63 and warps 4-7 key
-//                columns 64-127 of query row (warp % 4) * 32 + lane
-//   warp 8       TMA producer: Q per item (2 buffers), K and V per key tile (2-stage rings)
-//   warp 9       TMEM owner and single-thread tcgen05.mma issuer
-//   warp 10      mask warp: the key tile's boundary masks and their in-tile
-//                prefix / suffix ORs; for 32-bit masks also the tile's table
-//                of log2 weights (below)
-// Per key tile g (counted across items): S_g = Q K_g^T (SS MMA into TMEM,
-// double-buffered); the softmax warps turn S_g into bf16 P_g written over
-// the first 64 columns of S_g; then O += P_g V_g (TS MMA, P from TMEM, fp32 O
-// in TMEM, one O buffer per item parity). S_{g+1} is issued before PV_g so
-// the tensor core works while the softmax runs. An item's epilogue (O / l)
-// runs after the next item's first tile, when its last PV has long finished.
+// Persistent CTAs (one per SM), each running two work items at a time in two
+// independent slots, so that one slot's waits are covered by the other
+// slot's work. Items come from a static list, heads with the widest windows
+// first. Warp roles (384 threads):
+//   warp 0       TMA producer for both slots: Q per item, K and V per key tile
+//   warp 1       TMEM owner and single-thread tcgen05.mma issuer for both slots
+//   warps 2, 3   mask warp of slot 0 / slot 1: the key tile's boundary masks,
+//                their in-tile prefix / suffix ORs and the tile's descriptor
+//   warps 4-7    softmax of slot 0, warps 8-11 softmax of slot 1: one query
+//                row per thread (TMEM lane = row)
+// Per key tile of a slot: S = Q K^T (SS MMA into the slot's TMEM S columns),
+// the softmax turns S into bf16 P written back over S, then O += P V (TS MMA,
+// P from TMEM, fp32 O in the slot's TMEM O columns). The MMA thread issues,
+// per slot, S(g), PV(g), S(g+1), ... as their inputs become ready.
 //
-// Weights. The logit is x = S * log2(e)/sqrt(d) + log2(c_ij) (-inf where
-// c_ij = 0), so P = 2^(x - m) = c_ij 2^(S log2(e)/sqrt(d) - m). Key tiles are
-// visited diagonal first, then downward, then upward. Below the diagonal
-// the OR over (j, i] splits into SUF[c] (inside the key tile) and the row's
-// carry Y = OR over [j0 + 128, i]; above it into the row's carry
-// Z = OR over (i, j0] and PRE[c]. The carries of a query tile's rows form a
-// chain of nested sets, so a tile has few distinct carries; the mask warp
-// writes one row of log2 weights per distinct carry (indexed by its
-// popcount) and each softmax thread reads its row: one shared load and one
-// FMA per key. On the diagonal tile (and for 64-bit masks everywhere) a row
-// scans its keys away from itself with a running OR instead, recomputing
-// log2(s - popcount) only where some hash opens a block.
-// The reference maximum m moves only when a tile's maximum exceeds it by
-// more than 8 (then O and the row sum are rescaled), so every P <= 256.
+// Weights. P_ij = c_ij 2^(S_ij log2(e)/sqrt(d) - m): the count multiplies the
+// exponential as an exact small-integer float, so no logarithm is taken.
+// With R_ij the OR of the boundary masks strictly after min(i,j) up to
+// max(i,j), c_ij = s - popcount(R_ij), and R_ij splits into a part that
+// depends on the row only (a carry) and a part that depends on the key only,
+// the same for a whole warp: below the diagonal R = Y | suf[c] with Y the OR
+// from the tile's end to the row; above it R = Z | pre[c] with Z the OR from
+// the row to the tile's start. On the diagonal tile each warp owns 32 rows:
+// keys in its own 32-key block are scanned from the row outwards (before S
+// is ready), which yields the carries for the rest of the tile, whose keys
+// take range ORs that end (or start) at the warp's block. Key tiles are
+// visited diagonal first, then downward, then upward, so the carries pass
+// from tile to tile.
+// The reference m is a running upper bound: the largest S log2(e)/sqrt(d)
+// over the tile's keys that can carry weight raises it when it exceeds m by
+// more than 8, and O and the row sum are then rescaled; so P <= s 2^8, and
+// the row's own key (c = s) keeps the sum away from zero. Per tile a softmax
+// thread reads its row of S from TMEM twice, in chunks (the maximum, then
+// P), and writes P of keys [16ch, 16ch + 16) as bf16 pairs to columns
+// [8ch, 8ch + 8) of the S region, over columns it has already read.
 //
 // Every barrier wait is bounded in time (PLSH_DEVERR_TIMEOUT); on timeout all
 // roles leave their loops, in-flight copies and MMAs are drained and TMEM is
 // freed before the CTA returns.
 #include <cmath>
-#include <type_traits>
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -61,88 +65,77 @@ using namespace sm100;
 
 constexpr int kTile = PLSH_TILE;
 constexpr int kD = 128;
-constexpr int kThreads = 352;         // 11 warps
-constexpr int kSoftmaxWarps = 8;      // warps 0-7
-constexpr int kWarpTma = 8, kWarpMma = 9, kWarpMask = 10;
-constexpr int kHalf = 64;             // key columns per softmax thread
-constexpr int kStages = 2;
-constexpr int kChunkBytes = kTile * 64 * 2;         // 128 rows x 64 bf16 = 16 KB (one SW128 box)
-constexpr int kTileBytes = 2 * kChunkBytes;         // 128 x 128 bf16 = 32 KB
+constexpr int kThreads = 384;  // 12 warps
+constexpr int kSlots = 2;
+constexpr int kMaskStages = 2;
+constexpr int kChunkBytes = kTile * 64 * 2;  // 128 rows x 64 bf16 = 16 KB (one SW128 box)
+constexpr int kTileBytes = 2 * kChunkBytes;  // 128 x 128 bf16 = 32 KB
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;      // S buffers at columns 0 and 128 (P overwrites their first 64 columns)
-constexpr uint32_t kColO = 256;    // O buffers at columns 256 and 384
+constexpr uint32_t kColS = 0;              // S (then P) of slot z at columns 128 z
+constexpr uint32_t kColO = 256;            // O of slot z at columns 256 + 128 z
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kMaxSortedHeads = 256;
-constexpr int kTblRows = 33;       // table rows: popcounts 0..32
-constexpr int kTblStride = 132;    // floats per table row (spreads rows over banks)
+constexpr uint64_t kDrainNs = 100000000ull;
 
 template <typename MaskT>
 struct alignas(16) MaskStage {
-  MaskT bm[kTile + 4];   // bm[c]   = boundary mask of key j0 + c, c = 0..128 (all ones outside [0, n))
-  MaskT bmn[kTile];      // bmn[c]  = bm[c + 1]
-  MaskT pre[kTile];      // pre[c]  = OR bm[1 .. c]        (pre[0] = 0)
-  MaskT suf[kTile];      // suf[c]  = OR bm[c + 1 .. 127]  (suf[127] = 0)
-  MaskT preh[kHalf];     // preh[q] = OR bm[64 .. 64 + q]
-  MaskT sufl[kHalf];     // sufl[c] = OR bm[c + 1 .. 63]   (sufl[63] = 0)
+  MaskT bm[kTile + 4];  // bm[c]  = boundary mask of key j0 + c, c = 0..128 (all ones outside [0, n))
+  MaskT pre[kTile];     // pre[c] = OR bm[1 .. c]        (pre[0] = 0)
+  MaskT suf[kTile];     // suf[c] = OR bm[c + 1 .. 127]  (suf[127] = 0)
+  // range ORs against the 32-row block of warp q (diagonal tile only):
+  // dq[q][c] = OR bm[c + 1 .. 32q] for c < 32q, OR bm[32q + 32 .. c] for c >= 32q + 32
+  MaskT dq[4][kTile];
+  // the tile as the softmax needs it: valid (0 = end of the slot's work), kind (0 diagonal,
+  // 1 below, 2 above), first / last tile of its item, item index x
+  int valid, kind, first, last, x, pad0, pad1, pad2;
 };
 
-// Log2-weight table of one key tile (32-bit masks only).
-struct alignas(16) WeightTable {
-  float w[kTblRows][kTblStride];
+struct alignas(1024) SlotBuffers {
+  uint8_t q[kTileBytes];
+  uint8_t k[kTileBytes];
+  uint8_t v[kTileBytes];
 };
-struct NoTable {};
-
-template <typename MaskT>
-constexpr bool kUseTable = sizeof(MaskT) == 4;
 
 template <typename MaskT>
 struct __align__(1024) TcSmem {
-  uint8_t q[2][kTileBytes];
-  uint8_t k[kStages][kTileBytes];
-  uint8_t v[kStages][kTileBytes];
-  MaskStage<MaskT> m[kStages];
-  typename std::conditional<kUseTable<MaskT>, WeightTable, NoTable>::type tbl;
-  MaskT pfxq[kTile];                   // mask warp: OR over [i0, i0 + r] of the current item
-  MaskT sfxq[kTile];                   // mask warp: OR over (i0 + r, i0 + 127]
-  MaskT ykey[kTblRows + 3];            // mask warp: carry set of each popcount present
-  float pmax[2][2][kTile];             // [tile parity][half][row] partial row maxima
-  float psum[2][2][kTile];             // [item parity][half][row] partial row sums
-  float lg[PLSH_MAX_S + 4];            // lg[w] = log2(w), lg[0] = -inf
-  int16_t order[kMaxSortedHeads];      // heads by decreasing window width
+  SlotBuffers slot[kSlots];
+  MaskStage<MaskT> m[kSlots][kMaskStages];
+  int16_t order[kMaxSortedHeads];  // heads by decreasing window width
   int32_t width[kMaxSortedHeads];
-  uint64_t q_full[2], q_empty[2];
-  uint64_t k_full[kStages], k_empty[kStages];
-  uint64_t v_full[kStages], v_empty[kStages];
-  uint64_t m_full[kStages], m_empty[kStages];
-  uint64_t t_full, t_empty;            // weight table handoff
-  uint64_t s_full[2], p_full[2], pv_done[2];
-  uint64_t xmax[2], xsum[2];           // softmax half exchange: row maxima per tile, row sums per item
+  uint64_t q_full[kSlots], q_empty[kSlots];
+  uint64_t k_full[kSlots], k_empty[kSlots];
+  uint64_t v_full[kSlots], v_empty[kSlots];
+  uint64_t m_full[kSlots][kMaskStages], m_empty[kSlots][kMaskStages];
+  uint64_t s_full[kSlots], p_full[kSlots], o_full[kSlots];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
 };
+
+static_assert(sizeof(TcSmem<unsigned long long>) + 1024 <= 232448, "shared memory budget");
 
 struct Params {
   int B, H, H_kv, n, s, causal, T, items;
   const int32_t* spans;
 };
 
-// One key tile of one work item, in the order every role walks them. The
-// window of the next item is fetched one item ahead.
+// The key tiles of one slot's work items, in the order every role walks them:
+// items x0, x0 + stride, ...; within an item the diagonal tile, then the tiles
+// below, then (non-causal) the tiles above. The next item's window is fetched
+// one item ahead.
 struct TileIter {
   const Params* p;
   const int16_t* order;
-  int x;        // work item index
-  int k;        // work items started by this CTA so far (Q and O buffer = k & 1)
+  int x, stride;
+  int k;        // items started so far by this slot
   int it;       // key tile within the item
   int total;    // key tiles of the item
   int n_below;
-  int b, h, t, i0;
-  int g;        // key tile counted across this CTA's items
-  int u;        // table tiles (below / above the diagonal) counted across this CTA's items
+  int b, h, i0;
+  int g;        // key tiles so far by this slot
   bool valid;
   bool bad_window;  // the window read for this item was out of range (and was clamped)
-  int nx_lo, nx_hi; // window of item x + gridDim.x
+  int nx_lo, nx_hi;
 
   __device__ __forceinline__ int head_of(int xx) const {
     const int hr = xx / (p->B * p->T);
@@ -151,7 +144,7 @@ struct TileIter {
   __device__ __forceinline__ void fetch(int xx, int& lo, int& hi) const {
     if (xx < p->items) {
       const int hh = head_of(xx);
-      const int tt = (xx - (xx / (p->B * p->T)) * (p->B * p->T)) % p->T;
+      const int tt = (xx % (p->B * p->T)) % p->T;
       lo = p->spans[(static_cast<size_t>(hh) * p->T + tt) * 2];
       hi = p->spans[(static_cast<size_t>(hh) * p->T + tt) * 2 + 1];
     }
@@ -159,13 +152,11 @@ struct TileIter {
   __device__ __forceinline__ void load_item(int lo, int hi) {
     valid = x < p->items;
     if (!valid) return;
-    const int BT = p->B * p->T;
-    const int rem = x - (x / BT) * BT;
+    const int rem = x % (p->B * p->T);
     h = head_of(x);
     b = rem / p->T;
-    t = rem - b * p->T;
-    i0 = t * kTile;
-    fetch(x + gridDim.x, nx_lo, nx_hi);
+    i0 = (rem % p->T) * kTile;
+    fetch(x + stride, nx_lo, nx_hi);
     const int last_row = min(p->n, i0 + kTile) - 1;
     bad_window = lo < 0 || lo > i0 || hi >= p->n || hi < last_row;
     lo = max(0, min(lo, i0));
@@ -174,13 +165,13 @@ struct TileIter {
     total = 1 + n_below + (p->causal ? 0 : (hi - i0) / kTile);
     it = 0;
   }
-  __device__ __forceinline__ void start(const Params* pp, const int16_t* ord) {
+  __device__ __forceinline__ void start(const Params* pp, const int16_t* ord, int slot) {
     p = pp;
     order = ord;
-    x = blockIdx.x;
+    x = blockIdx.x + slot * gridDim.x;
+    stride = kSlots * gridDim.x;
     k = 0;
     g = 0;
-    u = 0;
     nx_lo = nx_hi = 0;
     int lo = 0, hi = 0;
     fetch(x, lo, hi);
@@ -188,9 +179,8 @@ struct TileIter {
   }
   __device__ __forceinline__ void next() {
     ++g;
-    if (it > 0) ++u;
     if (++it >= total) {
-      x += gridDim.x;
+      x += stride;
       ++k;
       load_item(nx_lo, nx_hi);
     }
@@ -223,7 +213,7 @@ __device__ __forceinline__ void load4(const MaskT* p, MaskT (&b)[4]) {
 }
 
 template <typename MaskT>
-__device__ __forceinline__ MaskT warp_prefix_or(MaskT v, int lane) {   // inclusive over lanes 0..lane
+__device__ __forceinline__ MaskT warp_prefix_or(MaskT v, int lane) {  // inclusive over lanes 0..lane
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const MaskT y = __shfl_up_sync(0xffffffffu, v, o);
@@ -233,7 +223,7 @@ __device__ __forceinline__ MaskT warp_prefix_or(MaskT v, int lane) {   // inclus
 }
 
 template <typename MaskT>
-__device__ __forceinline__ MaskT warp_suffix_or(MaskT v, int lane) {   // inclusive over lanes lane..31
+__device__ __forceinline__ MaskT warp_suffix_or(MaskT v, int lane) {  // inclusive over lanes lane..31
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const MaskT y = __shfl_down_sync(0xffffffffu, v, o);
@@ -242,133 +232,107 @@ __device__ __forceinline__ MaskT warp_suffix_or(MaskT v, int lane) {   // inclus
   return v;
 }
 
-__device__ __forceinline__ int lg_index(int s, int popcount) { return max(0, s - popcount); }
-
-// x[cc] <- x[cc] * sc + table row, for the 64 columns of this half (loads issued four at a time
-// so that at most 16 table values are live next to the 64 logits).
-__device__ __forceinline__ void logits_from_table(float (&x)[kHalf], const float* row, float sc) {
+__device__ __forceinline__ float max32(const uint32_t (&v)[32], float m) {
+  float mx[8];
 #pragma unroll
-  for (int g4 = 0; g4 < kHalf / 4; ++g4) {
-    if ((g4 & 3) == 0) asm volatile("" ::: "memory");
-    const float4 t4 = reinterpret_cast<const float4*>(row)[g4];
-    x[4 * g4 + 0] = fmaf(x[4 * g4 + 0], sc, t4.x);
-    x[4 * g4 + 1] = fmaf(x[4 * g4 + 1], sc, t4.y);
-    x[4 * g4 + 2] = fmaf(x[4 * g4 + 2], sc, t4.z);
-    x[4 * g4 + 3] = fmaf(x[4 * g4 + 3], sc, t4.w);
-  }
+  for (int u = 0; u < 8; ++u) mx[u] = __uint_as_float(v[u]);
+#pragma unroll
+  for (int c = 8; c < 32; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(v[c]));
+  return fmaxf(m, fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                        fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))));
 }
 
-// Scans for one row's half of a key tile: x[cc] <- S[c] * sc + log2(c_ij) for c = 64*half + cc.
-// kind 0: diagonal tile (row r is column r); kind 1: below the diagonal; kind 2: above.
-// R is the OR over the gap between the row and the current key, carried in from Y / Z.
+// float(v) for 0 <= v < 2^23, exactly: the float with the bits of 2^23 + v, minus 2^23.
+__device__ __forceinline__ float small_count(uint32_t v) { return __int_as_float(0x4B000000u | v) - 8388608.0f; }
+
+// s - popcount(carry | km) as a float, exactly, given cs = 2^23 + s.
+template <typename MaskT>
+__device__ __forceinline__ float count_weight(MaskT carry, MaskT km, float cs) {
+  return cs - __int_as_float(0x4B000000u | static_cast<uint32_t>(popc_m(static_cast<MaskT>(carry | km))));
+}
+
+// P = w 2^(S sc - m) for 16 keys (S as raw fp32 bits) with w = s - popcount(carry | km[k]),
+// packed as 8 bf16 pairs. Returns the sum of P.
+template <typename MaskT>
+__device__ __forceinline__ float p16_carry(const uint32_t (&sv)[16], const MaskT* km, MaskT carry, float sc,
+                                           float neg_m, float cs, uint32_t (&pk)[8]) {
+  float ls[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+  for (int g4 = 0; g4 < 4; ++g4) {
+    MaskT bb[4];
+    load4(km + 4 * g4, bb);
+    float p[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      p[e] = ex2_approx(fmaf(__uint_as_float(sv[4 * g4 + e]), sc, neg_m)) * count_weight(carry, bb[e], cs);
+      ls[e] += p[e];
+    }
+    pk[2 * g4] = pack_bf16x2(p[0], p[1]);
+    pk[2 * g4 + 1] = pack_bf16x2(p[2], p[3]);
+  }
+  return (ls[0] + ls[1]) + (ls[2] + ls[3]);
+}
+
+// The same with the counts given as bytes: the count of key k in byte k % 4 of c4[k / 4].
+__device__ __forceinline__ float p16_counts(const uint32_t (&sv)[16], const uint32_t (&c4)[4], float sc,
+                                            float neg_m, uint32_t (&pk)[8]) {
+  float ls[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+  for (int g4 = 0; g4 < 4; ++g4) {
+    float p[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      p[e] = ex2_approx(fmaf(__uint_as_float(sv[4 * g4 + e]), sc, neg_m)) * small_count((c4[g4] >> (8 * e)) & 0xffu);
+      ls[e] += p[e];
+    }
+    pk[2 * g4] = pack_bf16x2(p[0], p[1]);
+    pk[2 * g4 + 1] = pack_bf16x2(p[2], p[3]);
+  }
+  return (ls[0] + ls[1]) + (ls[2] + ls[3]);
+}
+
+// Diagonal tile, warp q (rows [32q, 32q + 32), row r): counts of the warp's own 32 keys, as bytes
+// (key 32q + k in byte k % 4 of cnt[k / 4]), and the carries for the other keys. Keys c <= r:
+// R = OR bm[c + 1 .. r], scanned from the row down; keys c > r: R = OR bm[r + 1 .. c]
+// (non-causal; count 0 when causal), scanned from the row up. On return
+// lo = OR bm[32q + 1 .. r] and hi = OR bm[r + 1 .. 32q + 31].
 template <typename MaskT, bool kCausal>
-__device__ __forceinline__ void logits_by_scan(float (&x)[kHalf], const MaskStage<MaskT>& ms, const float* lg,
-                                               int kind, int r, int half, int s, float sc, MaskT Y, MaskT Z) {
-  const int c0 = kHalf * half;
-  if (kind == 1) {
-    // R(127) = Y, R(63) = Y | OR bm[64..127], R(c) = R(c + 1) | bm[c + 1]
-    MaskT R = half ? Y : static_cast<MaskT>(Y | ms.suf[kHalf - 1]);
-    float lw = lg[lg_index(s, popc_m(R))];
+__device__ __forceinline__ void diag_scan(const MaskStage<MaskT>& ms, int q, int r, int s, uint32_t (&cnt)[8],
+                                          MaskT& lo, MaskT& hi) {
+  const MaskT* bq = ms.bm + 32 * q;
+  const int rr = r - 32 * q;  // the row within the block, 0..31
 #pragma unroll
-    for (int g4 = kHalf / 4 - 1; g4 >= 0; --g4) {
-      MaskT bb[4];
-      load4(&ms.bmn[c0 + 4 * g4], bb);
-      if (g4 == kHalf / 4 - 1 && half) bb[3] = 0;
-      if ((bb[0] | bb[1] | bb[2] | bb[3]) != 0) {
+  for (int u = 0; u < 8; ++u) cnt[u] = 0u;
+  MaskT R = 0;
 #pragma unroll
-        for (int e = 3; e >= 0; --e) {
-          R |= bb[e];
-          lw = lg[lg_index(s, popc_m(R))];
-          x[4 * g4 + e] = fmaf(x[4 * g4 + e], sc, lw);
-        }
-      } else {
+  for (int cc = 31; cc >= 0; --cc) {
+    if (cc < rr) R |= bq[cc + 1];
+    const uint32_t v = (cc <= rr) ? static_cast<uint32_t>(s - popc_m(R)) : 0u;
+    cnt[cc >> 2] |= v << (8 * (cc & 3));
+  }
+  lo = R;
+  MaskT R2 = 0;
+  if (!kCausal) {
 #pragma unroll
-        for (int e = 3; e >= 0; --e) x[4 * g4 + e] = fmaf(x[4 * g4 + e], sc, lw);
-      }
-    }
-  } else if (!kCausal && kind == 2) {
-    // R(0) = Z (holds bm[0]), R(63) = Z | OR bm[1..63], R(c) = R(c - 1) | bm[c]
-    MaskT R = half ? static_cast<MaskT>(Z | ms.pre[kHalf - 1]) : Z;
-    float lw = lg[lg_index(s, popc_m(R))];
-#pragma unroll
-    for (int g4 = 0; g4 < kHalf / 4; ++g4) {
-      MaskT bb[4];
-      load4(&ms.bm[c0 + 4 * g4], bb);
-      if (g4 == 0 && !half) bb[0] = 0;
-      if ((bb[0] | bb[1] | bb[2] | bb[3]) != 0) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          R |= bb[e];
-          lw = lg[lg_index(s, popc_m(R))];
-          x[4 * g4 + e] = fmaf(x[4 * g4 + e], sc, lw);
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) x[4 * g4 + e] = fmaf(x[4 * g4 + e], sc, lw);
-      }
-    }
-  } else {
-    // columns c <= r: R(c) = OR bm[c+1 .. r]; in the low half a row r >= 64 starts from OR bm[64..r]
-    MaskT R = (!half && r >= kHalf) ? ms.preh[r - kHalf] : static_cast<MaskT>(0);
-    float lw = lg[lg_index(s, popc_m(R))];
-#pragma unroll
-    for (int g4 = kHalf / 4 - 1; g4 >= 0; --g4) {
-      MaskT bb[4];
-      load4(&ms.bmn[c0 + 4 * g4], bb);
-      if ((bb[0] | bb[1] | bb[2] | bb[3]) != 0) {
-#pragma unroll
-        for (int e = 3; e >= 0; --e) {
-          const int cc = 4 * g4 + e, c = c0 + cc;
-          if (c < r) R |= bb[e];
-          lw = lg[lg_index(s, popc_m(R))];
-          x[cc] = (c <= r) ? fmaf(x[cc], sc, lw) : (kCausal ? -INFINITY : x[cc]);
-        }
-      } else {
-#pragma unroll
-        for (int e = 3; e >= 0; --e) {
-          const int cc = 4 * g4 + e, c = c0 + cc;
-          x[cc] = (c <= r) ? fmaf(x[cc], sc, lw) : (kCausal ? -INFINITY : x[cc]);
-        }
-      }
-    }
-    if (!kCausal) {
-      // columns c > r: R(c) = OR bm[r+1 .. c]; in the high half a row r < 64 starts from OR bm[r+1..63]
-      MaskT R2 = (half && r < kHalf) ? ms.sufl[r] : static_cast<MaskT>(0);
-      float lw2 = lg[lg_index(s, popc_m(R2))];
-#pragma unroll
-      for (int g4 = 0; g4 < kHalf / 4; ++g4) {
-        MaskT bb[4];
-        load4(&ms.bm[c0 + 4 * g4], bb);
-        if ((bb[0] | bb[1] | bb[2] | bb[3]) != 0) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int cc = 4 * g4 + e, c = c0 + cc;
-            if (c > r) R2 |= bb[e];
-            lw2 = lg[lg_index(s, popc_m(R2))];
-            if (c > r) x[cc] = fmaf(x[cc], sc, lw2);
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int cc = 4 * g4 + e, c = c0 + cc;
-            if (c > r) x[cc] = fmaf(x[cc], sc, lw2);
-          }
-        }
+    for (int cc = 0; cc < 32; ++cc) {
+      if (cc > rr) {
+        R2 |= bq[cc];
+        cnt[cc >> 2] |= static_cast<uint32_t>(s - popc_m(R2)) << (8 * (cc & 3));
       }
     }
   }
+  hi = R2;
 }
 
 template <typename MaskT, bool kCausal>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ Params prm,
-               const double* __restrict__ sigma,
-               const double* __restrict__ table, const MaskT* __restrict__ bmask, __nv_bfloat16* __restrict__ O,
-               float* __restrict__ row_sum, uint32_t* __restrict__ err) {
-  constexpr bool kTable = kUseTable<MaskT>;
-  extern __shared__ uint8_t smem_raw[];
-  auto& sm = *reinterpret_cast<TcSmem<MaskT>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+               const double* __restrict__ sigma, const double* __restrict__ table, const MaskT* __restrict__ bmask,
+               __nv_bfloat16* __restrict__ O, float* __restrict__ row_sum, uint32_t* __restrict__ err) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t smem_pad = (1024u - (static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw)) & 1023u)) & 1023u;
+  auto& sm = *reinterpret_cast<TcSmem<MaskT>*>(smem_raw + smem_pad);
   volatile int* abort_flag = &sm.abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n = prm.n, s = prm.s, H = prm.H;
@@ -395,8 +359,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       sm.width[h] = prm.spans[(static_cast<size_t>(h) * prm.T + tm) * 2 + 1] -
                     prm.spans[(static_cast<size_t>(h) * prm.T + tm) * 2];
   }
-  if (threadIdx.x < PLSH_MAX_S + 4)
-    sm.lg[threadIdx.x] = threadIdx.x == 0 ? -INFINITY : log2f(static_cast<float>(threadIdx.x));
   __syncthreads();
   if (H <= kMaxSortedHeads) {
     for (int h = threadIdx.x; h < H; h += kThreads) {
@@ -411,29 +373,25 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   }
   if (threadIdx.x == 0) {
     sm.abort_flag = 0;
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sm.q_full[i], 1);
-      mbar_init(&sm.q_empty[i], 1);
-      mbar_init(&sm.s_full[i], 1);
-      mbar_init(&sm.p_full[i], kSoftmaxWarps);
-      mbar_init(&sm.pv_done[i], 1);
-      mbar_init(&sm.xmax[i], kSoftmaxWarps);
-      mbar_init(&sm.xsum[i], kSoftmaxWarps);
+    for (int z = 0; z < kSlots; ++z) {
+      mbar_init(&sm.q_full[z], 1);
+      mbar_init(&sm.q_empty[z], 1);
+      mbar_init(&sm.k_full[z], 1);
+      mbar_init(&sm.k_empty[z], 1);
+      mbar_init(&sm.v_full[z], 1);
+      mbar_init(&sm.v_empty[z], 1);
+      mbar_init(&sm.s_full[z], 1);
+      mbar_init(&sm.p_full[z], 4);
+      mbar_init(&sm.o_full[z], 1);
+      for (int i = 0; i < kMaskStages; ++i) {
+        mbar_init(&sm.m_full[z][i], 1);
+        mbar_init(&sm.m_empty[z][i], 4);
+      }
     }
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&sm.k_full[i], 1);
-      mbar_init(&sm.k_empty[i], 1);
-      mbar_init(&sm.v_full[i], 1);
-      mbar_init(&sm.v_empty[i], 1);
-      mbar_init(&sm.m_full[i], 1);
-      mbar_init(&sm.m_empty[i], kSoftmaxWarps);
-    }
-    mbar_init(&sm.t_full, 1);
-    mbar_init(&sm.t_empty, kSoftmaxWarps);
     mbar_init(&sm.drain, 1);
     fence_mbarrier_init();
   }
-  if (warp == kWarpMma) {
+  if (warp == 1) {
     tmem_alloc(&sm.tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -442,372 +400,327 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
-  if (warp == kWarpTma) {
-    // ------------------------------------------------------------ TMA producer
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both slots)
+    // Six streams, Q (per item), K and V (per key tile) of each slot, each issued as soon as
+    // its buffer is free; the thread polls, so one slot's stall never holds up the other.
     if (lane == 0) {
       tma_prefetch_desc(&tmap_q);
       tma_prefetch_desc(&tmap_k);
       tma_prefetch_desc(&tmap_v);
-      TileIter ti;
-      ti.start(&prm, sm.order);
-      int issued_g = 0, issued_k = 0;
-      bool ok = true;
-      while (ok && ti.valid) {
-        const int zkv = ti.b * prm.H_kv + ti.h / (H / prm.H_kv);
-        if (ti.first()) {
-          const int qb = ti.k & 1;
-          if (ti.k >= 2 && !mbar_wait(&sm.q_empty[qb], ((ti.k >> 1) & 1) ^ 1, abort_flag, err)) break;
-          mbar_arrive_expect_tx(&sm.q_full[qb], kTileBytes);
-          tma_load_3d(sm.q[qb], &tmap_q, 0, ti.i0, ti.b * H + ti.h, &sm.q_full[qb]);
-          tma_load_3d(sm.q[qb] + kChunkBytes, &tmap_q, 64, ti.i0, ti.b * H + ti.h, &sm.q_full[qb]);
-          issued_k = ti.k + 1;
+      TileIter kit[kSlots], vit[kSlots];
+      for (int z = 0; z < kSlots; ++z) {
+        kit[z].start(&prm, sm.order, z);
+        vit[z].start(&prm, sm.order, z);
+      }
+      uint64_t idle_since = 0;
+      uint32_t spins = 0;
+      while (kit[0].valid || kit[1].valid || vit[0].valid || vit[1].valid) {
+        bool progress = false;
+#pragma unroll
+        for (int z = 0; z < kSlots; ++z) {
+          TileIter& ki = kit[z];
+          if (ki.valid) {
+            // Q of a new item once the slot's previous item has run its last S; K(g) once S(g-1) has run
+            const bool q_ok = !ki.first() || ki.k == 0 || mbar_test_wait(&sm.q_empty[z], (ki.k - 1) & 1);
+            const bool k_ok = ki.g == 0 || mbar_test_wait(&sm.k_empty[z], (ki.g - 1) & 1);
+            if (q_ok && k_ok) {
+              if (ki.first()) {
+                mbar_arrive_expect_tx(&sm.q_full[z], kTileBytes);
+                tma_load_3d(sm.slot[z].q, &tmap_q, 0, ki.i0, ki.b * H + ki.h, &sm.q_full[z]);
+                tma_load_3d(sm.slot[z].q + kChunkBytes, &tmap_q, 64, ki.i0, ki.b * H + ki.h, &sm.q_full[z]);
+              }
+              const int zkv = ki.b * prm.H_kv + ki.h / (H / prm.H_kv);
+              const int j0 = ki.j0();
+              mbar_arrive_expect_tx(&sm.k_full[z], kTileBytes);
+              tma_load_3d(sm.slot[z].k, &tmap_k, 0, j0, zkv, &sm.k_full[z]);
+              tma_load_3d(sm.slot[z].k + kChunkBytes, &tmap_k, 64, j0, zkv, &sm.k_full[z]);
+              ki.next();
+              progress = true;
+            }
+          }
+          TileIter& vi = vit[z];
+          if (vi.valid && (vi.g == 0 || mbar_test_wait(&sm.v_empty[z], (vi.g - 1) & 1))) {
+            const int zkv = vi.b * prm.H_kv + vi.h / (H / prm.H_kv);
+            const int j0 = vi.j0();
+            mbar_arrive_expect_tx(&sm.v_full[z], kTileBytes);
+            tma_load_3d(sm.slot[z].v, &tmap_v, 0, j0, zkv, &sm.v_full[z]);
+            tma_load_3d(sm.slot[z].v + kChunkBytes, &tmap_v, 64, j0, zkv, &sm.v_full[z]);
+            vi.next();
+            progress = true;
+          }
         }
-        const int st = ti.g % kStages;
-        const uint32_t ph = static_cast<uint32_t>(ti.g / kStages) & 1u;
-        const int j0 = ti.j0();
-        if (ti.g >= kStages && !mbar_wait(&sm.k_empty[st], ph ^ 1u, abort_flag, err)) break;
-        mbar_arrive_expect_tx(&sm.k_full[st], kTileBytes);
-        tma_load_3d(sm.k[st], &tmap_k, 0, j0, zkv, &sm.k_full[st]);
-        tma_load_3d(sm.k[st] + kChunkBytes, &tmap_k, 64, j0, zkv, &sm.k_full[st]);
-        ok = !(ti.g >= kStages && !mbar_wait(&sm.v_empty[st], ph ^ 1u, abort_flag, err));
-        if (ok) {
-          mbar_arrive_expect_tx(&sm.v_full[st], kTileBytes);
-          tma_load_3d(sm.v[st], &tmap_v, 0, j0, zkv, &sm.v_full[st]);
-          tma_load_3d(sm.v[st] + kChunkBytes, &tmap_v, 64, j0, zkv, &sm.v_full[st]);
+        if (progress) {
+          idle_since = 0;
+          spins = 0;
+        } else if ((++spins & 63u) == 0) {
+          const uint64_t now = global_timer_ns();
+          if (idle_since == 0) idle_since = now;
+          if (*abort_flag) break;
+          if (now - idle_since > kWaitLimitNs) {
+            *abort_flag = 1;
+            atomicOr(err, PLSH_DEVERR_TIMEOUT);
+            break;
+          }
         }
-        issued_g = ti.g + 1;
-        ti.next();
       }
       if (*abort_flag) {
         // let every copy already issued land before the CTA can exit
-        for (int kk = (issued_k > 2 ? issued_k - 2 : 0); kk < issued_k; ++kk)
-          mbar_wait_drain(&sm.q_full[kk & 1], (kk >> 1) & 1, 100000000ull);
-        for (int gg = (issued_g > kStages ? issued_g - kStages : 0); gg < issued_g; ++gg) {
-          const int st = gg % kStages;
-          const uint32_t ph = static_cast<uint32_t>(gg / kStages) & 1u;
-          mbar_wait_drain(&sm.k_full[st], ph, 100000000ull);
-          mbar_wait_drain(&sm.v_full[st], ph, 100000000ull);
+        for (int z = 0; z < kSlots; ++z) {
+          const int q_issued = kit[z].k + ((kit[z].valid && kit[z].it > 0) ? 1 : 0);
+          if (q_issued > 0) mbar_wait_drain(&sm.q_full[z], (q_issued - 1) & 1, kDrainNs);
+          if (kit[z].g > 0) mbar_wait_drain(&sm.k_full[z], (kit[z].g - 1) & 1, kDrainNs);
+          if (vit[z].g > 0) mbar_wait_drain(&sm.v_full[z], (vit[z].g - 1) & 1, kDrainNs);
         }
       }
     }
-  } else if (warp == kWarpMma) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (both slots)
+    // Per slot: S(g) needs Q, K(g) and PV(g-1) issued (P of g-1 lives in S's columns; the tensor
+    // core runs one thread's MMAs in order); PV(g) needs P(g) and V(g).
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, 1);
-      auto issue_s = [&](const TileIter& ti) -> bool {
-        const int qb = ti.k & 1;
-        if (ti.first() && !mbar_wait(&sm.q_full[qb], (ti.k >> 1) & 1, abort_flag, err)) return false;
-        const int st = ti.g % kStages;
-        if (!mbar_wait(&sm.k_full[st], static_cast<uint32_t>(ti.g / kStages) & 1u, abort_flag, err)) return false;
-        tc_fence_after();
-        const uint32_t q_addr = smem_u32(sm.q[qb]);
-        const uint32_t k_addr = smem_u32(sm.k[st]);
-        const uint32_t d_tmem = tmem + kColS + 128u * static_cast<uint32_t>(ti.g & 1);
+      TileIter st_it[kSlots], pv_it[kSlots];
+      for (int z = 0; z < kSlots; ++z) {
+        st_it[z].start(&prm, sm.order, z);
+        pv_it[z].start(&prm, sm.order, z);
+      }
+      uint64_t idle_since = 0;
+      uint32_t spins = 0;
+      while (pv_it[0].valid || pv_it[1].valid) {
+        bool progress = false;
 #pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t off = static_cast<uint32_t>((kk >> 2) * kChunkBytes + (kk & 3) * 32);
-          mma_ss(d_tmem, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024),
-                 idesc_qk, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(&sm.s_full[ti.g & 1]);
-        mma_commit(&sm.k_empty[st]);
-        if (ti.last()) mma_commit(&sm.q_empty[qb]);
-        return true;
-      };
-      auto issue_pv = [&](const TileIter& ti) -> bool {
-        const int st = ti.g % kStages;
-        if (!mbar_wait(&sm.p_full[ti.g & 1], static_cast<uint32_t>(ti.g >> 1) & 1u, abort_flag, err)) return false;
-        if (!mbar_wait(&sm.v_full[st], static_cast<uint32_t>(ti.g / kStages) & 1u, abort_flag, err)) return false;
-        tc_fence_after();
-        const uint32_t v_addr = smem_u32(sm.v[st]);
-        const uint32_t p_tmem = tmem + kColS + 128u * static_cast<uint32_t>(ti.g & 1);
-        const uint32_t o_tmem = tmem + kColO + 128u * static_cast<uint32_t>(ti.k & 1);
+        for (int z = 0; z < kSlots; ++z) {
+          TileIter& si = st_it[z];
+          TileIter& pi = pv_it[z];
+          if (si.valid && si.g == pi.g && (!si.first() || mbar_test_wait(&sm.q_full[z], si.k & 1)) &&
+              mbar_test_wait(&sm.k_full[z], si.g & 1)) {
+            tc_fence_after();
+            const uint32_t q_addr = smem_u32(sm.slot[z].q);
+            const uint32_t k_addr = smem_u32(sm.slot[z].k);
+            const uint32_t d_tmem = tmem + kColS + 128u * z;
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk) {
-          // 16 keys = two 8-row groups of the MN-major V tile; the two d halves sit kChunkBytes apart
-          mma_ts(o_tmem, p_tmem + 8u * kk, smem_desc_sw128(v_addr + kk * 2048, kChunkBytes, 1024), idesc_pv,
-                 (ti.it > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < kD / 16; ++kk) {
+              const uint32_t off = static_cast<uint32_t>((kk >> 2) * kChunkBytes + (kk & 3) * 32);
+              mma_ss(d_tmem, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024),
+                     idesc_qk, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(&sm.s_full[z]);
+            mma_commit(&sm.k_empty[z]);
+            if (si.last()) mma_commit(&sm.q_empty[z]);
+            si.next();
+            progress = true;
+          }
+          if (pi.valid && pi.g < si.g && mbar_test_wait(&sm.p_full[z], pi.g & 1) &&
+              mbar_test_wait(&sm.v_full[z], pi.g & 1)) {
+            tc_fence_after();
+            const uint32_t v_addr = smem_u32(sm.slot[z].v);
+            const uint32_t p_tmem = tmem + kColS + 128u * z;
+            const uint32_t o_tmem = tmem + kColO + 128u * z;
+#pragma unroll
+            for (int kk = 0; kk < kTile / 16; ++kk) {
+              // keys 16kk..16kk+15: P at columns 8kk..8kk+7; the keys are two 8-row groups of the
+              // MN-major V tile, whose two d halves sit kChunkBytes apart
+              mma_ts(o_tmem, p_tmem + 8u * kk,
+                     smem_desc_sw128(v_addr + kk * 2048, kChunkBytes, 1024), idesc_pv,
+                     (pi.it > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(&sm.v_empty[z]);
+            if (pi.last()) mma_commit(&sm.o_full[z]);
+            pi.next();
+            progress = true;
+          }
         }
-        mma_commit(&sm.pv_done[ti.g & 1]);
-        mma_commit(&sm.v_empty[st]);
-        return true;
-      };
-      // `nxt` runs one tile ahead of `cur`: S of the next tile is issued before PV of the current one
-      TileIter cur, nxt;
-      cur.start(&prm, sm.order);
-      nxt.start(&prm, sm.order);
-      bool ok = !cur.valid || issue_s(cur);
-      if (nxt.valid) nxt.next();
-      while (ok && cur.valid) {
-        if (nxt.valid) ok = issue_s(nxt);
-        if (ok) ok = issue_pv(cur);
-        cur.next();
-        if (nxt.valid) nxt.next();
+        if (progress) {
+          idle_since = 0;
+          spins = 0;
+        } else if ((++spins & 63u) == 0) {
+          const uint64_t now = global_timer_ns();
+          if (idle_since == 0) idle_since = now;
+          if (*abort_flag) break;
+          if (now - idle_since > kWaitLimitNs) {
+            *abort_flag = 1;
+            atomicOr(err, PLSH_DEVERR_TIMEOUT);
+            break;
+          }
+        }
       }
       // every MMA issued so far completes before `drain` arrives
       mma_commit(&sm.drain);
-      mbar_wait_drain(&sm.drain, 0, 100000000ull);
+      mbar_wait_drain(&sm.drain, 0, kDrainNs);
     }
-  } else if (warp == kWarpMask) {
-    // ------------------------------------------------------------ mask warp
-    TileIter ti;
-    ti.start(&prm, sm.order);
-    MaskT mid_b = 0;   // below the diagonal: OR over [j0 + 128, i0)
-    MaskT mid_a = 0;   // above the diagonal: OR over [i0 + 128, j0]
-    while (ti.valid) {
-      const int st = ti.g % kStages;
-      if (ti.g >= kStages &&
-          !mbar_wait(&sm.m_empty[st], (static_cast<uint32_t>(ti.g / kStages) & 1u) ^ 1u, abort_flag, err))
-        break;
-      const MaskT* bm_h = bmask + static_cast<size_t>(ti.h) * n;
-      MaskStage<MaskT>& ms = sm.m[st];
-      const int j0 = ti.j0();
-      const int kind = ti.kind();
-      MaskT xv[4];
+  } else if (warp == 2 || warp == 3) {
+    // ------------------------------------------------------------ mask warp of slot (warp - 2)
+    const int z = warp - 2;
+    TileIter ti, nx;
+    ti.start(&prm, sm.order, z);
+    nx.start(&prm, sm.order, z);
+    if (nx.valid) nx.next();
+    auto load_masks = [&](const TileIter& t, MaskT (&v)[4], MaskT& v128) {
+      const MaskT* bm_h = bmask + static_cast<size_t>(t.h) * n;
+      const int j0 = t.j0();
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int c = 4 * lane + e, j = j0 + c;
-        xv[e] = (j >= 0 && j < n) ? bm_h[j] : FULL;
-        ms.bm[c] = xv[e];
-        if (c >= 1) ms.bmn[c - 1] = xv[e];
+        const int j = j0 + 4 * lane + e;
+        v[e] = (j >= 0 && j < n) ? bm_h[j] : FULL;
       }
-      if (lane == 0) {
-        const int j = j0 + kTile;
-        const MaskT v = (j >= 0 && j < n) ? bm_h[j] : FULL;
-        ms.bm[kTile] = v;
-        ms.bmn[kTile - 1] = v;
+      const int j = j0 + kTile;
+      v128 = (lane == 0 && j >= 0 && j < n) ? bm_h[j] : FULL;
+    };
+    MaskT xv[4] = {FULL, FULL, FULL, FULL}, x128 = FULL;
+    if (ti.valid) load_masks(ti, xv, x128);
+    int g_end = 0;
+    bool ok = true;
+    while (ti.valid) {
+      const int st = ti.g % kMaskStages;
+      MaskT nv[4] = {FULL, FULL, FULL, FULL}, n128 = FULL;
+      if (nx.valid) load_masks(nx, nv, n128);  // lands while this tile is processed
+      if (ti.g >= kMaskStages) {
+        ok = mbar_wait(&sm.m_empty[z][st], (static_cast<uint32_t>(ti.g / kMaskStages) & 1u) ^ 1u, abort_flag, err);
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
+        }
       }
+      MaskStage<MaskT>& ms = sm.m[z][st];
       MaskT pre_v[4], suf_v[4];
       {  // pre[c] = OR bm[1..c]
         const MaskT p0 = lane == 0 ? static_cast<MaskT>(0) : xv[0];
         const MaskT p1 = p0 | xv[1], p2 = p1 | xv[2], p3 = p2 | xv[3];
         MaskT before = __shfl_up_sync(0xffffffffu, warp_prefix_or<MaskT>(p3, lane), 1);
         if (lane == 0) before = 0;
-        pre_v[0] = before | p0; pre_v[1] = before | p1; pre_v[2] = before | p2; pre_v[3] = before | p3;
+        pre_v[0] = before | p0;
+        pre_v[1] = before | p1;
+        pre_v[2] = before | p2;
+        pre_v[3] = before | p3;
       }
       {  // suf[c] = OR bm[c+1..127]
         const MaskT u2 = xv[3], u1 = u2 | xv[2], u0 = u1 | xv[1];
         MaskT after = __shfl_down_sync(0xffffffffu, warp_suffix_or<MaskT>(u0 | xv[0], lane), 1);
         if (lane == 31) after = 0;
-        suf_v[0] = after | u0; suf_v[1] = after | u1; suf_v[2] = after | u2; suf_v[3] = after;
+        suf_v[0] = after | u0;
+        suf_v[1] = after | u1;
+        suf_v[2] = after | u2;
+        suf_v[3] = after;
+      }
+      // range ORs against each warp's 32-row block of the diagonal tile
+      if (ti.kind() == 0) {
+#pragma unroll
+        for (int q = 1; q < 4; ++q) {  // dq[q][c] = OR bm[c + 1 .. 32q], c < 32q
+          MaskT v[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) v[e] = (4 * lane + e <= 32 * q) ? xv[e] : static_cast<MaskT>(0);
+          const MaskT u2 = v[3], u1 = u2 | v[2], u0 = u1 | v[1];
+          MaskT after = __shfl_down_sync(0xffffffffu, warp_suffix_or<MaskT>(u0 | v[0], lane), 1);
+          if (lane == 31) after = 0;
+          if (4 * lane < 32 * q) {
+            ms.dq[q][4 * lane] = after | u0;
+            ms.dq[q][4 * lane + 1] = after | u1;
+            ms.dq[q][4 * lane + 2] = after | u2;
+            ms.dq[q][4 * lane + 3] = after;
+          }
+        }
+        if (!kCausal) {
+#pragma unroll
+          for (int q = 0; q < 3; ++q) {  // dq[q][c] = OR bm[32q + 32 .. c], c >= 32q + 32
+            MaskT v[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) v[e] = (4 * lane + e >= 32 * q + 32) ? xv[e] : static_cast<MaskT>(0);
+            const MaskT p0 = v[0], p1 = p0 | v[1], p2 = p1 | v[2], p3 = p2 | v[3];
+            MaskT before = __shfl_up_sync(0xffffffffu, warp_prefix_or<MaskT>(p3, lane), 1);
+            if (lane == 0) before = 0;
+            if (4 * lane >= 32 * q + 32) {
+              ms.dq[q][4 * lane] = before | p0;
+              ms.dq[q][4 * lane + 1] = before | p1;
+              ms.dq[q][4 * lane + 2] = before | p2;
+              ms.dq[q][4 * lane + 3] = before | p3;
+            }
+          }
+        }
       }
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        ms.pre[4 * lane + e] = pre_v[e];
-        ms.suf[4 * lane + e] = suf_v[e];
+        const int c = 4 * lane + e;
+        ms.bm[c] = xv[e];
+        ms.pre[c] = pre_v[e];
+        ms.suf[c] = suf_v[e];
       }
-      {  // preh[q] = OR bm[64..64+q] (lanes 16..31 hold columns 64..127)
-        const bool hiL = lane >= 16;
-        const MaskT h0 = xv[0], h1 = h0 | xv[1], h2 = h1 | xv[2], h3 = h2 | xv[3];
-        MaskT before = __shfl_up_sync(0xffffffffu, warp_prefix_or<MaskT>(hiL ? h3 : static_cast<MaskT>(0), lane), 1);
-        if (lane <= 16) before = 0;
-        if (hiL) {
-          const int q = 4 * (lane - 16);
-          ms.preh[q + 0] = before | h0;
-          ms.preh[q + 1] = before | h1;
-          ms.preh[q + 2] = before | h2;
-          ms.preh[q + 3] = before | h3;
-        }
-      }
-      {  // sufl[c] = OR bm[c+1..63] (lanes 0..15 hold columns 0..63)
-        const bool loL = lane < 16;
-        const MaskT u2 = xv[3], u1 = u2 | xv[2], u0 = u1 | xv[1];
-        MaskT after = __shfl_down_sync(0xffffffffu, warp_suffix_or<MaskT>(loL ? static_cast<MaskT>(u0 | xv[0])
-                                                                              : static_cast<MaskT>(0), lane), 1);
-        if (lane >= 15) after = 0;
-        if (loL) {
-          ms.sufl[4 * lane + 0] = after | u0;
-          ms.sufl[4 * lane + 1] = after | u1;
-          ms.sufl[4 * lane + 2] = after | u2;
-          ms.sufl[4 * lane + 3] = after;
-        }
-      }
-      if constexpr (kTable) {
-        if (kind == 0) {
-          // the query tile's own prefix / suffix ORs, for this item's table tiles
-          const MaskT bm0 = __shfl_sync(0xffffffffu, xv[0], 0);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            sm.pfxq[4 * lane + e] = static_cast<MaskT>(bm0 | pre_v[e]);
-            sm.sfxq[4 * lane + e] = suf_v[e];
-          }
-          mid_b = 0;
-          mid_a = 0;
-        } else {
-          // the distinct carries of the tile's rows, then one table row per distinct carry
-          const MaskT bm0 = __shfl_sync(0xffffffffu, xv[0], 0);
-          if (kind == 2) mid_a |= bm0;
-          const MaskT mid = kind == 1 ? mid_b : mid_a;
-          __syncwarp();
-          uint32_t pres_lo = 0, pres_hi = 0;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int r = lane + 32 * e;
-            const MaskT cy = static_cast<MaskT>(mid | (kind == 1 ? sm.pfxq[r] : sm.sfxq[r]));
-            const int key = popc_m(cy);
-            if (key < 32) pres_lo |= 1u << key; else pres_hi |= 1u << (key - 32);
-          }
-          pres_lo = __reduce_or_sync(0xffffffffu, pres_lo);
-          pres_hi = __reduce_or_sync(0xffffffffu, pres_hi);
-          bool ok = true;
-          if (ti.u >= 1) ok = mbar_wait(&sm.t_empty, static_cast<uint32_t>((ti.u - 1) & 1), abort_flag, err);
-          if (!__all_sync(0xffffffffu, ok)) break;
-          // rows with the same popcount hold the same carry (the carries of a tile are nested)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int r = lane + 32 * e;
-            const MaskT cy = static_cast<MaskT>(mid | (kind == 1 ? sm.pfxq[r] : sm.sfxq[r]));
-            sm.ykey[popc_m(cy)] = cy;
-          }
-          __syncwarp();
-          for (int key = 0; key < kTblRows; ++key) {
-            const bool present = key < 32 ? ((pres_lo >> key) & 1u) : ((pres_hi >> (key - 32)) & 1u);
-            if (!present) continue;
-            const MaskT cy = sm.ykey[key];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int c = lane + 32 * e;
-              const MaskT Rc = kind == 1 ? static_cast<MaskT>(ms.suf[c] | cy) : static_cast<MaskT>(cy | ms.pre[c]);
-              sm.tbl.w[key][c] = sm.lg[lg_index(s, popc_m(Rc))];
-            }
-          }
-          if (kind == 1) mid_b |= static_cast<MaskT>(bm0 | __shfl_sync(0xffffffffu, suf_v[0], 0));
-          else mid_a |= __shfl_sync(0xffffffffu, pre_v[3], 31);
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.t_full);
-        }
+      if (lane == 0) {
+        ms.bm[kTile] = x128;
+        ms.valid = 1;
+        ms.kind = ti.kind();
+        ms.first = ti.first() ? 1 : 0;
+        ms.last = ti.last() ? 1 : 0;
+        ms.x = ti.x;
+        if (ti.first() && ti.bad_window) atomicOr(err, PLSH_DEVERR_WINDOW);
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.m_full[st]);
+      if (lane == 0) mbar_arrive(&sm.m_full[z][st]);
+      g_end = ti.g + 1;
       ti.next();
+      if (nx.valid) nx.next();
+#pragma unroll
+      for (int e = 0; e < 4; ++e) xv[e] = nv[e];
+      x128 = n128;
     }
-  } else if (warp < kSoftmaxWarps) {
-    // ------------------------------------------------------------ softmax
-    const int half = warp >= 4 ? 1 : 0;
+    // the end marker for the softmax warps
+    if (ok && !*abort_flag) {
+      const int st = g_end % kMaskStages;
+      ok = g_end < kMaskStages ||
+           mbar_wait(&sm.m_empty[z][st], (static_cast<uint32_t>(g_end / kMaskStages) & 1u) ^ 1u, abort_flag, err);
+      if (__all_sync(0xffffffffu, ok) && lane == 0) {
+        sm.m[z][st].valid = 0;
+        mbar_arrive(&sm.m_full[z][st]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax of slot (warp - 4) / 4
+    const int z = (warp - 4) >> 2;
     const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;   // row within the tile == TMEM lane
+    const int r = quarter * 32 + lane;  // row within the tile == TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t col_off = static_cast<uint32_t>(kHalf * half);
+    const uint32_t s_base = tmem + lane_off + kColS + 128u * z;
+    const uint32_t o_base = tmem + lane_off + kColO + 128u * z;
     const float sc = 1.4426950408889634f / sqrtf(static_cast<float>(kD));
+    const float cs = 8388608.0f + static_cast<float>(s);  // 2^23 + s
     float m2 = -INFINITY, l = 0.0f;
     MaskT Y = 0, Z = 0;
-    // epilogue still owed for the previous item
-    // (always the item just before the current tile's item: index x - gridDim.x, tile g - 1, count k - 1)
-    bool pend = false;
-    float pend_l = 0.0f, pend_m = 0.0f;
-    auto epilogue = [&](int pend_x, int pend_g, int pend_k) -> bool {
-      const int BT = prm.B * prm.T;
-      const int pend_h = (H <= kMaxSortedHeads) ? static_cast<int>(sm.order[pend_x / BT]) : pend_x / BT;
-      const int rem = pend_x % BT;
-      const int pend_b = rem / prm.T;
-      const int pend_i0 = (rem % prm.T) * kTile;
-      bool okw = mbar_wait(&sm.pv_done[pend_g & 1], static_cast<uint32_t>(pend_g >> 1) & 1u, abort_flag, err);
-      okw = __all_sync(0xffffffffu, okw && mbar_wait(&sm.xsum[pend_k & 1], static_cast<uint32_t>(pend_k >> 1) & 1u,
-                                                     abort_flag, err));
-      if (!okw) return false;
-      tc_fence_after();
-      const float ltot = pend_l + sm.psum[pend_k & 1][half ^ 1][r];
-      const int i = pend_i0 + r;
-      const float inv = 1.0f / ltot;
-      const uint32_t ob = tmem + lane_off + kColO + 128u * static_cast<uint32_t>(pend_k & 1) + col_off;
-      __nv_bfloat16* orow = O + ((static_cast<size_t>(pend_b) * H + pend_h) * n + (i < n ? i : 0)) * kD + col_off;
-#pragma unroll 1
-      for (int q2 = 0; q2 < 2; ++q2) {
-        uint32_t raw[32];
-        tmem_ld32(ob + 32u * q2, raw);
-        tmem_wait_ld();
-        if (i < n) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * q2);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            uint32_t pk[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-              pk[u] = pack_bf16x2(__uint_as_float(raw[8 * e + 2 * u]) * inv, __uint_as_float(raw[8 * e + 2 * u + 1]) * inv);
-            dst[e] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          }
-        }
-      }
-      tc_fence_before();
-      if (i < n) {
-        if (half == 0)
-          row_sum[(static_cast<size_t>(pend_b) * H + pend_h) * n + i] =
-              (log2f(ltot) + pend_m) * 0.6931471805599453f - logf(static_cast<float>(s));
-      }
-      pend = false;
-      return true;
-    };
-    TileIter ti;
-    ti.start(&prm, sm.order);
-    bool ok = true;
-    while (ti.valid) {
-      const int g = ti.g;
-      const int st = g % kStages;
-      const int kind = ti.kind();
-      if (ti.first()) {
+    int items_done = 0;
+    for (int g = 0;; ++g) {
+      const int st = g % kMaskStages;
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.m_full[z][st], static_cast<uint32_t>(g / kMaskStages) & 1u,
+                                             abort_flag, err)))
+        break;
+      const MaskStage<MaskT>& ms = sm.m[z][st];
+      if (!ms.valid) break;
+      const int kind = ms.kind, first = ms.first, last = ms.last, tx = ms.x;
+      if (first) {
         m2 = -INFINITY;
         l = 0.0f;
-        if (ti.bad_window && r == 0 && half == 0) atomicOr(err, PLSH_DEVERR_WINDOW);
       }
-      ok = mbar_wait(&sm.m_full[st], static_cast<uint32_t>(g / kStages) & 1u, abort_flag, err);
-      ok = ok && mbar_wait(&sm.s_full[g & 1], static_cast<uint32_t>(g >> 1) & 1u, abort_flag, err);
-      if (kTable && kind != 0) ok = ok && mbar_wait(&sm.t_full, static_cast<uint32_t>(ti.u & 1), abort_flag, err);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
+      // weights that need only the masks: the diagonal's own block and its carries
+      uint32_t cnt[8];
+      MaskT lo = 0, hi = 0;
+      if (kind == 0) diag_scan<MaskT, kCausal>(ms, quarter, r, s, cnt, lo, hi);
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[z], static_cast<uint32_t>(g & 1), abort_flag, err)))
+        break;
       tc_fence_after();
-      float x[kHalf];
-      {
-        const uint32_t base = tmem + lane_off + kColS + 128u * static_cast<uint32_t>(g & 1) + col_off;
-        uint32_t raw[2][32];
-        tmem_ld32(base, raw[0]);
-        tmem_ld32(base + 32u, raw[1]);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          x[e] = __uint_as_float(raw[0][e]);
-          x[32 + e] = __uint_as_float(raw[1][e]);
-        }
-      }
-      const MaskStage<MaskT>& ms = sm.m[st];
-      if (kind == 2) Z |= ms.bm[0];   // now OR over (i, j0]
-      if constexpr (kTable) {
-        if (kind != 0) {
-          const MaskT cy = kind == 1 ? Y : Z;
-          logits_from_table(x, &sm.tbl.w[popc_m(cy)][col_off], sc);
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.t_empty);
-        } else {
-          logits_by_scan<MaskT, kCausal>(x, ms, sm.lg, kind, r, half, s, sc, Y, Z);
-        }
-      } else {
-        logits_by_scan<MaskT, kCausal>(x, ms, sm.lg, kind, r, half, s, sc, Y, Z);
-      }
-      // carries past this tile
-      if (kind == 0) {
-        Y = static_cast<MaskT>(ms.bm[0] | ms.pre[r]);       // OR over [i0, i]
-        Z = kCausal ? static_cast<MaskT>(0) : ms.suf[r];     // OR over (i, i0 + 127]
-      } else if (kind == 1) {
-        Y = static_cast<MaskT>(Y | ms.bm[0] | ms.suf[0]);   // OR over [j0, i]
-      } else {
-        Z = static_cast<MaskT>(Z | ms.pre[kTile - 1]);      // OR over (i, j0 + 127]
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.m_empty[st]);
 
-      // ---- tile maximum (both halves) and reference update
-      float mx[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) mx[u] = x[u];
-#pragma unroll
-      for (int c = 8; c < kHalf; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
-      float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-      sm.pmax[g & 1][half][r] = mt;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.xmax[g & 1]);
-      ok = __all_sync(0xffffffffu, mbar_wait(&sm.xmax[g & 1], static_cast<uint32_t>(g >> 1) & 1u, abort_flag, err));
-      if (!ok) break;
-      mt = fmaxf(mt, sm.pmax[g & 1][half ^ 1][r]);
+      // ---- pass 1: the tile maximum of S over the 16-key chunks that can carry weight (when
+      // causal, the diagonal tile's chunks past the warp's own block cannot)
+      const int n_live = (kCausal && kind == 0) ? 2 * quarter + 2 : kTile / 16;
+      float mraw = -INFINITY;
+#pragma unroll 1
+      for (int ch = 0; ch < n_live; ch += 2) {
+        uint32_t sv[32];
+        tmem_ld32(s_base + 16u * ch, sv);
+        tmem_wait_ld();
+        mraw = max32(sv, mraw);
+      }
+      const float mt = mraw * sc;
+
+      // ---- reference update; O is rescaled in place (s_full(g) fired after PV(g-1) had completed)
       float alpha = 1.0f;
       bool need_rescale = false;
       if (mt > m2 + kRescaleThreshold) {
@@ -817,73 +730,127 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         }
         m2 = mt;
       }
-      const float neg_m = (m2 == -INFINITY) ? 0.0f : -m2;
-
-      // ---- rescale this half of the item's O when some row of the warp moved its reference
+      const float neg_m = -m2;
       if (__any_sync(0xffffffffu, need_rescale)) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&sm.pv_done[(g - 1) & 1], static_cast<uint32_t>((g - 1) >> 1) & 1u,
-                                               abort_flag, err));
-        if (!ok) break;
-        tc_fence_after();
 #pragma unroll 1
-        for (int q4 = 0; q4 < 4; ++q4) {
+        for (int q4 = 0; q4 < 8; ++q4) {
           uint32_t raw[16];
-          const uint32_t addr = tmem + lane_off + kColO + 128u * static_cast<uint32_t>(ti.k & 1) + col_off + 16u * q4;
-          tmem_ld16(addr, raw);
+          tmem_ld16(o_base + 16u * q4, raw);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 16; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * alpha);
-          tmem_st16(addr, raw);
+          tmem_st16(o_base + 16u * q4, raw);
         }
-        tmem_wait_st();
       }
 
-      // ---- P = 2^(x - m) as bf16 over the first 64 columns of S_g, partial row sum
-      const uint32_t p_base = tmem + lane_off + kColS + 128u * static_cast<uint32_t>(g & 1) + col_off / 2;
-      float ls[8];
+      // ---- pass 2: P = c 2^(S sc - m) chunk by chunk; P of keys [16ch, 16ch + 16) goes to columns
+      // [8ch, 8ch + 8), over S columns already read
+      const MaskT Zc = static_cast<MaskT>(Z | ms.bm[0]);
+      float lsum = 0.0f;
+#pragma unroll 1
+      for (int ch = 0; ch < kTile / 16; ++ch) {
+        uint32_t pk[8];
+        if (ch >= n_live) {
 #pragma unroll
-      for (int u = 0; u < 8; ++u) ls[u] = 0.0f;
+          for (int e = 0; e < 8; ++e) pk[e] = 0u;
+        } else {
+          uint32_t sv[16];
+          tmem_ld16(s_base + 16u * ch, sv);
+          tmem_wait_ld();
+          if (kind == 0 && (ch >> 1) == quarter) {
+            // the warp's own block on the diagonal: counts from the scan
+            uint32_t c4[4];
 #pragma unroll
-      for (int q2 = 0; q2 < 2; ++q2) {
-        uint32_t packed[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const float p0 = ex2_approx(x[32 * q2 + e] + neg_m);
-          const float p1 = ex2_approx(x[32 * q2 + e + 1] + neg_m);
-          ls[e & 7] += p0;
-          ls[(e + 1) & 7] += p1;
-          packed[e >> 1] = pack_bf16x2(p0, p1);
+            for (int u = 0; u < 4; ++u) c4[u] = (ch & 1) ? cnt[4 + u] : cnt[u];
+            lsum += p16_counts(sv, c4, sc, neg_m, pk);
+          } else {
+            // below: Y | suf[c]; above: Z | bm[0] | pre[c]; diagonal: lo | dq[c] below the
+            // warp's block, hi | dq[c] above it
+            const MaskT* km = kind == 1 ? ms.suf : (kind == 2 ? ms.pre : ms.dq[quarter]);
+            const MaskT carry = kind == 1 ? Y : (kind == 2 ? Zc : ((ch >> 1) < quarter ? lo : hi));
+            lsum += p16_carry<MaskT>(sv, km + 16 * ch, carry, sc, neg_m, cs, pk);
+          }
         }
-        tmem_st16(p_base + 16u * q2, packed);
+        tmem_st8(s_base + 8u * ch, pk);
       }
+      if (kind == 1) {
+        Y = static_cast<MaskT>(Y | ms.bm[0] | ms.suf[0]);  // OR over [j0, i]
+      } else if (kind == 2) {
+        Z = static_cast<MaskT>(Zc | ms.pre[kTile - 1]);    // OR over (i, j0 + 127]
+      } else {
+        Y = static_cast<MaskT>(ms.bm[0] | ms.pre[r]);      // OR over [i0, i]
+        if (!kCausal) Z = ms.suf[r];                        // OR over (i, i0 + 127]
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.m_empty[z][st]);
       tmem_wait_st();
-      l = l * alpha + (((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7])));
+      l = l * alpha + lsum;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.p_full[g & 1]);
+      if (lane == 0) mbar_arrive(&sm.p_full[z]);
 
-      // ---- the previous item's epilogue, now that its last PV has had a tile's time to finish
-      if (pend && !epilogue(ti.x - static_cast<int>(gridDim.x), g - 1, ti.k - 1)) {
-        ok = false;
-        break;
+      // ---- the item's epilogue: O / l, stored four rows at a time by each lane quad
+      if (last) {
+        const bool o_ok = mbar_wait(&sm.o_full[z], static_cast<uint32_t>(items_done & 1), abort_flag, err);
+        if (!__all_sync(0xffffffffu, o_ok)) break;
+        ++items_done;
+        tc_fence_after();
+        const int BT = prm.B * prm.T;
+        const int hh = (H <= kMaxSortedHeads) ? static_cast<int>(sm.order[tx / BT]) : tx / BT;
+        const int rem = tx % BT;
+        const int bb = rem / prm.T, i0 = (rem % prm.T) * kTile;
+        const float inv = 1.0f / l;
+        const int p4 = lane & 3;
+        const int quad_row = quarter * 32 + (lane & ~3);  // first of the quad's four rows
+        __nv_bfloat16* obase = O + (static_cast<size_t>(bb) * H + hh) * static_cast<size_t>(n) * kD;
+#pragma unroll 1
+        for (int blk = 0; blk < 4; ++blk) {
+          uint32_t raw[32];
+          tmem_ld32(o_base + 32u * blk, raw);
+          tmem_wait_ld();
+          uint32_t a[4][4];  // [16-byte chunk][word] of this row's 32 columns
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+              a[c][w] = pack_bf16x2(__uint_as_float(raw[8 * c + 2 * w]) * inv,
+                                    __uint_as_float(raw[8 * c + 2 * w + 1]) * inv);
+          // 4x4 transpose of 16-byte chunks inside the quad: lane p then holds chunk p of the quad's rows
+#pragma unroll
+          for (int msk = 2; msk >= 1; msk >>= 1) {
+            const bool lo = (p4 & msk) == 0;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              if (c & msk) continue;
+#pragma unroll
+              for (int w = 0; w < 4; ++w) {
+                const uint32_t send = lo ? a[c | msk][w] : a[c][w];
+                const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, msk);
+                if (lo) a[c | msk][w] = recv;
+                else a[c][w] = recv;
+              }
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int row = i0 + quad_row + e;
+            if (row < n)
+              *reinterpret_cast<uint4*>(obase + static_cast<size_t>(row) * kD + 32 * blk + 8 * p4) =
+                  make_uint4(a[e][0], a[e][1], a[e][2], a[e][3]);
+          }
+        }
+        tc_fence_before();
+        const int i = i0 + r;
+        if (i < n)
+          row_sum[(static_cast<size_t>(bb) * H + hh) * n + i] =
+              (log2f(l) + m2) * 0.6931471805599453f - logf(static_cast<float>(s));
       }
-      if (ti.last()) {
-        sm.psum[ti.k & 1][half][r] = l;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.xsum[ti.k & 1]);
-        pend = true;
-        pend_l = l;
-        pend_m = m2;
-      }
-      ti.next();
     }
-    // the CTA's last item: ti has moved past it
-    if (ok && pend) epilogue(ti.x - static_cast<int>(gridDim.x), ti.g - 1, ti.k - 1);
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kWarpMma) {
+  if (warp == 1) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
@@ -950,7 +917,8 @@ int launch_tc_typed(const AttnArgs& a, cudaStream_t st) {
   const size_t smem = sizeof(TcSmem<MaskT>) + 1024;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_tc_kernel)");
-  const int grid = prm.items < sm_count() ? prm.items : sm_count();
+  const int want = ceil_div(prm.items, kSlots);
+  const int grid = want < sm_count() ? want : sm_count();
   kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, prm, a.sigma, a.table, static_cast<const MaskT*>(a.bmask),
                                      static_cast<__nv_bfloat16*>(a.O), a.row_sum, a.err);
   e = cudaGetLastError();
