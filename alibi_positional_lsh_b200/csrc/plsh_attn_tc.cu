@@ -482,9 +482,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, 1);
       TileIter st_it[kSlots], pv_it[kSlots];
+      uint64_t q_desc[kSlots], k_desc[kSlots], v_desc[kSlots];
       for (int z = 0; z < kSlots; ++z) {
         st_it[z].start(&prm, sm.order, z);
         pv_it[z].start(&prm, sm.order, z);
+        q_desc[z] = smem_desc_sw128(smem_u32(sm.slot[z].q), 16, 1024);
+        k_desc[z] = smem_desc_sw128(smem_u32(sm.slot[z].k), 16, 1024);
+        v_desc[z] = smem_desc_sw128(smem_u32(sm.slot[z].v), kChunkBytes, 1024);
       }
       uint64_t idle_since = 0;
       uint32_t spins = 0;
@@ -494,41 +498,38 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         for (int z = 0; z < kSlots; ++z) {
           TileIter& si = st_it[z];
           TileIter& pi = pv_it[z];
-          if (si.valid && si.g == pi.g && (!si.first() || mbar_test_wait(&sm.q_full[z], si.k & 1)) &&
-              mbar_test_wait(&sm.k_full[z], si.g & 1)) {
-            tc_fence_after();
-            const uint32_t q_addr = smem_u32(sm.slot[z].q);
-            const uint32_t k_addr = smem_u32(sm.slot[z].k);
-            const uint32_t d_tmem = tmem + kColS + 128u * z;
-#pragma unroll
-            for (int kk = 0; kk < kD / 16; ++kk) {
-              const uint32_t off = static_cast<uint32_t>((kk >> 2) * kChunkBytes + (kk & 3) * 32);
-              mma_ss(d_tmem, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024),
-                     idesc_qk, kk > 0 ? 1u : 0u);
-            }
-            mma_commit(&sm.s_full[z]);
-            mma_commit(&sm.k_empty[z]);
-            if (si.last()) mma_commit(&sm.q_empty[z]);
-            si.next();
-            progress = true;
-          }
+          // PV first: it frees the slot's S columns for the next S
           if (pi.valid && pi.g < si.g && mbar_test_wait(&sm.p_full[z], pi.g & 1) &&
               mbar_test_wait(&sm.v_full[z], pi.g & 1)) {
             tc_fence_after();
-            const uint32_t v_addr = smem_u32(sm.slot[z].v);
             const uint32_t p_tmem = tmem + kColS + 128u * z;
             const uint32_t o_tmem = tmem + kColO + 128u * z;
 #pragma unroll
             for (int kk = 0; kk < kTile / 16; ++kk) {
               // keys 16kk..16kk+15: P at columns 8kk..8kk+7; the keys are two 8-row groups of the
               // MN-major V tile, whose two d halves sit kChunkBytes apart
-              mma_ts(o_tmem, p_tmem + 8u * kk,
-                     smem_desc_sw128(v_addr + kk * 2048, kChunkBytes, 1024), idesc_pv,
+              mma_ts(o_tmem, p_tmem + 8u * kk, v_desc[z] + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
                      (pi.it > 0 || kk > 0) ? 1u : 0u);
             }
             mma_commit(&sm.v_empty[z]);
             if (pi.last()) mma_commit(&sm.o_full[z]);
             pi.next();
+            progress = true;
+          }
+          if (si.valid && si.g == pi.g && (!si.first() || mbar_test_wait(&sm.q_full[z], si.k & 1)) &&
+              mbar_test_wait(&sm.k_full[z], si.g & 1)) {
+            tc_fence_after();
+            const uint32_t d_tmem = tmem + kColS + 128u * z;
+#pragma unroll
+            for (int kk = 0; kk < kD / 16; ++kk) {
+              // the descriptors' start address field counts 16-byte units
+              const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
+              mma_ss(d_tmem, q_desc[z] + off, k_desc[z] + off, idesc_qk, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(&sm.s_full[z]);
+            mma_commit(&sm.k_empty[z]);
+            if (si.last()) mma_commit(&sm.q_empty[z]);
+            si.next();
             progress = true;
           }
         }
