@@ -52,6 +52,13 @@ def _load() -> ctypes.CDLL:
     lib.plsh_attention_fwd.restype = i32
     lib.plsh_attention_fwd.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, i32, vp, vp, vp, i32,
                                        vp, vp, vp, vp]
+    lib.plsh_varlen_scratch_bytes.restype = ctypes.c_size_t
+    lib.plsh_varlen_scratch_bytes.argtypes = [i32, i32, i32]
+    lib.plsh_varlen_spans.restype = i32
+    lib.plsh_varlen_spans.argtypes = [vp, i32, i32, i32, i32, vp, vp]
+    lib.plsh_attention_varlen_fwd.restype = i32
+    lib.plsh_attention_varlen_fwd.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, i32, vp, vp, vp, i32,
+                                              vp, ctypes.c_size_t, vp, vp, vp, vp]
     return lib
 
 
@@ -119,6 +126,28 @@ def plsh_attention_fwd(Q, K, V, dtype: int, B: int, H: int, H_kv: int, n: int, d
                                    _dev_ptr(tile_span_dev, "tile_span_dev"), _dev_ptr(bmask_dev, "bmask_dev"),
                                    int(causal), _dev_ptr(O, "O"), _dev_ptr(row_sum, "row_sum"),
                                    _dev_ptr(err_dev, "err_dev"), _stream_ptr(stream)))
+
+
+def plsh_varlen_scratch_bytes(H: int, s: int, n: int) -> int:
+    return int(_lib.plsh_varlen_scratch_bytes(H, s, n))
+
+
+def plsh_varlen_spans(ids_dev, H: int, s: int, n: int, causal: int, spans_dev, stream=None) -> None:
+    _check(_lib.plsh_varlen_spans(_dev_ptr(ids_dev, "ids_dev"), H, s, n, int(causal),
+                                  _dev_ptr(spans_dev, "spans_dev"), _stream_ptr(stream)))
+
+
+def plsh_attention_varlen_fwd(Q, K, V, dtype: int, B: int, H: int, H_kv: int, n: int, d: int, sigma_dev, s: int,
+                              table_dev, ids_dev, bmask_dev, causal: int, scratch_dev, O, row_sum, err_dev,
+                              stream=None) -> None:
+    nbytes = 0 if scratch_dev is None else scratch_dev.numel() * scratch_dev.element_size()
+    _check(_lib.plsh_attention_varlen_fwd(_dev_ptr(Q, "Q"), _dev_ptr(K, "K"), _dev_ptr(V, "V"), dtype, B, H, H_kv,
+                                          n, d, _dev_ptr(sigma_dev, "sigma_dev"), s,
+                                          _dev_ptr(table_dev, "table_dev"), _dev_ptr(ids_dev, "ids_dev"),
+                                          _dev_ptr(bmask_dev, "bmask_dev"), int(causal),
+                                          _dev_ptr(scratch_dev, "scratch_dev"), ctypes.c_size_t(nbytes),
+                                          _dev_ptr(O, "O"), _dev_ptr(row_sum, "row_sum"),
+                                          _dev_ptr(err_dev, "err_dev"), _stream_ptr(stream)))
 
 
 def decode_device_error(word: int) -> list:

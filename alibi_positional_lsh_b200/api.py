@@ -6,7 +6,8 @@ with torch) and runs the whole path:
   a2 plsh_sample_bins  (K1)     -> bin ids
   a3 plsh_window       (K2)     -> b_max, tile windows, boundary masks
   a4 plsh_attention_fwd (K3)    -> O, row_sum
-All arithmetic of a2..a4 runs in libplsh's CUDA kernels.
+  a5 plsh_attention_varlen_fwd (K4, the per-sample comparator) -> the same O, row_sum
+All arithmetic of a2..a5 runs in libplsh's CUDA kernels.
 """
 from __future__ import annotations
 
@@ -16,7 +17,8 @@ import numpy as np
 import torch
 
 from . import (PLSH_BF16, PLSH_F32, PLSH_TILE, PlshError, decode_device_error, plsh_attention_fwd,
-               plsh_draw_table, plsh_sample_bins, plsh_window)
+               plsh_attention_varlen_fwd, plsh_draw_table, plsh_sample_bins, plsh_varlen_scratch_bytes,
+               plsh_window)
 
 
 class PlshForward:
@@ -49,6 +51,7 @@ class PlshForward:
         self.err = torch.zeros((4,), dtype=torch.int32, device=dev)
         self.O = torch.empty((B, H, n, d), dtype=dtype, device=dev)
         self.row_sum = torch.empty((B, H, n), dtype=torch.float32, device=dev)
+        self.scratch = None  # per-hash windows of the comparator, allocated on first use
 
     # a1 + a2 + a3
     def prepare(self, stream: Optional[torch.cuda.Stream] = None, table: Optional[np.ndarray] = None) -> None:
@@ -85,6 +88,25 @@ class PlshForward:
                            self.spans, self.bmask, int(self.causal), self.O, self.row_sum, self.err, st)
         return self.O, self.row_sum
 
+    # a5
+    def attend_varlen(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                      stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+        """The per-sample comparator (K4): the same T~ from s block-diagonal attentions."""
+        B, H, H_kv, n, d = self.B, self.H, self.H_kv, self.n, self.d
+        if q.shape != (B, H, n, d) or k.shape != (B, H_kv, n, d) or v.shape != (B, H_kv, n, d):
+            raise ValueError("q/k/v shapes do not match the plan")
+        for t, nm in ((q, "q"), (k, "k"), (v, "v")):
+            if t.dtype != self.dtype or t.device != self.O.device:
+                raise ValueError(f"{nm} must be {self.dtype} on {self.O.device}")
+        if self.scratch is None:
+            nbytes = plsh_varlen_scratch_bytes(H, self.s, n)
+            self.scratch = torch.empty((nbytes // 4,), dtype=torch.int32, device=self.O.device)
+        st = torch.cuda.current_stream() if stream is None else stream
+        plsh_attention_varlen_fwd(q, k, v, self.dtype_code, B, H, H_kv, n, d, self.sigma_dev, self.s,
+                                  self.table_dev, self.ids, self.bmask, int(self.causal), self.scratch, self.O,
+                                  self.row_sum, self.err, st)
+        return self.O, self.row_sum
+
     def __call__(self, q, k, v, stream=None, table=None):
         self.prepare(stream, table)
         return self.attend(q, k, v, stream)
@@ -92,15 +114,18 @@ class PlshForward:
     def run_host(self, q_host: torch.Tensor, k_host: torch.Tensor, v_host: torch.Tensor,
                  q_dev: torch.Tensor, k_dev: torch.Tensor, v_dev: torch.Tensor,
                  o_host: torch.Tensor, rs_host: Optional[torch.Tensor] = None,
-                 stream=None) -> None:
-        """End to end from (pinned) host inputs to host outputs on one stream."""
+                 stream=None, varlen: bool = False) -> None:
+        """End to end from (pinned) host inputs to host outputs on one stream (varlen: the comparator)."""
         st = torch.cuda.current_stream() if stream is None else stream
         with torch.cuda.stream(st):
             q_dev.copy_(q_host, non_blocking=True)
             k_dev.copy_(k_host, non_blocking=True)
             v_dev.copy_(v_host, non_blocking=True)
             self.prepare(st)
-            self.attend(q_dev, k_dev, v_dev, st)
+            if varlen:
+                self.attend_varlen(q_dev, k_dev, v_dev, st)
+            else:
+                self.attend(q_dev, k_dev, v_dev, st)
             o_host.copy_(self.O, non_blocking=True)
             if rs_host is not None:
                 rs_host.copy_(self.row_sum, non_blocking=True)

@@ -27,6 +27,7 @@ SOURCES = [
     "plsh_window.cu",
     "plsh_attn_simt.cu",
     "plsh_attn_tc.cu",
+    "plsh_varlen.cu",
 ]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -64,26 +64,83 @@ extern "C" int plsh_window(const int32_t* ids_dev, int H, int s, int n, int caus
                              static_cast<cudaStream_t>(stream));
 }
 
-extern "C" int plsh_attention_fwd(const void* Q, const void* K, const void* V, int dtype, int B, int H,
-                                  int H_kv, int n, int d, const double* sigma_dev, int s,
-                                  const double* table_dev, const int32_t* tile_span_dev,
-                                  const void* bmask_dev, int causal, void* O, float* row_sum,
-                                  uint32_t* err_dev, void* stream) {
-  const char* fn = "plsh_attention_fwd";
-  if (int rc = plsh::check_sizes(fn, H, s, n)) return rc;
+namespace plsh {
+namespace {
+
+// Checks shared by the two attention entry points.
+int check_attention(const char* fn, const void* Q, const void* K, const void* V, int dtype, int B, int H,
+                    int H_kv, int n, int d, int s, int causal, const void* bmask_dev, const void* O,
+                    const float* row_sum, const uint32_t* err_dev) {
+  if (int rc = check_sizes(fn, H, s, n)) return rc;
   if (B < 1 || B > 65535) return fail(PLSH_ERR_INVALID_ARG, "%s: need 1 <= B <= 65535 (B=%d)", fn, B);
   if (H_kv < 1 || H % H_kv != 0)
     return fail(PLSH_ERR_INVALID_ARG, "%s: H_kv must divide H (H=%d H_kv=%d)", fn, H, H_kv);
   if (causal != 0 && causal != 1) return fail(PLSH_ERR_INVALID_ARG, "%s: causal must be 0 or 1", fn);
   if (dtype != PLSH_BF16 && dtype != PLSH_F32) return fail(PLSH_ERR_UNSUPPORTED, "%s: dtype %d", fn, dtype);
   if (d != 64 && d != 128) return fail(PLSH_ERR_UNSUPPORTED, "%s: head dim %d (64 or 128 supported)", fn, d);
-  if (!Q || !K || !V || !O || !row_sum || !tile_span_dev || !bmask_dev || !err_dev)
+  if (!Q || !K || !V || !O || !row_sum || !bmask_dev || !err_dev)
     return fail(PLSH_ERR_INVALID_ARG, "%s: null pointer", fn);
-  if (!plsh::aligned16(Q) || !plsh::aligned16(K) || !plsh::aligned16(V) || !plsh::aligned16(O))
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
     return fail(PLSH_ERR_INVALID_ARG, "%s: Q, K, V and O must be 16-byte aligned", fn);
+  return PLSH_OK;
+}
+
+int launch_attention(const AttnArgs& a, cudaStream_t st) {
+  if (a.dtype == PLSH_BF16 && a.d == 128) return launch_attention_tc(a, st);
+  return launch_attention_simt(a, st);
+}
+
+}  // namespace
+}  // namespace plsh
+
+extern "C" int plsh_attention_fwd(const void* Q, const void* K, const void* V, int dtype, int B, int H,
+                                  int H_kv, int n, int d, const double* sigma_dev, int s,
+                                  const double* table_dev, const int32_t* tile_span_dev,
+                                  const void* bmask_dev, int causal, void* O, float* row_sum,
+                                  uint32_t* err_dev, void* stream) {
+  const char* fn = "plsh_attention_fwd";
+  if (int rc = plsh::check_attention(fn, Q, K, V, dtype, B, H, H_kv, n, d, s, causal, bmask_dev, O, row_sum,
+                                     err_dev))
+    return rc;
+  if (!tile_span_dev) return fail(PLSH_ERR_INVALID_ARG, "%s: null pointer", fn);
   plsh::AttnArgs a{Q, K, V, dtype, B, H, H_kv, n, d, s, causal, sigma_dev, table_dev,
-                   tile_span_dev, bmask_dev, O, row_sum, err_dev};
+                   tile_span_dev, bmask_dev, O, row_sum, err_dev, 0};
+  return plsh::launch_attention(a, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" size_t plsh_varlen_scratch_bytes(int H, int s, int n) {
+  if (H < 1 || s < 1 || n < 1) return 0;
+  return static_cast<size_t>(H) * static_cast<size_t>(s) * static_cast<size_t>(plsh::ceil_div(n, PLSH_TILE)) * 2 *
+         sizeof(int32_t);
+}
+
+extern "C" int plsh_varlen_spans(const int32_t* ids_dev, int H, int s, int n, int causal, int32_t* spans_dev,
+                                 void* stream) {
+  const char* fn = "plsh_varlen_spans";
+  if (int rc = plsh::check_sizes(fn, H, s, n)) return rc;
+  if (causal != 0 && causal != 1) return fail(PLSH_ERR_INVALID_ARG, "%s: causal must be 0 or 1", fn);
+  if (!ids_dev || !spans_dev) return fail(PLSH_ERR_INVALID_ARG, "%s: null pointer", fn);
+  return plsh::launch_varlen_spans(ids_dev, H, s, n, causal, spans_dev, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int plsh_attention_varlen_fwd(const void* Q, const void* K, const void* V, int dtype, int B, int H,
+                                         int H_kv, int n, int d, const double* sigma_dev, int s,
+                                         const double* table_dev, const int32_t* ids_dev, const void* bmask_dev,
+                                         int causal, void* scratch_dev, size_t scratch_bytes, void* O,
+                                         float* row_sum, uint32_t* err_dev, void* stream) {
+  const char* fn = "plsh_attention_varlen_fwd";
+  if (int rc = plsh::check_attention(fn, Q, K, V, dtype, B, H, H_kv, n, d, s, causal, bmask_dev, O, row_sum,
+                                     err_dev))
+    return rc;
+  if (!ids_dev || !scratch_dev) return fail(PLSH_ERR_INVALID_ARG, "%s: null pointer", fn);
+  if (!plsh::aligned16(scratch_dev)) return fail(PLSH_ERR_INVALID_ARG, "%s: scratch must be 16-byte aligned", fn);
+  const size_t need = plsh_varlen_scratch_bytes(H, s, n);
+  if (scratch_bytes < need)
+    return fail(PLSH_ERR_INVALID_ARG, "%s: scratch holds %zu bytes, %zu needed", fn, scratch_bytes, need);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (dtype == PLSH_BF16 && d == 128) return plsh::launch_attention_tc(a, st);
-  return plsh::launch_attention_simt(a, st);
+  int32_t* spans = static_cast<int32_t*>(scratch_dev);
+  if (int rc = plsh::launch_varlen_spans(ids_dev, H, s, n, causal, spans, st)) return rc;
+  plsh::AttnArgs a{Q, K, V, dtype, B, H, H_kv, n, d, s, causal, sigma_dev, table_dev,
+                   spans, bmask_dev, O, row_sum, err_dev, 1};
+  return plsh::launch_attention(a, st);
 }

@@ -69,7 +69,7 @@ attn_simt_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __re
                  int H_kv, int n, int s, int causal, const double* __restrict__ sigma,
                  const double* __restrict__ table, const int32_t* __restrict__ spans,
                  const MaskT* __restrict__ bmask, T* __restrict__ O, float* __restrict__ row_sum,
-                 uint32_t* __restrict__ err) {
+                 uint32_t* __restrict__ err, int varlen) {
   constexpr int TPR = D / 32;            // threads per query row
   constexpr int NT = kTile * TPR;
   constexpr int F4 = D / 4;              // float4 per row
@@ -97,18 +97,6 @@ attn_simt_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __re
       }
   }
 
-  // window of this tile
-  int lo = spans[(static_cast<size_t>(h) * T_tiles + t) * 2];
-  int hi = spans[(static_cast<size_t>(h) * T_tiles + t) * 2 + 1];
-  const int last_row = min(n, i0 + kTile) - 1;
-  if (lo < 0 || lo > i0 || hi >= n || hi < last_row) {
-    flags |= PLSH_DEVERR_WINDOW;
-    lo = max(0, min(lo, i0));
-    hi = min(n - 1, max(hi, last_row));
-  }
-  const int n_below = (i0 - lo + kTile - 1) / kTile;
-  const int n_above = causal ? 0 : (hi - i0) / kTile;
-
   // this thread's 32 dims of q: float4 indices f = part + TPR * m, m = 0..7
   const size_t q_row = ((static_cast<size_t>(b) * H + h) * n + (row_ok ? i : 0)) * D;
   float q[32];
@@ -126,111 +114,131 @@ attn_simt_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __re
 
   const size_t kv_base = (static_cast<size_t>(b) * H_kv + kvh) * static_cast<size_t>(n) * D;
   const MaskT* bm_h = bmask + static_cast<size_t>(h) * n;
-  const int total = 1 + n_below + n_above;
-  for (int it = 0; it < total; ++it) {
-    const int kind = it == 0 ? 0 : (it <= n_below ? 1 : 2);   // 0 diagonal, 1 below, 2 above
-    const int j0 = kind == 0 ? i0 : (kind == 1 ? i0 - kTile * it : i0 + kTile * (it - n_below));
-    __syncthreads();
-    for (int idx = tid; idx < kTile * F4; idx += NT) {
-      const int row = idx / F4, c4 = idx % F4;
-      const int j = j0 + row;
-      float4 kx = make_float4(0.f, 0.f, 0.f, 0.f), vx = kx;
-      if (j >= 0 && j < n) {
-        kx = load4(K + kv_base + static_cast<size_t>(j) * D + 4 * c4);
-        vx = load4(V + kv_base + static_cast<size_t>(j) * D + 4 * c4);
+  // K3: one pass over the union window with weights c_ij (sw = s). K4 (varlen): one pass per hash k
+  // over that hash's window with the hash-k masks alone, so each weight is hash k's 0/1 block
+  // indicator (sw = 1); the passes share the running maximum, sum and accumulator.
+  const int n_pass = varlen ? s : 1;
+  const int sw = varlen ? 1 : s;
+  const int last_row = min(n, i0 + kTile) - 1;
+  for (int pass = 0; pass < n_pass; ++pass) {
+    const MaskT bits = varlen ? static_cast<MaskT>(static_cast<MaskT>(1) << pass) : FULL;
+    const size_t span_at = varlen ? ((static_cast<size_t>(h) * s + pass) * T_tiles + t) * 2
+                                  : (static_cast<size_t>(h) * T_tiles + t) * 2;
+    int lo = spans[span_at];
+    int hi = spans[span_at + 1];
+    if (lo < 0 || lo > i0 || hi >= n || hi < last_row) {
+      flags |= PLSH_DEVERR_WINDOW;
+      lo = max(0, min(lo, i0));
+      hi = min(n - 1, max(hi, last_row));
+    }
+    const int n_below = (i0 - lo + kTile - 1) / kTile;
+    const int n_above = causal ? 0 : (hi - i0) / kTile;
+    const int total = 1 + n_below + n_above;
+    for (int it = 0; it < total; ++it) {
+      const int kind = it == 0 ? 0 : (it <= n_below ? 1 : 2);   // 0 diagonal, 1 below, 2 above
+      const int j0 = kind == 0 ? i0 : (kind == 1 ? i0 - kTile * it : i0 + kTile * (it - n_below));
+      __syncthreads();
+      for (int idx = tid; idx < kTile * F4; idx += NT) {
+        const int row = idx / F4, c4 = idx % F4;
+        const int j = j0 + row;
+        float4 kx = make_float4(0.f, 0.f, 0.f, 0.f), vx = kx;
+        if (j >= 0 && j < n) {
+          kx = load4(K + kv_base + static_cast<size_t>(j) * D + 4 * c4);
+          vx = load4(V + kv_base + static_cast<size_t>(j) * D + 4 * c4);
+        }
+        store4(&sm.k[row * D + 4 * c4], kx);
+        store4(&sm.v[row * D + 4 * c4], vx);
       }
-      store4(&sm.k[row * D + 4 * c4], kx);
-      store4(&sm.v[row * D + 4 * c4], vx);
-    }
-    for (int c = tid; c <= kTile; c += NT) {
-      const int j = j0 + c;
-      sm.bm[c] = (j >= 0 && j < n) ? bm_h[j] : FULL;
-    }
-    __syncthreads();
-    if (tid < kTile) {
-      MaskT a = 0, z = 0;
-      for (int q2 = tid + 1; q2 < kTile; ++q2) a |= sm.bm[q2];
-      for (int q2 = 1; q2 <= tid; ++q2) z |= sm.bm[q2];
-      sm.suf[tid] = a;
-      sm.pre[tid] = z;
-    }
-    if (kind == 0 && part == 0) {
-      unsigned char* wr = sm.wdiag + r * kDiagStride;
-      wr[r] = static_cast<unsigned char>(s);
-      MaskT R = 0;
-      for (int c = r - 1; c >= 0; --c) {
-        R |= sm.bm[c + 1];
-        wr[c] = static_cast<unsigned char>(s - popc_mask(R));
+      for (int c = tid; c <= kTile; c += NT) {
+        const int j = j0 + c;
+        sm.bm[c] = static_cast<MaskT>(((j >= 0 && j < n) ? bm_h[j] : FULL) & bits);
       }
-      sm.ycarry[r] = R | sm.bm[0];       // OR over [i0, i]
-      R = 0;
-      for (int c = r + 1; c < kTile; ++c) {
-        R |= sm.bm[c];
-        wr[c] = static_cast<unsigned char>(s - popc_mask(R));
+      __syncthreads();
+      if (tid < kTile) {
+        MaskT a = 0, z = 0;
+        for (int q2 = tid + 1; q2 < kTile; ++q2) a |= sm.bm[q2];
+        for (int q2 = 1; q2 <= tid; ++q2) z |= sm.bm[q2];
+        sm.suf[tid] = a;
+        sm.pre[tid] = z;
       }
-      sm.zcarry[r] = R;                  // OR over (i, i0 + 127]
-    }
-    __syncthreads();
-    if (kind == 2) Z |= sm.bm[0];          // now OR over (i, j0]
+      if (kind == 0 && part == 0) {
+        unsigned char* wr = sm.wdiag + r * kDiagStride;
+        wr[r] = static_cast<unsigned char>(sw);
+        MaskT R = 0;
+        for (int c = r - 1; c >= 0; --c) {
+          R |= sm.bm[c + 1];
+          wr[c] = static_cast<unsigned char>(sw - popc_mask(R));
+        }
+        sm.ycarry[r] = R | sm.bm[0];       // OR over [i0, i]
+        R = 0;
+        for (int c = r + 1; c < kTile; ++c) {
+          R |= sm.bm[c];
+          wr[c] = static_cast<unsigned char>(sw - popc_mask(R));
+        }
+        sm.zcarry[r] = R;                  // OR over (i, i0 + 127]
+      }
+      __syncthreads();
+      if (kind == 2) Z |= sm.bm[0];          // now OR over (i, j0]
 
-#pragma unroll 1
-    for (int chunk = 0; chunk < kTile / 32; ++chunk) {
-      float sv[32];
-      int wv[32];
-#pragma unroll
-      for (int cc = 0; cc < 32; ++cc) {
-        const int c = chunk * 32 + cc;
-        int w;
-        if (kind == 0) w = (causal && c > r) ? 0 : sm.wdiag[r * kDiagStride + c];
-        else if (kind == 1) w = s - popc_mask(static_cast<MaskT>(sm.suf[c] | Y));
-        else w = s - popc_mask(static_cast<MaskT>(Z | sm.pre[c]));
-        float dot = 0.0f;
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          const float4 kx = *reinterpret_cast<const float4*>(&sm.k[c * D + 4 * (part + TPR * m)]);
-          dot = fmaf(q[4 * m], kx.x, dot);
-          dot = fmaf(q[4 * m + 1], kx.y, dot);
-          dot = fmaf(q[4 * m + 2], kx.z, dot);
-          dot = fmaf(q[4 * m + 3], kx.w, dot);
+  #pragma unroll 1
+      for (int chunk = 0; chunk < kTile / 32; ++chunk) {
+        float sv[32];
+        int wv[32];
+  #pragma unroll
+        for (int cc = 0; cc < 32; ++cc) {
+          const int c = chunk * 32 + cc;
+          int w;
+          if (kind == 0) w = (causal && c > r) ? 0 : sm.wdiag[r * kDiagStride + c];
+          else if (kind == 1) w = sw - popc_mask(static_cast<MaskT>(sm.suf[c] | Y));
+          else w = sw - popc_mask(static_cast<MaskT>(Z | sm.pre[c]));
+          float dot = 0.0f;
+  #pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            const float4 kx = *reinterpret_cast<const float4*>(&sm.k[c * D + 4 * (part + TPR * m)]);
+            dot = fmaf(q[4 * m], kx.x, dot);
+            dot = fmaf(q[4 * m + 1], kx.y, dot);
+            dot = fmaf(q[4 * m + 2], kx.z, dot);
+            dot = fmaf(q[4 * m + 3], kx.w, dot);
+          }
+  #pragma unroll
+          for (int o = TPR / 2; o >= 1; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+          sv[cc] = w > 0 ? dot * scale : -INFINITY;
+          wv[cc] = w;
         }
-#pragma unroll
-        for (int o = TPR / 2; o >= 1; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-        sv[cc] = w > 0 ? dot * scale : -INFINITY;
-        wv[cc] = w;
-      }
-      float cmax = -INFINITY;
-#pragma unroll
-      for (int cc = 0; cc < 32; ++cc) cmax = fmaxf(cmax, sv[cc]);
-      if (cmax == -INFINITY) continue;
-      const float m_new = fmaxf(m_run, cmax);
-      const float corr = expf(m_run - m_new);   // 0 when m_run = -inf
-      l_run *= corr;
-#pragma unroll
-      for (int e = 0; e < 32; ++e) acc[e] *= corr;
-      m_run = m_new;
-#pragma unroll
-      for (int cc = 0; cc < 32; ++cc) {
-        if (wv[cc] <= 0) continue;
-        const int c = chunk * 32 + cc;
-        const float p = static_cast<float>(wv[cc]) * expf(sv[cc] - m_run);
-        l_run += p;
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          const float4 vx = *reinterpret_cast<const float4*>(&sm.v[c * D + 4 * (part + TPR * m)]);
-          acc[4 * m] = fmaf(p, vx.x, acc[4 * m]);
-          acc[4 * m + 1] = fmaf(p, vx.y, acc[4 * m + 1]);
-          acc[4 * m + 2] = fmaf(p, vx.z, acc[4 * m + 2]);
-          acc[4 * m + 3] = fmaf(p, vx.w, acc[4 * m + 3]);
+        float cmax = -INFINITY;
+  #pragma unroll
+        for (int cc = 0; cc < 32; ++cc) cmax = fmaxf(cmax, sv[cc]);
+        if (cmax == -INFINITY) continue;
+        const float m_new = fmaxf(m_run, cmax);
+        const float corr = expf(m_run - m_new);   // 0 when m_run = -inf
+        l_run *= corr;
+  #pragma unroll
+        for (int e = 0; e < 32; ++e) acc[e] *= corr;
+        m_run = m_new;
+  #pragma unroll
+        for (int cc = 0; cc < 32; ++cc) {
+          if (wv[cc] <= 0) continue;
+          const int c = chunk * 32 + cc;
+          const float p = static_cast<float>(wv[cc]) * expf(sv[cc] - m_run);
+          l_run += p;
+  #pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            const float4 vx = *reinterpret_cast<const float4*>(&sm.v[c * D + 4 * (part + TPR * m)]);
+            acc[4 * m] = fmaf(p, vx.x, acc[4 * m]);
+            acc[4 * m + 1] = fmaf(p, vx.y, acc[4 * m + 1]);
+            acc[4 * m + 2] = fmaf(p, vx.z, acc[4 * m + 2]);
+            acc[4 * m + 3] = fmaf(p, vx.w, acc[4 * m + 3]);
+          }
         }
       }
-    }
-    if (kind == 0) {
-      Y = sm.ycarry[r];
-      Z = sm.zcarry[r];
-    } else if (kind == 1) {
-      Y |= static_cast<MaskT>(sm.bm[0] | sm.suf[0]);   // tile fully passed: OR over [j0, i]
-    } else {
-      Z |= sm.pre[kTile - 1];                           // OR over (i, j0 + 127]
+      if (kind == 0) {
+        Y = sm.ycarry[r];
+        Z = sm.zcarry[r];
+      } else if (kind == 1) {
+        Y |= static_cast<MaskT>(sm.bm[0] | sm.suf[0]);   // tile fully passed: OR over [j0, i]
+      } else {
+        Z |= sm.pre[kTile - 1];                           // OR over (i, j0 + 127]
+      }
     }
   }
 
@@ -257,7 +265,7 @@ int launch_simt_typed(const AttnArgs& a, cudaStream_t st) {
   kern<<<grid, kTile * (D / 32), smem, st>>>(
       static_cast<const T*>(a.Q), static_cast<const T*>(a.K), static_cast<const T*>(a.V), a.H, a.H_kv, a.n, a.s,
       a.causal, a.sigma, a.table, a.spans, static_cast<const MaskT*>(a.bmask), static_cast<T*>(a.O), a.row_sum,
-      a.err);
+      a.err, a.varlen);
   e = cudaGetLastError();
   return e == cudaSuccess ? PLSH_OK : cuda_fail(e, "attn_simt_kernel launch");
 }

@@ -46,6 +46,12 @@
 // P), and writes P of keys [16ch, 16ch + 16) as bf16 pairs to columns
 // [8ch, 8ch + 8) of the S region, over columns it has already read.
 //
+// The per-sample comparator (K4) runs the same machinery with each item walked
+// once per hash k over that hash's own window, the boundary masks reduced to
+// bit k and the weight count s replaced by 1: each pass adds hash k's 0/1
+// block-diagonal attention, and the passes share one online softmax, so the
+// result is the same T~ (Methodology 3, Theorem 2.2's construction).
+//
 // Every barrier wait is bounded in time (PLSH_DEVERR_TIMEOUT); on timeout all
 // roles leave their loops, in-flight copies and MMAs are drained and TMEM is
 // freed before the CTA returns.
@@ -116,38 +122,57 @@ static_assert(sizeof(TcSmem<unsigned long long>) + 1024 <= 232448, "shared memor
 
 struct Params {
   int B, H, H_kv, n, s, causal, T, items;
+  // varlen = 0: spans are [H][T][2] union windows (K3). varlen = 1: spans are [H][s][T][2]
+  // per-hash windows and every item is walked once per hash (K4, the per-sample comparator).
+  int varlen;
   const int32_t* spans;
 };
 
 // The key tiles of one slot's work items, in the order every role walks them:
 // items x0, x0 + stride, ...; within an item the diagonal tile, then the tiles
-// below, then (non-causal) the tiles above. The next item's window is fetched
-// one item ahead.
+// below, then (non-causal) the tiles above. For the per-sample comparator an
+// item is walked once per hash k (a sub-item), each time over that hash's
+// window. The next (sub-)item's window is fetched one ahead.
 struct TileIter {
   const Params* p;
   const int16_t* order;
   int x, stride;
   int k;        // items started so far by this slot
-  int it;       // key tile within the item
-  int total;    // key tiles of the item
+  int sub;      // sub-item (hash) within the item: 0 for K3
+  int it;       // key tile within the sub-item
+  int total;    // key tiles of the sub-item
   int n_below;
   int b, h, i0;
   int g;        // key tiles so far by this slot
   bool valid;
-  bool bad_window;  // the window read for this item was out of range (and was clamped)
+  bool bad_window;  // the window read for this sub-item was out of range (and was clamped)
   int nx_lo, nx_hi;
 
+  __device__ __forceinline__ int n_sub() const { return p->varlen ? p->s : 1; }
   __device__ __forceinline__ int head_of(int xx) const {
     const int hr = xx / (p->B * p->T);
     return (p->H <= kMaxSortedHeads) ? static_cast<int>(order[hr]) : hr;
   }
-  __device__ __forceinline__ void fetch(int xx, int& lo, int& hi) const {
+  __device__ __forceinline__ void fetch(int xx, int sb, int& lo, int& hi) const {
     if (xx < p->items) {
       const int hh = head_of(xx);
       const int tt = (xx % (p->B * p->T)) % p->T;
-      lo = p->spans[(static_cast<size_t>(hh) * p->T + tt) * 2];
-      hi = p->spans[(static_cast<size_t>(hh) * p->T + tt) * 2 + 1];
+      const size_t at = p->varlen ? ((static_cast<size_t>(hh) * p->s + sb) * p->T + tt) * 2
+                                  : (static_cast<size_t>(hh) * p->T + tt) * 2;
+      lo = p->spans[at];
+      hi = p->spans[at + 1];
     }
+  }
+  __device__ __forceinline__ void load_sub(int lo, int hi) {
+    if (sub + 1 < n_sub()) fetch(x, sub + 1, nx_lo, nx_hi);
+    else fetch(x + stride, 0, nx_lo, nx_hi);
+    const int last_row = min(p->n, i0 + kTile) - 1;
+    bad_window = lo < 0 || lo > i0 || hi >= p->n || hi < last_row;
+    lo = max(0, min(lo, i0));
+    hi = min(p->n - 1, max(hi, last_row));
+    n_below = (i0 - lo + kTile - 1) / kTile;
+    total = 1 + n_below + (p->causal ? 0 : (hi - i0) / kTile);
+    it = 0;
   }
   __device__ __forceinline__ void load_item(int lo, int hi) {
     valid = x < p->items;
@@ -156,14 +181,8 @@ struct TileIter {
     h = head_of(x);
     b = rem / p->T;
     i0 = (rem % p->T) * kTile;
-    fetch(x + stride, nx_lo, nx_hi);
-    const int last_row = min(p->n, i0 + kTile) - 1;
-    bad_window = lo < 0 || lo > i0 || hi >= p->n || hi < last_row;
-    lo = max(0, min(lo, i0));
-    hi = min(p->n - 1, max(hi, last_row));
-    n_below = (i0 - lo + kTile - 1) / kTile;
-    total = 1 + n_below + (p->causal ? 0 : (hi - i0) / kTile);
-    it = 0;
+    sub = 0;
+    load_sub(lo, hi);
   }
   __device__ __forceinline__ void start(const Params* pp, const int16_t* ord, int slot) {
     p = pp;
@@ -174,15 +193,20 @@ struct TileIter {
     g = 0;
     nx_lo = nx_hi = 0;
     int lo = 0, hi = 0;
-    fetch(x, lo, hi);
+    fetch(x, 0, lo, hi);
     load_item(lo, hi);
   }
   __device__ __forceinline__ void next() {
     ++g;
     if (++it >= total) {
-      x += stride;
-      ++k;
-      load_item(nx_lo, nx_hi);
+      if (sub + 1 < n_sub()) {
+        ++sub;
+        load_sub(nx_lo, nx_hi);
+      } else {
+        x += stride;
+        ++k;
+        load_item(nx_lo, nx_hi);
+      }
     }
   }
   __device__ __forceinline__ int kind() const { return it == 0 ? 0 : (it <= n_below ? 1 : 2); }
@@ -190,8 +214,8 @@ struct TileIter {
     const int kd = kind();
     return kd == 0 ? i0 : (kd == 1 ? i0 - kTile * it : i0 + kTile * (it - n_below));
   }
-  __device__ __forceinline__ bool first() const { return it == 0; }
-  __device__ __forceinline__ bool last() const { return it == total - 1; }
+  __device__ __forceinline__ bool first() const { return it == 0 && sub == 0; }
+  __device__ __forceinline__ bool last() const { return it == total - 1 && sub == n_sub() - 1; }
 };
 
 template <typename MaskT>
@@ -355,9 +379,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   // heads by decreasing window width of their middle query tile, ties by head index (the same order in every CTA)
   if (H <= kMaxSortedHeads) {
     const int tm = prm.T / 2;
-    for (int h = threadIdx.x; h < H; h += kThreads)
-      sm.width[h] = prm.spans[(static_cast<size_t>(h) * prm.T + tm) * 2 + 1] -
-                    prm.spans[(static_cast<size_t>(h) * prm.T + tm) * 2];
+    const int nsub = prm.varlen ? s : 1;
+    for (int h = threadIdx.x; h < H; h += kThreads) {
+      int w = 0;
+      for (int sb = 0; sb < nsub; ++sb) {
+        const size_t at = (static_cast<size_t>(h) * nsub + sb) * prm.T + tm;
+        w += prm.spans[at * 2 + 1] - prm.spans[at * 2];
+      }
+      sm.width[h] = w;
+    }
   }
   __syncthreads();
   if (H <= kMaxSortedHeads) {
@@ -467,7 +497,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       if (*abort_flag) {
         // let every copy already issued land before the CTA can exit
         for (int z = 0; z < kSlots; ++z) {
-          const int q_issued = kit[z].k + ((kit[z].valid && kit[z].it > 0) ? 1 : 0);
+          const int q_issued = kit[z].k + ((kit[z].valid && !kit[z].first()) ? 1 : 0);
           if (q_issued > 0) mbar_wait_drain(&sm.q_full[z], (q_issued - 1) & 1, kDrainNs);
           if (kit[z].g > 0) mbar_wait_drain(&sm.k_full[z], (kit[z].g - 1) & 1, kDrainNs);
           if (vit[z].g > 0) mbar_wait_drain(&sm.v_full[z], (vit[z].g - 1) & 1, kDrainNs);
@@ -509,7 +539,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
               // keys 16kk..16kk+15: P at columns 8kk..8kk+7; the keys are two 8-row groups of the
               // MN-major V tile, whose two d halves sit kChunkBytes apart
               mma_ts(o_tmem, p_tmem + 8u * kk, v_desc[z] + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
-                     (pi.it > 0 || kk > 0) ? 1u : 0u);
+                     (!pi.first() || kk > 0) ? 1u : 0u);
             }
             mma_commit(&sm.v_empty[z]);
             if (pi.last()) mma_commit(&sm.o_full[z]);
@@ -558,16 +588,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     ti.start(&prm, sm.order, z);
     nx.start(&prm, sm.order, z);
     if (nx.valid) nx.next();
+    // the masks of a tile; a comparator sub-item keeps only its own hash's bit
     auto load_masks = [&](const TileIter& t, MaskT (&v)[4], MaskT& v128) {
       const MaskT* bm_h = bmask + static_cast<size_t>(t.h) * n;
+      const MaskT bits = prm.varlen ? static_cast<MaskT>(static_cast<MaskT>(1) << t.sub) : FULL;
       const int j0 = t.j0();
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int j = j0 + 4 * lane + e;
-        v[e] = (j >= 0 && j < n) ? bm_h[j] : FULL;
+        v[e] = static_cast<MaskT>(((j >= 0 && j < n) ? bm_h[j] : FULL) & bits);
       }
       const int j = j0 + kTile;
-      v128 = (lane == 0 && j >= 0 && j < n) ? bm_h[j] : FULL;
+      v128 = static_cast<MaskT>(((lane == 0 && j >= 0 && j < n) ? bm_h[j] : FULL) & bits);
     };
     MaskT xv[4] = {FULL, FULL, FULL, FULL}, x128 = FULL;
     if (ti.valid) load_masks(ti, xv, x128);
@@ -684,7 +716,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     const uint32_t s_base = tmem + lane_off + kColS + 128u * z;
     const uint32_t o_base = tmem + lane_off + kColO + 128u * z;
     const float sc = 1.4426950408889634f / sqrtf(static_cast<float>(kD));
-    const float cs = 8388608.0f + static_cast<float>(s);  // 2^23 + s
+    // weights count hashes: all s of them, or (comparator) the one hash of the sub-item
+    const int sw = prm.varlen ? 1 : s;
+    const float cs = 8388608.0f + static_cast<float>(sw);  // 2^23 + sw
     float m2 = -INFINITY, l = 0.0f;
     MaskT Y = 0, Z = 0;
     int items_done = 0;
@@ -703,7 +737,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       // weights that need only the masks: the diagonal's own block and its carries
       uint32_t cnt[8];
       MaskT lo = 0, hi = 0;
-      if (kind == 0) diag_scan<MaskT, kCausal>(ms, quarter, r, s, cnt, lo, hi);
+      if (kind == 0) diag_scan<MaskT, kCausal>(ms, quarter, r, sw, cnt, lo, hi);
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[z], static_cast<uint32_t>(g & 1), abort_flag, err)))
         break;
       tc_fence_after();
@@ -913,6 +947,7 @@ int launch_tc_typed(const AttnArgs& a, cudaStream_t st) {
   prm.causal = a.causal;
   prm.T = ceil_div(a.n, kTile);
   prm.items = a.B * a.H * prm.T;
+  prm.varlen = a.varlen;
   prm.spans = a.spans;
   auto kern = attn_tc_kernel<MaskT, kCausal>;
   const size_t smem = sizeof(TcSmem<MaskT>) + 1024;

@@ -29,7 +29,11 @@ struct AttnArgs {
   const double* sigma; const double* table;
   const int32_t* spans; const void* bmask;
   void* O; float* row_sum; uint32_t* err;
+  // 0: K3 (spans = [H][T][2] union windows, weights c_ij). 1: K4, the per-sample comparator
+  // (spans = [H][s][T][2] per-hash windows; each sample's block indicator, summed over samples).
+  int varlen;
 };
+int launch_varlen_spans(const int32_t* ids, int H, int s, int n, int causal, int32_t* spans, cudaStream_t st);
 int launch_attention_simt(const AttnArgs& a, cudaStream_t st);
 int launch_attention_tc(const AttnArgs& a, cudaStream_t st);
 

@@ -239,11 +239,19 @@ def run_ours(args, rank, world, local):
     plan = PlshForward(w.B, w.H, w.H_kv, w.n, w.d, w.s, w.causal, w.sigmas(), wr.seed, w.torch_dtype, dev)
     stream = torch.cuda.current_stream()
 
+    varlen = args.path == "varlen"
+
+    def attend():
+        if varlen:
+            plan.attend_varlen(q, k, v, stream)
+        else:
+            plan.attend(q, k, v, stream)
+
     def step(ev=None):
         plan.prepare(stream)
         if ev is not None:
             ev[0].record(stream)
-        plan.attend(q, k, v, stream)
+        attend()
         if ev is not None:
             ev[1].record(stream)
 
@@ -253,7 +261,11 @@ def run_ours(args, rank, world, local):
     errs = plan.device_errors()
     if errs:
         raise RuntimeError(f"device errors during warm-up: {errs}")
-    spans = plan.spans.cpu().numpy()
+    if varlen:   # per-hash windows [H][s][T][2]: every hash's window is visited
+        T = (w.n + TILE - 1) // TILE
+        spans = plan.scratch.cpu().numpy()[: w.H * w.s * T * 2].reshape(w.H * w.s, T, 2)
+    else:
+        spans = plan.spans.cpu().numpy()
     tiles_min = issued_tiles(spans, w.causal)
     tiles_run = kernel_tiles(spans, w.causal)
 
@@ -288,7 +300,7 @@ def run_ours(args, rank, world, local):
     rh = torch.empty_like(plan.row_sum, device="cpu").pin_memory()
     qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     for _ in range(3):
-        plan.run_host(qh, kh, vh, qd, kd, vd, oh, rh, stream)
+        plan.run_host(qh, kh, vh, qd, kd, vd, oh, rh, stream, varlen=varlen)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     Ke = max(3, min(K, 20))
@@ -296,13 +308,38 @@ def run_ours(args, rank, world, local):
     torch.cuda.synchronize()
     e0.record(stream)
     for _ in range(Ke):
-        plan.run_host(qh, kh, vh, qd, kd, vd, oh, rh, stream)
+        plan.run_host(qh, kh, vh, qd, kd, vd, oh, rh, stream, varlen=varlen)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = dist_max(e0.elapsed_time(e1) / Ke, world)
     h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh)) + plan.table_host.numel() * 8
     d2h = oh.numel() * oh.element_size() + rh.numel() * 4
+
+    # the other attention path on the same plan and inputs, for comparison (not part of the step)
+    other = None
+    if world == 1:
+        def other_attend():
+            if varlen:
+                plan.attend(q, k, v, stream)
+            else:
+                plan.attend_varlen(q, k, v, stream)
+        for _ in range(2):
+            other_attend()
+        ts = []
+        for _ in range(5):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            other_attend()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        errs = plan.device_errors()
+        if errs:
+            raise RuntimeError(f"device errors in the comparison path: {errs}")
+        other = {"path": "fused (plsh_attention_fwd)" if varlen else "per-sample comparator (plsh_attention_varlen_fwd)",
+                 "attention_ms": float(np.median(ts)),
+                 "this_path_speedup": float(np.median(ts)) / attn_avg}
 
     tokens = w.B * w.n * world
     value = tokens / (ms_step * 1e-3)
@@ -336,6 +373,7 @@ def run_ours(args, rank, world, local):
 
     line = {
         "metric": "PLSH-ALiBi fwd query-tokens/s at n=32k, s=20; achieved % of roofline",
+        "path": "per-sample comparator (plsh_attention_varlen_fwd)" if varlen else "fused (plsh_attention_fwd)",
         "value": value,
         "unit": "query-tokens/s",
         "n_gpus": world,
@@ -354,13 +392,16 @@ def run_ours(args, rank, world, local):
         "roofline": roof,
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "query-tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "path": "PlshForward.run_host: pinned host Q/K/V -> device -> table, K1, K2, K3 -> host O, row_sum"},
-        "gpu_launches": 4 * K,
-        "gpu_launches_per_step": {"sample_bins_kernel": 1, "mask_bmax_kernel": 1, "spans_kernel": 1,
-                                  roof["kernel"]: 1},
+                "path": "PlshForward.run_host: pinned host Q/K/V -> device -> table, K1, K2, "
+                        + ("K4" if varlen else "K3") + " -> host O, row_sum"},
+        "gpu_launches": (5 if varlen else 4) * K,
+        "gpu_launches_per_step": dict({"sample_bins_kernel": 1, "mask_bmax_kernel": 1, "spans_kernel": 1,
+                                       roof["kernel"]: 1}, **({"varlen_spans_kernel": 1} if varlen else {})),
         "step_breakdown_ms": {"attention": attn_avg, "table+bins+window": ms_step - attn_avg},
         "clocks": clocks,
     }
+    if other is not None:
+        line["comparison"] = other
     if rank == 0 and not args.no_cpu_baseline:
         sampler = OracleSampler(w)
         rate, desc = sampler.run(args.cpu_seconds)
@@ -417,6 +458,8 @@ def main(argv=None):
     ap.add_argument("--workload", default=workloads.HEADLINE, choices=list(workloads.WORKLOADS))
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", choices=["fused", "varlen"], default="fused",
+                    help="attention path timed: the fused kernel (K3) or the per-sample comparator (K4)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller cases for profiling)")
     args = ap.parse_args(argv)

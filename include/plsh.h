@@ -168,6 +168,57 @@ PLSH_API int plsh_attention_fwd(const void* Q, const void* K, const void* V, int
                        const void* bmask_dev, int causal, void* O, float* row_sum,
                        uint32_t* err_dev, void* stream);
 
+/*
+ * plsh_varlen_scratch_bytes -- bytes of scratch plsh_attention_varlen_fwd
+ * needs: 8 * H * s * ceil(n/128) (one int32 pair per head, hash and query
+ * tile). Returns 0 for a non-positive size.
+ */
+PLSH_API size_t plsh_varlen_scratch_bytes(int H, int s, int n);
+
+/*
+ * plsh_varlen_spans (K4 set-up) -- the key window of every query tile in
+ * each single hash's blocks.
+ *
+ * Cites: Methodology 3 (Theorem 2.2's construction: attention restricted,
+ * per sample, to that sample's blocks) and Methodology 1, structure (blocks
+ * are contiguous). For head h, hash k and query rows [128t, min(n,128t+128)):
+ * lo = the first position of the hash-k block holding row 128t, hi = the last
+ * position of the hash-k block holding the tile's last row, or that row
+ * itself when causal.
+ *
+ *   ids_dev    [H][s][n] int32 from plsh_sample_bins (non-decreasing in n).
+ *   spans_dev  [H][s][ceil(n/128)][2] int32 out, (lo, hi) inclusive.
+ */
+PLSH_API int plsh_varlen_spans(const int32_t* ids_dev, int H, int s, int n, int causal, int32_t* spans_dev,
+                               void* stream);
+
+/*
+ * plsh_attention_varlen_fwd (K4) -- the per-sample comparator: the same
+ * T~ and row_sum as plsh_attention_fwd, computed the way Theorem 2.2 builds
+ * it (Methodology 3): for each hash k separately, every query row attends
+ * only to the keys of its own hash-k block (the block-diagonal mask M(h_k)),
+ * and the s block-diagonal attentions are summed, numerator and denominator,
+ * before the division:
+ *   O_i = sum_k sum_j M_k[i,j] e^{S_ij} V_j / sum_k sum_j M_k[i,j] e^{S_ij}.
+ * Each query tile visits the key tiles of every hash's window, so the
+ * tensor work grows with the sum of the s windows instead of their union.
+ *
+ *   Arguments as plsh_attention_fwd, with
+ *   ids_dev        [H][s][n] int32 from plsh_sample_bins.
+ *   bmask_dev      [H][n] from plsh_window (bit k gives hash k's blocks).
+ *   scratch_dev    caller-owned device memory of at least
+ *                  plsh_varlen_scratch_bytes(H, s, n) bytes, 16-byte
+ *                  aligned; it receives the per-hash windows
+ *                  (plsh_varlen_spans) and is read by the attention kernel
+ *                  on the same stream. Nothing in it needs clearing.
+ *   scratch_bytes  its size; smaller than needed is PLSH_ERR_INVALID_ARG.
+ */
+PLSH_API int plsh_attention_varlen_fwd(const void* Q, const void* K, const void* V, int dtype, int B, int H,
+                                       int H_kv, int n, int d, const double* sigma_dev, int s,
+                                       const double* table_dev, const int32_t* ids_dev, const void* bmask_dev,
+                                       int causal, void* scratch_dev, size_t scratch_bytes, void* O,
+                                       float* row_sum, uint32_t* err_dev, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -39,7 +39,7 @@ import numpy as np
 __all__ = [
     "splitmix64", "uniform_open", "uniform_closed_open", "draw_table",
     "bins", "bin_ids", "hash_mask", "match_counts", "mean_mask", "counts_rows",
-    "boundary_bits", "block_lengths", "bmax", "tile_spans", "alibi_matrix",
+    "boundary_bits", "block_lengths", "bmax", "tile_spans", "varlen_spans", "alibi_matrix",
     "approx_attention", "exact_attention", "forward", "forward_exact",
     "COUNTER_HEAD_SHIFT", "TILE",
 ]
@@ -239,6 +239,32 @@ def tile_spans(ids_hs: np.ndarray, causal: bool, tile: int = TILE) -> np.ndarray
             c[cols[None, :] > rows[:, None]] = 0
         nz = np.nonzero(c.sum(axis=0))[0]
         out[t] = (nz.min(), nz.max())
+    return out
+
+
+def varlen_spans(ids_hs: np.ndarray, causal: bool, tile: int = TILE,
+                 tiles: Optional[Sequence[int]] = None) -> np.ndarray:
+    """Per-hash key windows of the per-sample comparator, int64 [s][T][2] = (lo, hi).
+
+    [nl M3]: Theorem 2.2's construction attends, for each sample k, only
+    inside that sample's blocks. For hash k and query rows
+    [t*tile, min(n, (t+1)*tile)), [lo, hi] is the smallest key range holding
+    every j in the same hash-k bin as some row i of the tile (and j <= i when
+    causal). Brute force over the rows' bin-equality rows; `tiles` limits the
+    work to those tile indices (the others stay -1).
+    """
+    s, n = ids_hs.shape
+    T = (n + tile - 1) // tile
+    out = np.full((s, T, 2), -1, dtype=np.int64)
+    cols = np.arange(n)
+    for k in range(s):
+        for t in (range(T) if tiles is None else tiles):
+            rows = np.arange(t * tile, min(n, (t + 1) * tile))
+            same = ids_hs[k][rows][:, None] == ids_hs[k][None, :]
+            if causal:
+                same &= cols[None, :] <= rows[:, None]
+            nz = np.nonzero(same.any(axis=0))[0]
+            out[k, t] = (nz.min(), nz.max())
     return out
 
 

@@ -7,7 +7,8 @@ a plausible mistake in the oracle and checks that some pin catches it.
 
 Pins used (none of them re-types the oracle's own formula):
   * published SplitMix64 test vectors (golden file);
-  * hand-worked bins, boundary bits, counts, b_max, windows (golden file);
+  * hand-worked bins, boundary bits, counts, b_max, windows and per-hash
+    windows (golden file); per-hash windows against block starts / ends;
   * a hand-worked 3-token T~ / T* example with exact fractions (golden file);
   * the Gamma(2, sigma) and U[0,1) laws of the table (KS tests, moments);
   * the exact identity E_h[M(h)] = L* (Monte Carlo, 10^6 draws);
@@ -110,6 +111,8 @@ def check_bins_worked(orc):
         assert c[i, j] == v and c[j, i] == v, (i, j, c[i, j], v)
     assert orc.tile_spans(ids, False, hh["tile"]).tolist() == hh["spans_noncausal"]
     assert orc.tile_spans(ids, True, hh["tile"]).tolist() == hh["spans_causal"]
+    assert orc.varlen_spans(ids, False, hh["tile"]).tolist() == hh["varlen_spans_noncausal"]
+    assert orc.varlen_spans(ids, True, hh["tile"]).tolist() == hh["varlen_spans_causal"]
 
 
 def _tables_for_invariants(orc):
@@ -169,6 +172,29 @@ def check_boundary_identity(orc, n=300):
                 acc |= int(bm[j])
                 want = s - bin(acc).count("1")
                 assert c[i, j] == want and c[j, i] == want, (h, i, j)
+
+
+def check_varlen_spans_from_blocks(orc, n=900, tile=128):
+    """Per-hash windows equal (start of the first row's block, end of the last row's block).
+
+    Blocks are contiguous (Methodology 1, structure), so the keys sharing a hash-k block with
+    some row of a tile run from the first row's block start to the last row's block end; when
+    causal the end is the last row. Block starts and ends come from the run lengths here.
+    """
+    for table in _tables_for_invariants(orc):
+        ids = orc.bin_ids(table, n)
+        for h in range(ids.shape[0]):
+            for causal in (False, True):
+                got = orc.varlen_spans(ids[h], causal, tile)
+                for k in range(ids.shape[1]):
+                    L = orc.block_lengths(ids[h, k])
+                    ends = np.cumsum(L) - 1
+                    starts = ends - L + 1
+                    blk = np.repeat(np.arange(len(L)), L)     # block index of every position
+                    for t in range(got.shape[1]):
+                        first, last = t * tile, min(n, (t + 1) * tile) - 1
+                        want = (starts[blk[first]], last if causal else ends[blk[last]])
+                        assert tuple(got[k, t]) == want, (h, k, t, causal, got[k, t], want)
 
 
 def check_expectation_identity(orc, n=64, draws=1_000_000, sigmas=(1.0, 4.0, 16.0)):

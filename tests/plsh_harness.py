@@ -20,15 +20,24 @@ def f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu", torch.float64).numpy()
 
 
-def run_gpu(B, H, H_kv, n, d, s, causal, sigma, seed, q, k, v, table: Optional[np.ndarray] = None):
-    """The whole path through the C-ABI; q, k, v are CPU tensors (copied to cuda:0)."""
+def run_gpu(B, H, H_kv, n, d, s, causal, sigma, seed, q, k, v, table: Optional[np.ndarray] = None,
+            varlen: bool = False):
+    """The whole path through the C-ABI; q, k, v are CPU tensors (copied to cuda:0).
+
+    varlen=True runs the per-sample comparator (plsh_attention_varlen_fwd) for the attention step
+    and also returns its per-hash windows.
+    """
     from alibi_positional_lsh_b200 import PlshForward
     plan = PlshForward(B, H, H_kv, n, d, s, causal, sigma, seed, q.dtype, "cuda:0")
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
     # poison the outputs so a row the kernel never writes cannot pass
     plan.O.fill_(float("nan"))
     plan.row_sum.fill_(float("nan"))
-    plan(qd, kd, vd, table=table)
+    if varlen:
+        plan.prepare(table=table)
+        plan.attend_varlen(qd, kd, vd)
+    else:
+        plan(qd, kd, vd, table=table)
     errs = plan.device_errors()
     out = dict(
         errors=errs,
@@ -40,6 +49,9 @@ def run_gpu(B, H, H_kv, n, d, s, causal, sigma, seed, q, k, v, table: Optional[n
         O=f64(plan.O),
         row_sum=plan.row_sum.cpu().numpy().astype(np.float64),
     )
+    if varlen:
+        T = (n + 127) // 128
+        out["varlen_spans"] = plan.scratch.cpu().numpy().astype(np.int64)[: H * s * T * 2].reshape(H, s, T, 2)
     return out
 
 

@@ -132,6 +132,24 @@ def _spans_ignore_causal(ids_hs, causal, tile=O.TILE):
     return _orig["tile_spans"](ids_hs, False, tile)
 
 
+def _varlen_union_window(ids_hs, causal, tile=O.TILE, tiles=None):
+    # wrong reading: every hash takes the union window of all hashes (the K3 window)
+    one = _orig["tile_spans"](ids_hs, causal, tile)
+    return np.repeat(one[None], ids_hs.shape[0], axis=0)
+
+
+def _varlen_shared_row(ids_hs, causal, tile=O.TILE, tiles=None):
+    # wrong index: the window of the tile's first row only (misses the last row's block)
+    s, n = ids_hs.shape
+    out = _orig["varlen_spans"](ids_hs, causal, tile, tiles)
+    for k in range(s):
+        for t in range(out.shape[1]):
+            i = t * tile
+            same = np.nonzero(ids_hs[k] == ids_hs[k][i])[0]
+            out[k, t] = (same.min(), i if causal else same.max())
+    return out
+
+
 def _bmax_interior_only(ids_hs):
     return int(max(O.block_lengths(ids_hs[k])[1:-1].max(initial=1) for k in range(ids_hs.shape[0])))
 
@@ -151,6 +169,8 @@ MUTATIONS = [
     ("forward", _forward_wrong_gqa, [P.check_rows_and_gqa]),
     ("tile_spans", _spans_ignore_causal, [P.check_bins_worked]),
     ("bmax", _bmax_interior_only, [P.check_bins_worked]),
+    ("varlen_spans", _varlen_union_window, [P.check_bins_worked, P.check_varlen_spans_from_blocks]),
+    ("varlen_spans", _varlen_shared_row, [P.check_bins_worked, P.check_varlen_spans_from_blocks]),
 ]
 
 

@@ -26,6 +26,10 @@ def test_bins_worked_examples():
     P.check_bins_worked(oracle)
 
 
+def test_varlen_spans_match_block_ends():
+    P.check_varlen_spans_from_blocks(oracle)
+
+
 def test_blocks_contiguous():
     P.check_contiguous_blocks(oracle)
 
