@@ -24,6 +24,7 @@ PLSH_BF16 = 0
 PLSH_F32 = 1
 PLSH_TILE = 128
 PLSH_MAX_S = 64
+PLSH_VARLEN_STATIC_SCRATCH_BYTES = 4 << 20
 DEVERR_BITS = {1: "RANGE", 2: "TABLE", 4: "WINDOW", 8: "TIMEOUT", 16: "SIGMA"}
 
 
@@ -35,7 +36,7 @@ class PlshError(RuntimeError):
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is not built: run `python -m alibi_positional_lsh_b200.build` "
+        raise ImportError(f"{LIB_PATH} is not built: run `python alibi_positional_lsh_b200/build.py` "
                           "(or __graft_entry__.build()) first")
     lib = ctypes.CDLL(LIB_PATH)
     vp, i32, u64, dp = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64, ctypes.c_void_p
@@ -59,6 +60,9 @@ def _load() -> ctypes.CDLL:
     lib.plsh_attention_varlen_fwd.restype = i32
     lib.plsh_attention_varlen_fwd.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, i32, vp, vp, vp, i32,
                                               vp, ctypes.c_size_t, vp, vp, vp, vp]
+    lib.plsh_attention_varlen_fwd_static.restype = i32
+    lib.plsh_attention_varlen_fwd_static.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, i32, vp, vp,
+                                                     vp, i32, vp, vp, vp, vp]
     return lib
 
 
@@ -148,6 +152,16 @@ def plsh_attention_varlen_fwd(Q, K, V, dtype: int, B: int, H: int, H_kv: int, n:
                                           _dev_ptr(scratch_dev, "scratch_dev"), ctypes.c_size_t(nbytes),
                                           _dev_ptr(O, "O"), _dev_ptr(row_sum, "row_sum"),
                                           _dev_ptr(err_dev, "err_dev"), _stream_ptr(stream)))
+
+
+def plsh_attention_varlen_fwd_static(Q, K, V, dtype: int, B: int, H: int, H_kv: int, n: int, d: int, sigma_dev,
+                                     s: int, table_dev, ids_dev, bmask_dev, causal: int, O, row_sum, err_dev,
+                                     stream=None) -> None:
+    _check(_lib.plsh_attention_varlen_fwd_static(
+        _dev_ptr(Q, "Q"), _dev_ptr(K, "K"), _dev_ptr(V, "V"), dtype, B, H, H_kv, n, d,
+        _dev_ptr(sigma_dev, "sigma_dev"), s, _dev_ptr(table_dev, "table_dev"), _dev_ptr(ids_dev, "ids_dev"),
+        _dev_ptr(bmask_dev, "bmask_dev"), int(causal), _dev_ptr(O, "O"), _dev_ptr(row_sum, "row_sum"),
+        _dev_ptr(err_dev, "err_dev"), _stream_ptr(stream)))
 
 
 def decode_device_error(word: int) -> list:

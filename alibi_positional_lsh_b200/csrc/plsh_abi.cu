@@ -4,6 +4,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "plsh_internal.h"
 
@@ -139,6 +140,71 @@ extern "C" int plsh_attention_varlen_fwd(const void* Q, const void* K, const voi
     return fail(PLSH_ERR_INVALID_ARG, "%s: scratch holds %zu bytes, %zu needed", fn, scratch_bytes, need);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int32_t* spans = static_cast<int32_t*>(scratch_dev);
+  if (int rc = plsh::launch_varlen_spans(ids_dev, H, s, n, causal, spans, st)) return rc;
+  plsh::AttnArgs a{Q, K, V, dtype, B, H, H_kv, n, d, s, causal, sigma_dev, table_dev,
+                   spans, bmask_dev, O, row_sum, err_dev, 1};
+  return plsh::launch_attention(a, st);
+}
+
+// ---------------------------------------------------------------- comparator without caller scratch
+//
+// plsh_attention_varlen_fwd_static: the per-sample comparator for callers that cannot hand the
+// library any device memory of their own for scratch. Such a caller has only its inputs and
+// outputs: it may run where the device allocator must not be entered (a hook inside the
+// caller's own memory management) or where every device allocation is budgeted up front. The
+// per-hash windows then live in a fixed file-scope device buffer of this library.
+namespace plsh {
+namespace {
+
+// Per-hash windows of the comparator: [H][s][ceil(n/128)][2] int32, fully written by the window
+// kernel before the attention kernel reads it, so nothing in it needs to start at zero.
+static __device__ __align__(256) int32_t g_varlen_static_scratch[PLSH_VARLEN_STATIC_SCRATCH_BYTES / sizeof(int32_t)];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mutex;
+void* g_static_ptr[kMaxDevices] = {};
+
+// The buffer's device address on the current device, looked up once per device (with that
+// device current) and cached.
+int static_scratch_ptr(const char* fn, void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(PLSH_ERR_RANGE, "%s: device ordinal %d not supported", fn, dev);
+  std::lock_guard<std::mutex> lock(g_static_mutex);
+  if (!g_static_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_varlen_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(g_varlen_static_scratch)");
+    g_static_ptr[dev] = p;
+  }
+  *out = g_static_ptr[dev];
+  return PLSH_OK;
+}
+
+}  // namespace
+}  // namespace plsh
+
+extern "C" int plsh_attention_varlen_fwd_static(const void* Q, const void* K, const void* V, int dtype, int B,
+                                                int H, int H_kv, int n, int d, const double* sigma_dev, int s,
+                                                const double* table_dev, const int32_t* ids_dev,
+                                                const void* bmask_dev, int causal, void* O, float* row_sum,
+                                                uint32_t* err_dev, void* stream) {
+  const char* fn = "plsh_attention_varlen_fwd_static";
+  if (int rc = plsh::check_attention(fn, Q, K, V, dtype, B, H, H_kv, n, d, s, causal, bmask_dev, O, row_sum,
+                                     err_dev))
+    return rc;
+  if (!ids_dev) return fail(PLSH_ERR_INVALID_ARG, "%s: null pointer", fn);
+  const size_t need = plsh_varlen_scratch_bytes(H, s, n);
+  if (need > PLSH_VARLEN_STATIC_SCRATCH_BYTES)
+    return fail(PLSH_ERR_RANGE,
+                "%s: the per-hash windows need %zu bytes (8 * H * s * ceil(n/128)), more than the %zu-byte "
+                "static buffer; use plsh_attention_varlen_fwd with caller scratch",
+                fn, need, static_cast<size_t>(PLSH_VARLEN_STATIC_SCRATCH_BYTES));
+  void* scratch = nullptr;
+  if (int rc = plsh::static_scratch_ptr(fn, &scratch)) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t* spans = static_cast<int32_t*>(scratch);
   if (int rc = plsh::launch_varlen_spans(ids_dev, H, s, n, causal, spans, st)) return rc;
   plsh::AttnArgs a{Q, K, V, dtype, B, H, H_kv, n, d, s, causal, sigma_dev, table_dev,
                    spans, bmask_dev, O, row_sum, err_dev, 1};

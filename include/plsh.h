@@ -22,7 +22,8 @@
  *   - "_dev" pointers are device memory owned by the caller; "_host"
  *     pointers are host memory owned by the caller. The library allocates
  *     no device memory and keeps no state between calls except the
- *     thread-local error string and a cached driver entry point.
+ *     thread-local error string, a cached driver entry point and, for
+ *     plsh_attention_varlen_fwd_static, the cached address of its buffer.
  *   - Device work is enqueued on `stream` (a cudaStream_t passed as void*,
  *     NULL = legacy default stream) and is asynchronous: no entry point
  *     synchronises the device.
@@ -218,6 +219,38 @@ PLSH_API int plsh_attention_varlen_fwd(const void* Q, const void* K, const void*
                                        const double* table_dev, const int32_t* ids_dev, const void* bmask_dev,
                                        int causal, void* scratch_dev, size_t scratch_bytes, void* O,
                                        float* row_sum, uint32_t* err_dev, void* stream);
+
+/* Size of the library's own buffer behind plsh_attention_varlen_fwd_static. */
+#define PLSH_VARLEN_STATIC_SCRATCH_BYTES (4u << 20)
+
+/*
+ * plsh_attention_varlen_fwd_static -- plsh_attention_varlen_fwd without
+ * caller scratch. The paper has no counterpart: this is a calling
+ * convention, not part of the method.
+ *
+ * It is for callers that cannot give the library device memory of their
+ * own: code that may not enter the device allocator at the point of the
+ * call (a hook running inside the caller's own memory management), or that
+ * budgets every device allocation up front. The per-hash windows go to a
+ * fixed buffer inside the library instead: a file-scope __device__ array of
+ * PLSH_VARLEN_STATIC_SCRATCH_BYTES (4 MiB) per device. Nothing in it needs to
+ * start at zero, and the library allocates nothing.
+ *
+ *   Arguments and results as plsh_attention_varlen_fwd, without scratch_dev
+ *   and scratch_bytes.
+ *   Limit: 8 * H * s * ceil(n/128) <= PLSH_VARLEN_STATIC_SCRATCH_BYTES, else
+ *   PLSH_ERR_RANGE with nothing launched (H=16, s=20 fits up to n = 209,664).
+ *   The first call on a device looks the buffer's address up
+ *   (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *   first call before any stream capture. Calls that overlap on one device
+ *   (on different streams, or from different host threads without ordering)
+ *   share the buffer and race: order them, or use plsh_attention_varlen_fwd.
+ */
+PLSH_API int plsh_attention_varlen_fwd_static(const void* Q, const void* K, const void* V, int dtype, int B,
+                                              int H, int H_kv, int n, int d, const double* sigma_dev, int s,
+                                              const double* table_dev, const int32_t* ids_dev,
+                                              const void* bmask_dev, int causal, void* O, float* row_sum,
+                                              uint32_t* err_dev, void* stream);
 
 #ifdef __cplusplus
 }
