@@ -122,9 +122,8 @@ static_assert(sizeof(TcSmem<unsigned long long>) + 1024 <= 232448, "shared memor
 
 struct Params {
   int B, H, H_kv, n, s, causal, T, items;
-  // varlen = 0: spans are [H][T][2] union windows (K3). varlen = 1: spans are [H][s][T][2]
-  // per-hash windows and every item is walked once per hash (K4, the per-sample comparator).
-  int varlen;
+  // [H][T][2] union windows (K3), or [H][s][T][2] per-hash windows for the comparator (K4, the
+  // kVarlen instantiations, which walk every item once per hash)
   const int32_t* spans;
 };
 
@@ -133,6 +132,7 @@ struct Params {
 // below, then (non-causal) the tiles above. For the per-sample comparator an
 // item is walked once per hash k (a sub-item), each time over that hash's
 // window. The next (sub-)item's window is fetched one ahead.
+template <bool kVarlen>
 struct TileIter {
   const Params* p;
   const int16_t* order;
@@ -148,7 +148,7 @@ struct TileIter {
   bool bad_window;  // the window read for this sub-item was out of range (and was clamped)
   int nx_lo, nx_hi;
 
-  __device__ __forceinline__ int n_sub() const { return p->varlen ? p->s : 1; }
+  __device__ __forceinline__ int n_sub() const { return kVarlen ? p->s : 1; }
   __device__ __forceinline__ int head_of(int xx) const {
     const int hr = xx / (p->B * p->T);
     return (p->H <= kMaxSortedHeads) ? static_cast<int>(order[hr]) : hr;
@@ -157,14 +157,14 @@ struct TileIter {
     if (xx < p->items) {
       const int hh = head_of(xx);
       const int tt = (xx % (p->B * p->T)) % p->T;
-      const size_t at = p->varlen ? ((static_cast<size_t>(hh) * p->s + sb) * p->T + tt) * 2
-                                  : (static_cast<size_t>(hh) * p->T + tt) * 2;
+      const size_t at = kVarlen ? ((static_cast<size_t>(hh) * p->s + sb) * p->T + tt) * 2
+                                : (static_cast<size_t>(hh) * p->T + tt) * 2;
       lo = p->spans[at];
       hi = p->spans[at + 1];
     }
   }
   __device__ __forceinline__ void load_sub(int lo, int hi) {
-    if (sub + 1 < n_sub()) fetch(x, sub + 1, nx_lo, nx_hi);
+    if (kVarlen && sub + 1 < n_sub()) fetch(x, sub + 1, nx_lo, nx_hi);
     else fetch(x + stride, 0, nx_lo, nx_hi);
     const int last_row = min(p->n, i0 + kTile) - 1;
     bad_window = lo < 0 || lo > i0 || hi >= p->n || hi < last_row;
@@ -199,7 +199,7 @@ struct TileIter {
   __device__ __forceinline__ void next() {
     ++g;
     if (++it >= total) {
-      if (sub + 1 < n_sub()) {
+      if (kVarlen && sub + 1 < n_sub()) {
         ++sub;
         load_sub(nx_lo, nx_hi);
       } else {
@@ -214,8 +214,8 @@ struct TileIter {
     const int kd = kind();
     return kd == 0 ? i0 : (kd == 1 ? i0 - kTile * it : i0 + kTile * (it - n_below));
   }
-  __device__ __forceinline__ bool first() const { return it == 0 && sub == 0; }
-  __device__ __forceinline__ bool last() const { return it == total - 1 && sub == n_sub() - 1; }
+  __device__ __forceinline__ bool first() const { return it == 0 && (!kVarlen || sub == 0); }
+  __device__ __forceinline__ bool last() const { return it == total - 1 && (!kVarlen || sub == n_sub() - 1); }
 };
 
 template <typename MaskT>
@@ -348,7 +348,7 @@ __device__ __forceinline__ void diag_scan(const MaskStage<MaskT>& ms, int q, int
   hi = R2;
 }
 
-template <typename MaskT, bool kCausal>
+template <typename MaskT, bool kCausal, bool kVarlen>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ Params prm,
@@ -379,7 +379,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   // heads by decreasing window width of their middle query tile, ties by head index (the same order in every CTA)
   if (H <= kMaxSortedHeads) {
     const int tm = prm.T / 2;
-    const int nsub = prm.varlen ? s : 1;
+    const int nsub = kVarlen ? s : 1;
     for (int h = threadIdx.x; h < H; h += kThreads) {
       int w = 0;
       for (int sb = 0; sb < nsub; ++sb) {
@@ -438,7 +438,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       tma_prefetch_desc(&tmap_q);
       tma_prefetch_desc(&tmap_k);
       tma_prefetch_desc(&tmap_v);
-      TileIter kit[kSlots], vit[kSlots];
+      TileIter<kVarlen> kit[kSlots], vit[kSlots];
       for (int z = 0; z < kSlots; ++z) {
         kit[z].start(&prm, sm.order, z);
         vit[z].start(&prm, sm.order, z);
@@ -449,7 +449,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         bool progress = false;
 #pragma unroll
         for (int z = 0; z < kSlots; ++z) {
-          TileIter& ki = kit[z];
+          TileIter<kVarlen>& ki = kit[z];
           if (ki.valid) {
             // Q of a new item once the slot's previous item has run its last S; K(g) once S(g-1) has run
             const bool q_ok = !ki.first() || ki.k == 0 || mbar_test_wait(&sm.q_empty[z], (ki.k - 1) & 1);
@@ -469,7 +469,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
               progress = true;
             }
           }
-          TileIter& vi = vit[z];
+          TileIter<kVarlen>& vi = vit[z];
           if (vi.valid && (vi.g == 0 || mbar_test_wait(&sm.v_empty[z], (vi.g - 1) & 1))) {
             const int zkv = vi.b * prm.H_kv + vi.h / (H / prm.H_kv);
             const int j0 = vi.j0();
@@ -511,7 +511,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, 1);
-      TileIter st_it[kSlots], pv_it[kSlots];
+      TileIter<kVarlen> st_it[kSlots], pv_it[kSlots];
       uint64_t q_desc[kSlots], k_desc[kSlots], v_desc[kSlots];
       for (int z = 0; z < kSlots; ++z) {
         st_it[z].start(&prm, sm.order, z);
@@ -526,8 +526,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         bool progress = false;
 #pragma unroll
         for (int z = 0; z < kSlots; ++z) {
-          TileIter& si = st_it[z];
-          TileIter& pi = pv_it[z];
+          TileIter<kVarlen>& si = st_it[z];
+          TileIter<kVarlen>& pi = pv_it[z];
           // PV first: it frees the slot's S columns for the next S
           if (pi.valid && pi.g < si.g && mbar_test_wait(&sm.p_full[z], pi.g & 1) &&
               mbar_test_wait(&sm.v_full[z], pi.g & 1)) {
@@ -584,14 +584,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   } else if (warp == 2 || warp == 3) {
     // ------------------------------------------------------------ mask warp of slot (warp - 2)
     const int z = warp - 2;
-    TileIter ti, nx;
+    TileIter<kVarlen> ti, nx;
     ti.start(&prm, sm.order, z);
     nx.start(&prm, sm.order, z);
     if (nx.valid) nx.next();
     // the masks of a tile; a comparator sub-item keeps only its own hash's bit
-    auto load_masks = [&](const TileIter& t, MaskT (&v)[4], MaskT& v128) {
+    auto load_masks = [&](const TileIter<kVarlen>& t, MaskT (&v)[4], MaskT& v128) {
       const MaskT* bm_h = bmask + static_cast<size_t>(t.h) * n;
-      const MaskT bits = prm.varlen ? static_cast<MaskT>(static_cast<MaskT>(1) << t.sub) : FULL;
+      const MaskT bits = kVarlen ? static_cast<MaskT>(static_cast<MaskT>(1) << t.sub) : FULL;
       const int j0 = t.j0();
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -717,7 +717,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     const uint32_t o_base = tmem + lane_off + kColO + 128u * z;
     const float sc = 1.4426950408889634f / sqrtf(static_cast<float>(kD));
     // weights count hashes: all s of them, or (comparator) the one hash of the sub-item
-    const int sw = prm.varlen ? 1 : s;
+    const int sw = kVarlen ? 1 : s;
     const float cs = 8388608.0f + static_cast<float>(sw);  // 2^23 + sw
     float m2 = -INFINITY, l = 0.0f;
     MaskT Y = 0, Z = 0;
@@ -932,7 +932,7 @@ int sm_count() {
   return count;
 }
 
-template <typename MaskT, bool kCausal>
+template <typename MaskT, bool kCausal, bool kVarlen>
 int launch_tc_typed(const AttnArgs& a, cudaStream_t st) {
   CUtensorMap mq, mk, mv;
   if (int rc = make_map(&mq, a.Q, a.n, a.B * a.H)) return rc;
@@ -947,9 +947,8 @@ int launch_tc_typed(const AttnArgs& a, cudaStream_t st) {
   prm.causal = a.causal;
   prm.T = ceil_div(a.n, kTile);
   prm.items = a.B * a.H * prm.T;
-  prm.varlen = a.varlen;
   prm.spans = a.spans;
-  auto kern = attn_tc_kernel<MaskT, kCausal>;
+  auto kern = attn_tc_kernel<MaskT, kCausal, kVarlen>;
   const size_t smem = sizeof(TcSmem<MaskT>) + 1024;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_tc_kernel)");
@@ -966,9 +965,18 @@ int launch_tc_typed(const AttnArgs& a, cudaStream_t st) {
 int launch_attention_tc(const AttnArgs& a, cudaStream_t st) {
   if (static_cast<long long>(a.B) * a.H * ceil_div(a.n, kTile) > 0x7fffffffLL)
     return fail(PLSH_ERR_RANGE, "plsh_attention_fwd: too many query tiles");
+  if (a.varlen) {
+    if (a.causal)
+      return a.s <= 32 ? launch_tc_typed<uint32_t, true, true>(a, st)
+                       : launch_tc_typed<unsigned long long, true, true>(a, st);
+    return a.s <= 32 ? launch_tc_typed<uint32_t, false, true>(a, st)
+                     : launch_tc_typed<unsigned long long, false, true>(a, st);
+  }
   if (a.causal)
-    return a.s <= 32 ? launch_tc_typed<uint32_t, true>(a, st) : launch_tc_typed<unsigned long long, true>(a, st);
-  return a.s <= 32 ? launch_tc_typed<uint32_t, false>(a, st) : launch_tc_typed<unsigned long long, false>(a, st);
+    return a.s <= 32 ? launch_tc_typed<uint32_t, true, false>(a, st)
+                     : launch_tc_typed<unsigned long long, true, false>(a, st);
+  return a.s <= 32 ? launch_tc_typed<uint32_t, false, false>(a, st)
+                   : launch_tc_typed<unsigned long long, false, false>(a, st);
 }
 
 }  // namespace plsh

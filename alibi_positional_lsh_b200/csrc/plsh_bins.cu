@@ -9,7 +9,9 @@
 // expression. Ids are stored relative to position 0 so they fit int32.
 //
 // HBM-bound: 4 bytes written per (head, hash, position), no reads beyond
-// the 16-byte table entry. Each thread writes 4 consecutive ids (one 16-byte
+// the 16-byte table entry; the quotient is a multiply by the reciprocal with
+// an exactness test (floor_quotient), so the float64 divide runs only near
+// bin boundaries. Each thread writes 4 consecutive ids (one 16-byte
 // store) when the row is 16-byte aligned.
 #include <cmath>
 
@@ -21,10 +23,23 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kPerThread = 4;
 
-__device__ __forceinline__ int32_t bin_id(double pos, double u, double delta, double base,
+// floor(RN((pos + u) / delta)) without a division for almost every position. With
+// a = RN(pos + u) and rcp = RN(1 / delta), xa = RN(a * rcp) is within 3 * 2^-53 * xa of
+// q = RN(a / delta) (each of the three roundings is relative 2^-53). If xa lies more than
+// 2^-50 * xa from both integers around it, q lies strictly between them too and
+// floor(q) = floor(xa); otherwise the exact quotient is taken.
+__device__ __forceinline__ double floor_quotient(double pos, double u, double delta, double rcp) {
+  const double a = __dadd_rn(pos, u);
+  const double xa = __dmul_rn(a, rcp);
+  const double fl = floor(xa);
+  const double tol = xa * 0x1p-50;
+  if (xa - fl > tol && (fl + 1.0) - xa > tol) return fl;
+  return floor(__ddiv_rn(a, delta));
+}
+
+__device__ __forceinline__ int32_t bin_id(double pos, double u, double delta, double rcp, double base,
                                           uint32_t& flags) {
-  const double x = __ddiv_rn(__dadd_rn(pos, u), delta);
-  const double id = floor(x) - base;
+  const double id = floor_quotient(pos, u, delta, rcp) - base;
   if (!(id >= 0.0 && id <= 2147483647.0)) {
     flags |= PLSH_DEVERR_RANGE;
     return 2147483647;
@@ -43,6 +58,7 @@ __global__ void __launch_bounds__(kThreads) sample_bins_kernel(const double* __r
   const bool ok = isfinite(delta) && delta > 0.0 && isfinite(u);
   if (!ok) flags |= PLSH_DEVERR_TABLE;
   const double base = ok ? floor(__ddiv_rn(u, delta)) : 0.0;
+  const double rcp = ok ? __drcp_rn(delta) : 0.0;
   int32_t* row = ids + (static_cast<size_t>(h) * s + k) * n;
   const bool vec = (n % kPerThread) == 0;  // rows start 16-byte aligned when n % 4 == 0
   const int stride = gridDim.x * kThreads * kPerThread;
@@ -51,7 +67,7 @@ __global__ void __launch_bounds__(kThreads) sample_bins_kernel(const double* __r
 #pragma unroll
     for (int e = 0; e < kPerThread; ++e) {
       const int i = i0 + e;
-      v[e] = (ok && i < n) ? bin_id(static_cast<double>(i), u, delta, base, flags) : 0;
+      v[e] = (ok && i < n) ? bin_id(static_cast<double>(i), u, delta, rcp, base, flags) : 0;
     }
     if (vec && i0 + kPerThread <= n) {
       *reinterpret_cast<int4*>(row + i0) = make_int4(v[0], v[1], v[2], v[3]);

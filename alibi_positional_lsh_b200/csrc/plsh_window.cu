@@ -13,8 +13,10 @@
 // bin is s - popcount(OR of bmask over (min(i,j), max(i,j)]), which is how
 // the attention kernels read the weights.
 //
-// Block ends and starts are found by an exponential-then-binary search on
-// the non-decreasing ids, so each block costs O(log length) reads.
+// The masks and block lengths come from one coalesced pass over the ids
+// (block lengths via a CTA-wide scan of block starts); only the block
+// holding each CTA's first position, and the window ends, are found by an
+// exponential-then-binary search on the non-decreasing ids.
 #include "plsh_internal.h"
 
 namespace plsh {
@@ -58,30 +60,90 @@ __device__ __forceinline__ int block_end(const int32_t* __restrict__ row, int p,
   return good;
 }
 
+// Boundary masks and longest blocks for 1024 positions of one head per CTA, all s hashes.
+// Per hash a thread holds 4 consecutive ids; a block starts where the id changes and ends
+// before the next change. Each block's length is taken at its last position, from the latest
+// block start at or before it: within the thread, else from earlier threads of the CTA (a
+// CTA-wide max-scan of the threads' last starts), else the block began before the CTA's first
+// position p0 and its start is carry[k], found once per CTA and hash by a search.
 template <typename MaskT>
 __global__ void __launch_bounds__(kThreads) mask_bmax_kernel(const int32_t* __restrict__ ids, int s, int n,
                                                              MaskT* __restrict__ bmask,
                                                              int32_t* __restrict__ bmax) {
+  constexpr int kPer = 4;
+  constexpr int kSpan = kThreads * kPer;
+  constexpr int kWarps = kThreads / 32;
+  __shared__ int carry[PLSH_MAX_S];
+  __shared__ int warp_last[kWarps];
   const int h = blockIdx.y;
-  const int p = blockIdx.x * kThreads + threadIdx.x;
+  const int p0 = blockIdx.x * kSpan;
+  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+  const int32_t* base = ids + static_cast<size_t>(h) * s * n;
+  if (t < s) {
+    const int32_t* row = base + static_cast<size_t>(t) * n;
+    carry[t] = block_start(row, p0, row[p0]);
+  }
+  __syncthreads();
+  const int pb = p0 + kPer * t;                     // this thread's first position
+  const bool vec = (n % 4 == 0) && (pb + kPer <= n);  // 16-byte aligned full int4
+  MaskT m[kPer] = {0, 0, 0, 0};
   int longest = 0;
-  if (p < n) {
-    MaskT m = 0;
-    const int32_t* base = ids + static_cast<size_t>(h) * s * n;
-    for (int k = 0; k < s; ++k) {
-      const int32_t* row = base + static_cast<size_t>(k) * n;
-      const int32_t a = row[p];
-      if (p == 0 || row[p - 1] != a) m |= static_cast<MaskT>(1) << k;
-      const bool ends_here = (p == n - 1) || (row[p + 1] != a);
-      if (ends_here) {
-        const int len = p - block_start(row, p, a) + 1;
-        longest = len > longest ? len : longest;
+  for (int k = 0; k < s; ++k) {
+    const int32_t* row = base + static_cast<size_t>(k) * n;
+    int32_t id[kPer];
+    if (vec) {
+      const int4 v = *reinterpret_cast<const int4*>(row + pb);
+      id[0] = v.x; id[1] = v.y; id[2] = v.z; id[3] = v.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) id[e] = (pb + e < n) ? row[pb + e] : 0;
+    }
+    const int32_t prev = (pb > 0 && pb < n) ? row[pb - 1] : 0;
+    const int32_t next = (pb + kPer < n) ? row[pb + kPer] : 0;
+    bool st[kPer], en[kPer];
+    int mylast = -1;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) {
+      const int p = pb + e;
+      const bool ok = p < n;
+      st[e] = ok && (p == 0 || id[e] != (e > 0 ? id[e - 1] : prev));
+      en[e] = ok && (p == n - 1 || id[e] != (e + 1 < kPer ? id[e + 1] : next));
+      if (st[e]) {
+        m[e] |= static_cast<MaskT>(1) << k;
+        mylast = p;
       }
     }
-    bmask[static_cast<size_t>(h) * n + p] = m;
+    // latest block start before this thread's positions, over the CTA
+    int incl = mylast;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl = max(incl, y);
+    }
+    if (lane == 31) warp_last[w] = incl;
+    __syncthreads();
+    int before = __shfl_up_sync(0xffffffffu, incl, 1);
+    if (lane == 0) before = -1;
+    for (int w2 = 0; w2 < w; ++w2) before = max(before, warp_last[w2]);
+    __syncthreads();  // warp_last is rewritten for the next hash
+    int cur = before >= 0 ? before : carry[k];
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) {
+      if (st[e]) cur = pb + e;
+      if (en[e]) longest = max(longest, pb + e - cur + 1);
+    }
+  }
+  MaskT* out = bmask + static_cast<size_t>(h) * n;
+  if (vec && sizeof(MaskT) == 4) {
+    *reinterpret_cast<uint4*>(out + pb) = make_uint4(static_cast<uint32_t>(m[0]), static_cast<uint32_t>(m[1]),
+                                                     static_cast<uint32_t>(m[2]), static_cast<uint32_t>(m[3]));
+  } else {
+#pragma unroll
+    for (int e = 0; e < kPer; ++e)
+      if (pb + e < n) out[pb + e] = m[e];
   }
   longest = __reduce_max_sync(0xffffffffu, longest);
-  if ((threadIdx.x & 31) == 0 && longest > 0) atomicMax(bmax + h, longest);
+  if (lane == 0 && longest > 0) atomicMax(bmax + h, longest);
 }
 
 // One warp per (head, query tile); lanes walk the hashes.
@@ -115,7 +177,7 @@ int launch_window(const int32_t* ids, int H, int s, int n, int causal, int32_t* 
   (void)err;
   cudaError_t e = cudaMemsetAsync(bmax, 0, sizeof(int32_t) * H, st);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(bmax)");
-  dim3 g1(ceil_div(n, kThreads), H);
+  dim3 g1(ceil_div(n, 4 * kThreads), H);
   if (s <= 32)
     mask_bmax_kernel<uint32_t><<<g1, kThreads, 0, st>>>(ids, s, n, static_cast<uint32_t*>(bmask), bmax);
   else
