@@ -163,11 +163,31 @@ def dist_setup(n_gpus: int):
 
 
 def dist_max(x: float, world: int) -> float:
+    """Max over ranks (a CUDA tensor under NCCL, a CPU tensor under gloo)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_workload(w: workloads.Workload, rank: int) -> workloads.Workload:
+    """Each rank solves an independent problem of the same shape (its own seed)."""
+    return w.with_(seed=w.seed + 1000 * rank)
+
+
+def job_value(tokens_per_rank: int, world: int, ms_step_max: float) -> float:
+    """Whole-job query-tokens/s: the tokens every rank processed over the slowest rank's step time."""
+    return tokens_per_rank * world / (ms_step_max * 1e-3)
+
+
+def config_of(w: workloads.Workload, world: int) -> dict:
+    qkv = (w.B * w.H * w.n * w.d + 2 * w.B * w.H_kv * w.n * w.d) * (2 if w.dtype == "bf16" else 4)
+    return {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.H_kv, "n": w.n, "d": w.d, "s": w.s,
+            "causal": w.causal, "global_batch": w.B * world, "seq_len": w.n,
+            "parallelism": f"independent problem per GPU x{world}",
+            "l2": f"no flush: Q+K+V = {qkv / 1e6:.0f} MB per step, larger than the 126 MB L2"}
 
 
 def barrier(world: int):
@@ -234,7 +254,7 @@ def run_ours(args, rank, world, local):
         w = w.with_(B=args.batch)
     dev = f"cuda:{local}"
     torch.cuda.set_device(local)
-    wr = w.with_(seed=w.seed + 1000 * rank)          # independent problem per rank
+    wr = rank_workload(w, rank)                      # independent problem per rank
     q, k, v = workloads.make_qkv_device(wr, dev)
     plan = PlshForward(w.B, w.H, w.H_kv, w.n, w.d, w.s, w.causal, w.sigmas(), wr.seed, w.torch_dtype, dev)
     stream = torch.cuda.current_stream()
@@ -342,7 +362,7 @@ def run_ours(args, rank, world, local):
                  "this_path_speedup": float(np.median(ts)) / attn_avg}
 
     tokens = w.B * w.n * world
-    value = tokens / (ms_step * 1e-3)
+    value = job_value(w.B * w.n, world, ms_step)
     peaks, peak_src = load_peaks()
     elt = 2 if w.dtype == "bf16" else 4
     qkvo_bytes = (w.B * w.H * w.n * w.d * 2 + 2 * w.B * w.H_kv * w.n * w.d) * elt
@@ -385,10 +405,7 @@ def run_ours(args, rank, world, local):
         "vs_baseline": None,
         "dtype": w.dtype,
         "data": "synthetic (iid N(0,1) Q/K/V drawn on the device, seeded per rank)",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.H_kv, "n": w.n, "d": w.d, "s": w.s,
-                   "causal": w.causal, "global_batch": w.B * world, "seq_len": w.n,
-                   "parallelism": f"independent problem per GPU x{world}",
-                   "l2": f"no flush: Q+K+V = {(qkvo_bytes * 3 // 4) / 1e6:.0f} MB per step, larger than the 126 MB L2"},
+        "config": config_of(w, world),
         "roofline": roof,
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "query-tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -441,8 +458,7 @@ def run_reference(args, rank, world):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic (iid N(0,1) Q/K/V, seeded)",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.H_kv, "n": w.n, "d": w.d, "s": w.s,
-                   "causal": w.causal},
+        "config": config_of(w, world),
         "cpu_baseline": {"value": value, "unit": "query-tokens/s", "cores": sampler.cores, "kind": "oracle",
                          "sample": f"each step: {desc}"},
         "e2e": {"value": value, "unit": "query-tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
