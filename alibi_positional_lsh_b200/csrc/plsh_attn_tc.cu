@@ -10,20 +10,21 @@
 // c_ij > 0 (Methodology 2, block-size control), and only those key tiles are
 // visited (Methodology 3: attention restricted to short random blocks).
 //
-// Persistent CTAs (one per SM), each running two work items at a time in two
-// independent slots, so that one slot's waits are covered by the other
-// slot's work. Items come from a static list, heads with the widest windows
-// first. Warp roles (384 threads):
-//   warp 0       TMA producer for both slots: Q per item, K and V per key tile
-//   warp 1       TMEM owner and single-thread tcgen05.mma issuer for both slots
-//   warps 2, 3   mask warp of slot 0 / slot 1: the key tile's boundary masks,
-//                their in-tile prefix / suffix ORs and the tile's descriptor
-//   warps 4-7    softmax of slot 0, warps 8-11 softmax of slot 1: one query
-//                row per thread (TMEM lane = row)
-// Per key tile of a slot: S = Q K^T (SS MMA into the slot's TMEM S columns),
-// the softmax turns S into bf16 P written back over S, then O += P V (TS MMA,
-// P from TMEM, fp32 O in the slot's TMEM O columns). The MMA thread issues,
-// per slot, S(g), PV(g), S(g+1), ... as their inputs become ready.
+// Persistent CTAs (one per SM) walk a static list of items, heads with the
+// widest windows first. Warp roles (352 threads):
+//   warps 0-7    softmax: warp w owns rows 32 (w % 4) .. + 31 (TMEM lane
+//                quarter w % 4) and keys 64 (w / 4) .. + 63 of every tile
+//   warp 8       TMA producer: Q per item (two buffers), K and V per key tile
+//                (two stages each)
+//   warp 9       TMEM owner and single-thread tcgen05.mma issuer
+//   warp 10      mask warp: the key tile's boundary masks, their in-tile
+//                prefix / suffix ORs and the tile's descriptor
+// TMEM holds S twice (tiles of even and odd index) and O twice (items of even
+// and odd index): S(g+1) = Q K^T is issued before O += P(g) V, so the tensor
+// core computes the next tile's scores while the softmax works on the
+// current one; the softmax turns S into bf16 P written back over S, and the
+// PV MMA reads P from TMEM. The two warps sharing a row exchange their half
+// maxima per tile and their half sums per item through shared memory.
 //
 // Weights. P_ij = c_ij 2^(S_ij log2(e)/sqrt(d) - m): the count multiplies the
 // exponential as an exact small-integer float, so no logarithm is taken.
@@ -71,14 +72,16 @@ using namespace sm100;
 
 constexpr int kTile = PLSH_TILE;
 constexpr int kD = 128;
-constexpr int kThreads = 384;  // 12 warps
-constexpr int kSlots = 2;
+constexpr int kThreads = 352;  // 11 warps
+constexpr int kSoftmaxWarps = 8;
+constexpr int kWarpTma = 8, kWarpMma = 9, kWarpMask = 10;
+constexpr int kStages = 2;     // K and V buffers
 constexpr int kMaskStages = 2;
 constexpr int kChunkBytes = kTile * 64 * 2;  // 128 rows x 64 bf16 = 16 KB (one SW128 box)
 constexpr int kTileBytes = 2 * kChunkBytes;  // 128 x 128 bf16 = 32 KB
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;              // S (then P) of slot z at columns 128 z
-constexpr uint32_t kColO = 256;            // O of slot z at columns 256 + 128 z
+constexpr uint32_t kColS = 0;              // S (then P) of tile g at columns 128 (g % 2)
+constexpr uint32_t kColO = 256;            // O of item k at columns 256 + 128 (k % 2)
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kMaxSortedHeads = 256;
 constexpr uint64_t kDrainNs = 100000000ull;
@@ -91,33 +94,33 @@ struct alignas(16) MaskStage {
   // range ORs against the 32-row block of warp q (diagonal tile only):
   // dq[q][c] = OR bm[c + 1 .. 32q] for c < 32q, OR bm[32q + 32 .. c] for c >= 32q + 32
   MaskT dq[4][kTile];
-  // the tile as the softmax needs it: valid (0 = end of the slot's work), kind (0 diagonal,
+  // the tile as the softmax needs it: valid (0 = end of the CTA's work), kind (0 diagonal,
   // 1 below, 2 above), first / last tile of its item, item index x
   int valid, kind, first, last, x, pad0, pad1, pad2;
 };
 
-struct alignas(1024) SlotBuffers {
-  uint8_t q[kTileBytes];
-  uint8_t k[kTileBytes];
-  uint8_t v[kTileBytes];
-};
-
 template <typename MaskT>
 struct __align__(1024) TcSmem {
-  SlotBuffers slot[kSlots];
-  MaskStage<MaskT> m[kSlots][kMaskStages];
+  uint8_t q[2][kTileBytes];
+  uint8_t k[kStages][kTileBytes];
+  uint8_t v[kStages][kTileBytes];
+  MaskStage<MaskT> m[kMaskStages];
+  float pmax[2][2][kTile];         // [tile parity][key half][row] half maxima of S
+  float psum[2][2][kTile];         // [item parity][key half][row] half sums of P
   int16_t order[kMaxSortedHeads];  // heads by decreasing window width
   int32_t width[kMaxSortedHeads];
-  uint64_t q_full[kSlots], q_empty[kSlots];
-  uint64_t k_full[kSlots], k_empty[kSlots];
-  uint64_t v_full[kSlots], v_empty[kSlots];
-  uint64_t m_full[kSlots][kMaskStages], m_empty[kSlots][kMaskStages];
-  uint64_t s_full[kSlots], p_full[kSlots], o_full[kSlots];
+  uint64_t q_full[2], q_empty[2];
+  uint64_t k_full[kStages], k_empty[kStages];
+  uint64_t v_full[kStages], v_empty[kStages];
+  uint64_t m_full[kMaskStages], m_empty[kMaskStages];
+  uint64_t s_full[2], p_full[2], pv_done[2];
+  uint64_t xmax[2], xsum[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
 };
 
+static_assert(kStages == 2, "the descriptor selects assume two K/V stages");
 static_assert(sizeof(TcSmem<unsigned long long>) + 1024 <= 232448, "shared memory budget");
 
 struct Params {
@@ -127,7 +130,7 @@ struct Params {
   const int32_t* spans;
 };
 
-// The key tiles of one slot's work items, in the order every role walks them:
+// The key tiles of a CTA's work items, in the order every role walks them:
 // items x0, x0 + stride, ...; within an item the diagonal tile, then the tiles
 // below, then (non-causal) the tiles above. For the per-sample comparator an
 // item is walked once per hash k (a sub-item), each time over that hash's
@@ -137,13 +140,13 @@ struct TileIter {
   const Params* p;
   const int16_t* order;
   int x, stride;
-  int k;        // items started so far by this slot
+  int k;        // items started so far by this CTA
   int sub;      // sub-item (hash) within the item: 0 for K3
   int it;       // key tile within the sub-item
   int total;    // key tiles of the sub-item
   int n_below;
   int b, h, i0;
-  int g;        // key tiles so far by this slot
+  int g;        // key tiles so far by this CTA
   bool valid;
   bool bad_window;  // the window read for this sub-item was out of range (and was clamped)
   int nx_lo, nx_hi;
@@ -184,11 +187,11 @@ struct TileIter {
     sub = 0;
     load_sub(lo, hi);
   }
-  __device__ __forceinline__ void start(const Params* pp, const int16_t* ord, int slot) {
+  __device__ __forceinline__ void start(const Params* pp, const int16_t* ord) {
     p = pp;
     order = ord;
-    x = blockIdx.x + slot * gridDim.x;
-    stride = kSlots * gridDim.x;
+    x = blockIdx.x;
+    stride = gridDim.x;
     k = 0;
     g = 0;
     nx_lo = nx_hi = 0;
@@ -254,6 +257,14 @@ __device__ __forceinline__ MaskT warp_suffix_or(MaskT v, int lane) {  // inclusi
     if (lane + o < 32) v |= y;
   }
   return v;
+}
+
+// Orders every later use of r after the preceding tcgen05.wait::ld (the registers of an
+// asynchronous TMEM load are only valid after the wait).
+template <int N>
+__device__ __forceinline__ void regs_after_wait(uint32_t (&r)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
 }
 
 __device__ __forceinline__ float max32(const uint32_t (&v)[32], float m) {
@@ -403,25 +414,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   }
   if (threadIdx.x == 0) {
     sm.abort_flag = 0;
-    for (int z = 0; z < kSlots; ++z) {
-      mbar_init(&sm.q_full[z], 1);
-      mbar_init(&sm.q_empty[z], 1);
-      mbar_init(&sm.k_full[z], 1);
-      mbar_init(&sm.k_empty[z], 1);
-      mbar_init(&sm.v_full[z], 1);
-      mbar_init(&sm.v_empty[z], 1);
-      mbar_init(&sm.s_full[z], 1);
-      mbar_init(&sm.p_full[z], 4);
-      mbar_init(&sm.o_full[z], 1);
-      for (int i = 0; i < kMaskStages; ++i) {
-        mbar_init(&sm.m_full[z][i], 1);
-        mbar_init(&sm.m_empty[z][i], 4);
-      }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.q_full[i], 1);
+      mbar_init(&sm.q_empty[i], 1);
+      mbar_init(&sm.k_full[i], 1);
+      mbar_init(&sm.k_empty[i], 1);
+      mbar_init(&sm.v_full[i], 1);
+      mbar_init(&sm.v_empty[i], 1);
+      mbar_init(&sm.s_full[i], 1);
+      mbar_init(&sm.p_full[i], kSoftmaxWarps);
+      mbar_init(&sm.pv_done[i], 1);
+      mbar_init(&sm.xmax[i], kSoftmaxWarps);
+      mbar_init(&sm.xsum[i], kSoftmaxWarps);
+    }
+    for (int i = 0; i < kMaskStages; ++i) {
+      mbar_init(&sm.m_full[i], 1);
+      mbar_init(&sm.m_empty[i], kSoftmaxWarps);
     }
     mbar_init(&sm.drain, 1);
     fence_mbarrier_init();
   }
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     tmem_alloc(&sm.tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -430,163 +443,123 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer (both slots)
-    // Six streams, Q (per item), K and V (per key tile) of each slot, each issued as soon as
-    // its buffer is free; the thread polls, so one slot's stall never holds up the other.
+  if (warp == kWarpTma) {
+    // ------------------------------------------------------------ TMA producer
+    // Q per item (two buffers by item parity), K and V per key tile (two stages each).
     if (lane == 0) {
       tma_prefetch_desc(&tmap_q);
       tma_prefetch_desc(&tmap_k);
       tma_prefetch_desc(&tmap_v);
-      TileIter<kVarlen> kit[kSlots], vit[kSlots];
-      for (int z = 0; z < kSlots; ++z) {
-        kit[z].start(&prm, sm.order, z);
-        vit[z].start(&prm, sm.order, z);
-      }
-      uint64_t idle_since = 0;
-      uint32_t spins = 0;
-      while (kit[0].valid || kit[1].valid || vit[0].valid || vit[1].valid) {
-        bool progress = false;
-#pragma unroll
-        for (int z = 0; z < kSlots; ++z) {
-          TileIter<kVarlen>& ki = kit[z];
-          if (ki.valid) {
-            // Q of a new item once the slot's previous item has run its last S; K(g) once S(g-1) has run
-            const bool q_ok = !ki.first() || ki.k == 0 || mbar_test_wait(&sm.q_empty[z], (ki.k - 1) & 1);
-            const bool k_ok = ki.g == 0 || mbar_test_wait(&sm.k_empty[z], (ki.g - 1) & 1);
-            if (q_ok && k_ok) {
-              if (ki.first()) {
-                mbar_arrive_expect_tx(&sm.q_full[z], kTileBytes);
-                tma_load_3d(sm.slot[z].q, &tmap_q, 0, ki.i0, ki.b * H + ki.h, &sm.q_full[z]);
-                tma_load_3d(sm.slot[z].q + kChunkBytes, &tmap_q, 64, ki.i0, ki.b * H + ki.h, &sm.q_full[z]);
-              }
-              const int zkv = ki.b * prm.H_kv + ki.h / (H / prm.H_kv);
-              const int j0 = ki.j0();
-              mbar_arrive_expect_tx(&sm.k_full[z], kTileBytes);
-              tma_load_3d(sm.slot[z].k, &tmap_k, 0, j0, zkv, &sm.k_full[z]);
-              tma_load_3d(sm.slot[z].k + kChunkBytes, &tmap_k, 64, j0, zkv, &sm.k_full[z]);
-              ki.next();
-              progress = true;
-            }
-          }
-          TileIter<kVarlen>& vi = vit[z];
-          if (vi.valid && (vi.g == 0 || mbar_test_wait(&sm.v_empty[z], (vi.g - 1) & 1))) {
-            const int zkv = vi.b * prm.H_kv + vi.h / (H / prm.H_kv);
-            const int j0 = vi.j0();
-            mbar_arrive_expect_tx(&sm.v_full[z], kTileBytes);
-            tma_load_3d(sm.slot[z].v, &tmap_v, 0, j0, zkv, &sm.v_full[z]);
-            tma_load_3d(sm.slot[z].v + kChunkBytes, &tmap_v, 64, j0, zkv, &sm.v_full[z]);
-            vi.next();
-            progress = true;
-          }
+      TileIter<kVarlen> ti;
+      ti.start(&prm, sm.order);
+      int issued_g = 0, issued_v = 0, issued_k = 0;  // K tiles, V tiles and Q items issued
+      while (ti.valid) {
+        const int zkv = ti.b * prm.H_kv + ti.h / (H / prm.H_kv);
+        if (ti.first()) {
+          const int qb = ti.k & 1;
+          if (ti.k >= 2 && !mbar_wait(&sm.q_empty[qb], ((ti.k >> 1) & 1) ^ 1, abort_flag, err)) break;
+          mbar_arrive_expect_tx(&sm.q_full[qb], kTileBytes);
+          tma_load_3d(sm.q[qb], &tmap_q, 0, ti.i0, ti.b * H + ti.h, &sm.q_full[qb]);
+          tma_load_3d(sm.q[qb] + kChunkBytes, &tmap_q, 64, ti.i0, ti.b * H + ti.h, &sm.q_full[qb]);
+          issued_k = ti.k + 1;
         }
-        if (progress) {
-          idle_since = 0;
-          spins = 0;
-        } else if ((++spins & 63u) == 0) {
-          const uint64_t now = global_timer_ns();
-          if (idle_since == 0) idle_since = now;
-          if (*abort_flag) break;
-          if (now - idle_since > kWaitLimitNs) {
-            *abort_flag = 1;
-            atomicOr(err, PLSH_DEVERR_TIMEOUT);
-            break;
-          }
-        }
+        const int st = ti.g % kStages;
+        const uint32_t ph = static_cast<uint32_t>(ti.g / kStages) & 1u;
+        const int j0 = ti.j0();
+        if (ti.g >= kStages && !mbar_wait(&sm.k_empty[st], ph ^ 1u, abort_flag, err)) break;
+        mbar_arrive_expect_tx(&sm.k_full[st], kTileBytes);
+        tma_load_3d(sm.k[st], &tmap_k, 0, j0, zkv, &sm.k_full[st]);
+        tma_load_3d(sm.k[st] + kChunkBytes, &tmap_k, 64, j0, zkv, &sm.k_full[st]);
+        issued_g = ti.g + 1;
+        if (ti.g >= kStages && !mbar_wait(&sm.v_empty[st], ph ^ 1u, abort_flag, err)) break;
+        mbar_arrive_expect_tx(&sm.v_full[st], kTileBytes);
+        tma_load_3d(sm.v[st], &tmap_v, 0, j0, zkv, &sm.v_full[st]);
+        tma_load_3d(sm.v[st] + kChunkBytes, &tmap_v, 64, j0, zkv, &sm.v_full[st]);
+        issued_v = ti.g + 1;
+        ti.next();
       }
       if (*abort_flag) {
         // let every copy already issued land before the CTA can exit
-        for (int z = 0; z < kSlots; ++z) {
-          const int q_issued = kit[z].k + ((kit[z].valid && !kit[z].first()) ? 1 : 0);
-          if (q_issued > 0) mbar_wait_drain(&sm.q_full[z], (q_issued - 1) & 1, kDrainNs);
-          if (kit[z].g > 0) mbar_wait_drain(&sm.k_full[z], (kit[z].g - 1) & 1, kDrainNs);
-          if (vit[z].g > 0) mbar_wait_drain(&sm.v_full[z], (vit[z].g - 1) & 1, kDrainNs);
-        }
+        for (int kk = (issued_k > 2 ? issued_k - 2 : 0); kk < issued_k; ++kk)
+          mbar_wait_drain(&sm.q_full[kk & 1], (kk >> 1) & 1, kDrainNs);
+        for (int gg = (issued_g > kStages ? issued_g - kStages : 0); gg < issued_g; ++gg)
+          mbar_wait_drain(&sm.k_full[gg % kStages], static_cast<uint32_t>(gg / kStages) & 1u, kDrainNs);
+        for (int gg = (issued_v > kStages ? issued_v - kStages : 0); gg < issued_v; ++gg)
+          mbar_wait_drain(&sm.v_full[gg % kStages], static_cast<uint32_t>(gg / kStages) & 1u, kDrainNs);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (both slots)
-    // Per slot: S(g) needs Q, K(g) and PV(g-1) issued (P of g-1 lives in S's columns; the tensor
-    // core runs one thread's MMAs in order); PV(g) needs P(g) and V(g).
+  } else if (warp == kWarpMma) {
+    // ------------------------------------------------------------ MMA issuer
+    // S of the next tile is issued before PV of the current one: S is double-buffered in TMEM
+    // and S(g+1) computes while the softmax works on S(g). P(g-1) lives in S(g+1)'s buffer; it is
+    // read by PV(g-1), which was issued before S(g+1), and the tensor core runs them in order.
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, 1);
-      TileIter<kVarlen> st_it[kSlots], pv_it[kSlots];
-      uint64_t q_desc[kSlots], k_desc[kSlots], v_desc[kSlots];
-      for (int z = 0; z < kSlots; ++z) {
-        st_it[z].start(&prm, sm.order, z);
-        pv_it[z].start(&prm, sm.order, z);
-        q_desc[z] = smem_desc_sw128(smem_u32(sm.slot[z].q), 16, 1024);
-        k_desc[z] = smem_desc_sw128(smem_u32(sm.slot[z].k), 16, 1024);
-        v_desc[z] = smem_desc_sw128(smem_u32(sm.slot[z].v), kChunkBytes, 1024);
+      uint64_t q_desc[2], k_desc[kStages], v_desc[kStages];
+      for (int i = 0; i < 2; ++i) q_desc[i] = smem_desc_sw128(smem_u32(sm.q[i]), 16, 1024);
+      for (int i = 0; i < kStages; ++i) {
+        k_desc[i] = smem_desc_sw128(smem_u32(sm.k[i]), 16, 1024);
+        v_desc[i] = smem_desc_sw128(smem_u32(sm.v[i]), kChunkBytes, 1024);
       }
-      uint64_t idle_since = 0;
-      uint32_t spins = 0;
-      while (pv_it[0].valid || pv_it[1].valid) {
-        bool progress = false;
+      auto issue_s = [&](const TileIter<kVarlen>& ti) -> bool {
+        const int qb = ti.k & 1;
+        if (ti.first() && !mbar_wait(&sm.q_full[qb], (ti.k >> 1) & 1, abort_flag, err)) return false;
+        const int st = ti.g % kStages;
+        if (!mbar_wait(&sm.k_full[st], static_cast<uint32_t>(ti.g / kStages) & 1u, abort_flag, err)) return false;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + kColS + 128u * static_cast<uint32_t>(ti.g & 1);
 #pragma unroll
-        for (int z = 0; z < kSlots; ++z) {
-          TileIter<kVarlen>& si = st_it[z];
-          TileIter<kVarlen>& pi = pv_it[z];
-          // PV first: it frees the slot's S columns for the next S
-          if (pi.valid && pi.g < si.g && mbar_test_wait(&sm.p_full[z], pi.g & 1) &&
-              mbar_test_wait(&sm.v_full[z], pi.g & 1)) {
-            tc_fence_after();
-            const uint32_t p_tmem = tmem + kColS + 128u * z;
-            const uint32_t o_tmem = tmem + kColO + 128u * z;
-#pragma unroll
-            for (int kk = 0; kk < kTile / 16; ++kk) {
-              // keys 16kk..16kk+15: P at columns 8kk..8kk+7; the keys are two 8-row groups of the
-              // MN-major V tile, whose two d halves sit kChunkBytes apart
-              mma_ts(o_tmem, p_tmem + 8u * kk, v_desc[z] + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
-                     (!pi.first() || kk > 0) ? 1u : 0u);
-            }
-            mma_commit(&sm.v_empty[z]);
-            if (pi.last()) mma_commit(&sm.o_full[z]);
-            pi.next();
-            progress = true;
-          }
-          if (si.valid && si.g == pi.g && (!si.first() || mbar_test_wait(&sm.q_full[z], si.k & 1)) &&
-              mbar_test_wait(&sm.k_full[z], si.g & 1)) {
-            tc_fence_after();
-            const uint32_t d_tmem = tmem + kColS + 128u * z;
-#pragma unroll
-            for (int kk = 0; kk < kD / 16; ++kk) {
-              // the descriptors' start address field counts 16-byte units
-              const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
-              mma_ss(d_tmem, q_desc[z] + off, k_desc[z] + off, idesc_qk, kk > 0 ? 1u : 0u);
-            }
-            mma_commit(&sm.s_full[z]);
-            mma_commit(&sm.k_empty[z]);
-            if (si.last()) mma_commit(&sm.q_empty[z]);
-            si.next();
-            progress = true;
-          }
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          // the descriptors' start address field counts 16-byte units
+          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
+          mma_ss(d_tmem, (qb ? q_desc[1] : q_desc[0]) + off, (st ? k_desc[1] : k_desc[0]) + off, idesc_qk,
+                 kk > 0 ? 1u : 0u);
         }
-        if (progress) {
-          idle_since = 0;
-          spins = 0;
-        } else if ((++spins & 63u) == 0) {
-          const uint64_t now = global_timer_ns();
-          if (idle_since == 0) idle_since = now;
-          if (*abort_flag) break;
-          if (now - idle_since > kWaitLimitNs) {
-            *abort_flag = 1;
-            atomicOr(err, PLSH_DEVERR_TIMEOUT);
-            break;
-          }
+        mma_commit(&sm.s_full[ti.g & 1]);
+        mma_commit(&sm.k_empty[st]);
+        if (ti.last()) mma_commit(&sm.q_empty[qb]);
+        return true;
+      };
+      auto issue_pv = [&](const TileIter<kVarlen>& ti) -> bool {
+        const int st = ti.g % kStages;
+        if (!mbar_wait(&sm.p_full[ti.g & 1], static_cast<uint32_t>(ti.g >> 1) & 1u, abort_flag, err)) return false;
+        if (!mbar_wait(&sm.v_full[st], static_cast<uint32_t>(ti.g / kStages) & 1u, abort_flag, err)) return false;
+        tc_fence_after();
+        const uint32_t p_tmem = tmem + kColS + 128u * static_cast<uint32_t>(ti.g & 1);
+        const uint32_t o_tmem = tmem + kColO + 128u * static_cast<uint32_t>(ti.k & 1);
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk) {
+          // keys 16kk..16kk+15: P of key half kk/4 at columns 64 (kk/4) + 8 (kk%4); the keys are two
+          // 8-row groups of the MN-major V tile, whose two d halves sit kChunkBytes apart
+          mma_ts(o_tmem, p_tmem + 64u * (kk >> 2) + 8u * (kk & 3),
+                 (st ? v_desc[1] : v_desc[0]) + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
+                 (!ti.first() || kk > 0) ? 1u : 0u);
         }
+        mma_commit(&sm.pv_done[ti.g & 1]);
+        mma_commit(&sm.v_empty[st]);
+        return true;
+      };
+      TileIter<kVarlen> cur, nxt;
+      cur.start(&prm, sm.order);
+      nxt.start(&prm, sm.order);
+      bool ok = !cur.valid || issue_s(cur);
+      if (nxt.valid) nxt.next();
+      while (ok && cur.valid) {
+        if (nxt.valid) ok = issue_s(nxt);
+        if (ok) ok = issue_pv(cur);
+        cur.next();
+        if (nxt.valid) nxt.next();
       }
       // every MMA issued so far completes before `drain` arrives
       mma_commit(&sm.drain);
       mbar_wait_drain(&sm.drain, 0, kDrainNs);
     }
-  } else if (warp == 2 || warp == 3) {
-    // ------------------------------------------------------------ mask warp of slot (warp - 2)
-    const int z = warp - 2;
+  } else if (warp == kWarpMask) {
+    // ------------------------------------------------------------ mask warp
     TileIter<kVarlen> ti, nx;
-    ti.start(&prm, sm.order, z);
-    nx.start(&prm, sm.order, z);
+    ti.start(&prm, sm.order);
+    nx.start(&prm, sm.order);
     if (nx.valid) nx.next();
     // the masks of a tile; a comparator sub-item keeps only its own hash's bit
     auto load_masks = [&](const TileIter<kVarlen>& t, MaskT (&v)[4], MaskT& v128) {
@@ -610,13 +583,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       MaskT nv[4] = {FULL, FULL, FULL, FULL}, n128 = FULL;
       if (nx.valid) load_masks(nx, nv, n128);  // lands while this tile is processed
       if (ti.g >= kMaskStages) {
-        ok = mbar_wait(&sm.m_empty[z][st], (static_cast<uint32_t>(ti.g / kMaskStages) & 1u) ^ 1u, abort_flag, err);
+        ok = mbar_wait(&sm.m_empty[st], (static_cast<uint32_t>(ti.g / kMaskStages) & 1u) ^ 1u, abort_flag, err);
         if (!__all_sync(0xffffffffu, ok)) {
           ok = false;
           break;
         }
       }
-      MaskStage<MaskT>& ms = sm.m[z][st];
+      MaskStage<MaskT>& ms = sm.m[st];
       MaskT pre_v[4], suf_v[4];
       {  // pre[c] = OR bm[1..c]
         const MaskT p0 = lane == 0 ? static_cast<MaskT>(0) : xv[0];
@@ -689,7 +662,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         if (ti.first() && ti.bad_window) atomicOr(err, PLSH_DEVERR_WINDOW);
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.m_full[z][st]);
+      if (lane == 0) mbar_arrive(&sm.m_full[st]);
       g_end = ti.g + 1;
       ti.next();
       if (nx.valid) nx.next();
@@ -701,33 +674,31 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     if (ok && !*abort_flag) {
       const int st = g_end % kMaskStages;
       ok = g_end < kMaskStages ||
-           mbar_wait(&sm.m_empty[z][st], (static_cast<uint32_t>(g_end / kMaskStages) & 1u) ^ 1u, abort_flag, err);
+           mbar_wait(&sm.m_empty[st], (static_cast<uint32_t>(g_end / kMaskStages) & 1u) ^ 1u, abort_flag, err);
       if (__all_sync(0xffffffffu, ok) && lane == 0) {
-        sm.m[z][st].valid = 0;
-        mbar_arrive(&sm.m_full[z][st]);
+        sm.m[st].valid = 0;
+        mbar_arrive(&sm.m_full[st]);
       }
     }
   } else {
-    // ------------------------------------------------------------ softmax of slot (warp - 4) / 4
-    const int z = (warp - 4) >> 2;
+    // ------------------------------------------------------------ softmax: quarter warp & 3, key half warp >> 2
     const int quarter = warp & 3;
+    const int hf = warp >> 2;           // this warp's key half: keys [64 hf, 64 hf + 64) of every tile
     const int r = quarter * 32 + lane;  // row within the tile == TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t s_base = tmem + lane_off + kColS + 128u * z;
-    const uint32_t o_base = tmem + lane_off + kColO + 128u * z;
     const float sc = 1.4426950408889634f / sqrtf(static_cast<float>(kD));
     // weights count hashes: all s of them, or (comparator) the one hash of the sub-item
     const int sw = kVarlen ? 1 : s;
     const float cs = 8388608.0f + static_cast<float>(sw);  // 2^23 + sw
     float m2 = -INFINITY, l = 0.0f;
     MaskT Y = 0, Z = 0;
-    int items_done = 0;
+    int items = 0;  // items finished by this warp
     for (int g = 0;; ++g) {
       const int st = g % kMaskStages;
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.m_full[z][st], static_cast<uint32_t>(g / kMaskStages) & 1u,
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.m_full[st], static_cast<uint32_t>(g / kMaskStages) & 1u,
                                              abort_flag, err)))
         break;
-      const MaskStage<MaskT>& ms = sm.m[z][st];
+      const MaskStage<MaskT>& ms = sm.m[st];
       if (!ms.valid) break;
       const int kind = ms.kind, first = ms.first, last = ms.last, tx = ms.x;
       if (first) {
@@ -738,24 +709,37 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       uint32_t cnt[8];
       MaskT lo = 0, hi = 0;
       if (kind == 0) diag_scan<MaskT, kCausal>(ms, quarter, r, sw, cnt, lo, hi);
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[z], static_cast<uint32_t>(g & 1), abort_flag, err)))
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[g & 1], static_cast<uint32_t>(g >> 1) & 1u, abort_flag, err)))
         break;
       tc_fence_after();
+      const uint32_t s_base = tmem + lane_off + kColS + 128u * static_cast<uint32_t>(g & 1);
 
-      // ---- pass 1: the tile maximum of S over the 16-key chunks that can carry weight (when
-      // causal, the diagonal tile's chunks past the warp's own block cannot)
+      // ---- pass 1: this half's maximum of S over the 16-key chunks that can carry weight (when
+      // causal, the diagonal tile's chunks past the warp's own block cannot); exchange with the
+      // other half of the row
       const int n_live = (kCausal && kind == 0) ? 2 * quarter + 2 : kTile / 16;
       float mraw = -INFINITY;
-#pragma unroll 1
-      for (int ch = 0; ch < n_live; ch += 2) {
-        uint32_t sv[32];
-        tmem_ld32(s_base + 16u * ch, sv);
+      {
+        const int c0 = 4 * hf;
+        uint32_t sa[32], sb[32];
+        if (c0 < n_live) tmem_ld32(s_base + 16u * c0, sa);
+        if (c0 + 2 < n_live) tmem_ld32(s_base + 16u * (c0 + 2), sb);
         tmem_wait_ld();
-        mraw = max32(sv, mraw);
+        regs_after_wait(sa);
+        regs_after_wait(sb);
+        if (c0 < n_live) mraw = max32(sa, mraw);
+        if (c0 + 2 < n_live) mraw = max32(sb, mraw);
       }
+      sm.pmax[g & 1][hf][r] = mraw;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.xmax[g & 1]);
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.xmax[g & 1], static_cast<uint32_t>(g >> 1) & 1u, abort_flag, err)))
+        break;
+      mraw = fmaxf(mraw, sm.pmax[g & 1][hf ^ 1][r]);
       const float mt = mraw * sc;
 
-      // ---- reference update; O is rescaled in place (s_full(g) fired after PV(g-1) had completed)
+      // ---- reference update (the same in both halves); this half of O is rescaled in place once
+      // PV(g-1) has completed
       float alpha = 1.0f;
       bool need_rescale = false;
       if (mt > m2 + kRescaleThreshold) {
@@ -767,23 +751,29 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       }
       const float neg_m = -m2;
       if (__any_sync(0xffffffffu, need_rescale)) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.pv_done[(g - 1) & 1], static_cast<uint32_t>((g - 1) >> 1) & 1u,
+                                               abort_flag, err)))
+          break;
+        tc_fence_after();
+        const uint32_t o_half = tmem + lane_off + kColO + 128u * static_cast<uint32_t>(items & 1) + 64u * hf;
 #pragma unroll 1
-        for (int q4 = 0; q4 < 8; ++q4) {
+        for (int q4 = 0; q4 < 4; ++q4) {
           uint32_t raw[16];
-          tmem_ld16(o_base + 16u * q4, raw);
+          tmem_ld16(o_half + 16u * q4, raw);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 16; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * alpha);
-          tmem_st16(o_base + 16u * q4, raw);
+          tmem_st16(o_half + 16u * q4, raw);
         }
       }
 
-      // ---- pass 2: P = c 2^(S sc - m) chunk by chunk; P of keys [16ch, 16ch + 16) goes to columns
-      // [8ch, 8ch + 8), over S columns already read
+      // ---- pass 2: P = c 2^(S sc - m) for this half's 4 chunks; P of chunk 4 hf + c goes to
+      // columns 64 hf + 8c, over S columns of this half already read
       const MaskT Zc = static_cast<MaskT>(Z | ms.bm[0]);
       float lsum = 0.0f;
 #pragma unroll 1
-      for (int ch = 0; ch < kTile / 16; ++ch) {
+      for (int c = 0; c < 4; ++c) {
+        const int ch = 4 * hf + c;
         uint32_t pk[8];
         if (ch >= n_live) {
 #pragma unroll
@@ -792,6 +782,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
           uint32_t sv[16];
           tmem_ld16(s_base + 16u * ch, sv);
           tmem_wait_ld();
+          regs_after_wait(sv);
           if (kind == 0 && (ch >> 1) == quarter) {
             // the warp's own block on the diagonal: counts from the scan
             uint32_t c4[4];
@@ -799,14 +790,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
             for (int u = 0; u < 4; ++u) c4[u] = (ch & 1) ? cnt[4 + u] : cnt[u];
             lsum += p16_counts(sv, c4, sc, neg_m, pk);
           } else {
-            // below: Y | suf[c]; above: Z | bm[0] | pre[c]; diagonal: lo | dq[c] below the
-            // warp's block, hi | dq[c] above it
+            // below: Y | suf[c]; above: Z | bm[0] | pre[c]; diagonal: lo | dq[c] below the warp's
+            // block, hi | dq[c] above it
             const MaskT* km = kind == 1 ? ms.suf : (kind == 2 ? ms.pre : ms.dq[quarter]);
             const MaskT carry = kind == 1 ? Y : (kind == 2 ? Zc : ((ch >> 1) < quarter ? lo : hi));
             lsum += p16_carry<MaskT>(sv, km + 16 * ch, carry, sc, neg_m, cs, pk);
           }
         }
-        tmem_st8(s_base + 8u * ch, pk);
+        tmem_st8(s_base + 64u * hf + 8u * c, pk);
       }
       if (kind == 1) {
         Y = static_cast<MaskT>(Y | ms.bm[0] | ms.suf[0]);  // OR over [j0, i]
@@ -817,32 +808,39 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         if (!kCausal) Z = ms.suf[r];                        // OR over (i, i0 + 127]
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.m_empty[z][st]);
+      if (lane == 0) mbar_arrive(&sm.m_empty[st]);
       tmem_wait_st();
       l = l * alpha + lsum;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.p_full[z]);
+      if (lane == 0) mbar_arrive(&sm.p_full[g & 1]);
 
-      // ---- the item's epilogue: O / l, stored four rows at a time by each lane quad
+      // ---- the item's epilogue: this half of O / l, stored four rows at a time by each lane quad
       if (last) {
-        const bool o_ok = mbar_wait(&sm.o_full[z], static_cast<uint32_t>(items_done & 1), abort_flag, err);
-        if (!__all_sync(0xffffffffu, o_ok)) break;
-        ++items_done;
+        const int kb = items & 1;
+        sm.psum[kb][hf][r] = l;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.xsum[kb]);
+        const bool ok_sum = mbar_wait(&sm.xsum[kb], static_cast<uint32_t>(items >> 1) & 1u, abort_flag, err);
+        const bool ok_pv = ok_sum && mbar_wait(&sm.pv_done[g & 1], static_cast<uint32_t>(g >> 1) & 1u, abort_flag, err);
+        if (!__all_sync(0xffffffffu, ok_pv)) break;
         tc_fence_after();
+        const float ltot = l + sm.psum[kb][hf ^ 1][r];
         const int BT = prm.B * prm.T;
         const int hh = (H <= kMaxSortedHeads) ? static_cast<int>(sm.order[tx / BT]) : tx / BT;
         const int rem = tx % BT;
         const int bb = rem / prm.T, i0 = (rem % prm.T) * kTile;
-        const float inv = 1.0f / l;
+        const float inv = 1.0f / ltot;
         const int p4 = lane & 3;
         const int quad_row = quarter * 32 + (lane & ~3);  // first of the quad's four rows
-        __nv_bfloat16* obase = O + (static_cast<size_t>(bb) * H + hh) * static_cast<size_t>(n) * kD;
+        const uint32_t o_half = tmem + lane_off + kColO + 128u * static_cast<uint32_t>(kb) + 64u * hf;
+        __nv_bfloat16* obase = O + (static_cast<size_t>(bb) * H + hh) * static_cast<size_t>(n) * kD + 64 * hf;
 #pragma unroll 1
-        for (int blk = 0; blk < 4; ++blk) {
+        for (int blk = 0; blk < 2; ++blk) {
           uint32_t raw[32];
-          tmem_ld32(o_base + 32u * blk, raw);
+          tmem_ld32(o_half + 32u * blk, raw);
           tmem_wait_ld();
+          regs_after_wait(raw);
           uint32_t a[4][4];  // [16-byte chunk][word] of this row's 32 columns
 #pragma unroll
           for (int c = 0; c < 4; ++c)
@@ -853,15 +851,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
           // 4x4 transpose of 16-byte chunks inside the quad: lane p then holds chunk p of the quad's rows
 #pragma unroll
           for (int msk = 2; msk >= 1; msk >>= 1) {
-            const bool lo = (p4 & msk) == 0;
+            const bool lo_lane = (p4 & msk) == 0;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
               if (c & msk) continue;
 #pragma unroll
               for (int w = 0; w < 4; ++w) {
-                const uint32_t send = lo ? a[c | msk][w] : a[c][w];
+                const uint32_t send = lo_lane ? a[c | msk][w] : a[c][w];
                 const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, msk);
-                if (lo) a[c | msk][w] = recv;
+                if (lo_lane) a[c | msk][w] = recv;
                 else a[c][w] = recv;
               }
             }
@@ -876,16 +874,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         }
         tc_fence_before();
         const int i = i0 + r;
-        if (i < n)
+        if (hf == 0 && i < n)
           row_sum[(static_cast<size_t>(bb) * H + hh) * n + i] =
-              (log2f(l) + m2) * 0.6931471805599453f - logf(static_cast<float>(s));
+              (log2f(ltot) + m2) * 0.6931471805599453f - logf(static_cast<float>(s));
+        ++items;
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
@@ -952,8 +951,7 @@ int launch_tc_typed(const AttnArgs& a, cudaStream_t st) {
   const size_t smem = sizeof(TcSmem<MaskT>) + 1024;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_tc_kernel)");
-  const int want = ceil_div(prm.items, kSlots);
-  const int grid = want < sm_count() ? want : sm_count();
+  const int grid = prm.items < sm_count() ? prm.items : sm_count();
   kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, prm, a.sigma, a.table, static_cast<const MaskT*>(a.bmask),
                                      static_cast<__nv_bfloat16*>(a.O), a.row_sum, a.err);
   e = cudaGetLastError();
