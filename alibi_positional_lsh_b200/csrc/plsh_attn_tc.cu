@@ -107,6 +107,7 @@ struct __align__(1024) TcSmem {
   MaskStage<MaskT> m[kMaskStages];
   float pmax[2][2][kTile];         // [tile parity][key half][row] half maxima of S
   float psum[2][2][kTile];         // [item parity][key half][row] half sums of P
+  uint32_t cw[8][kSoftmaxWarps * 32];  // diagonal tile: own-block counts, one column per softmax thread
   int16_t order[kMaxSortedHeads];  // heads by decreasing window width
   int32_t width[kMaxSortedHeads];
   uint64_t q_full[2], q_empty[2];
@@ -327,33 +328,42 @@ __device__ __forceinline__ float p16_counts(const uint32_t (&sv)[16], const uint
 }
 
 // Diagonal tile, warp q (rows [32q, 32q + 32), row r): counts of the warp's own 32 keys, as bytes
-// (key 32q + k in byte k % 4 of cnt[k / 4]), and the carries for the other keys. Keys c <= r:
-// R = OR bm[c + 1 .. r], scanned from the row down; keys c > r: R = OR bm[r + 1 .. c]
-// (non-causal; count 0 when causal), scanned from the row up. On return
-// lo = OR bm[32q + 1 .. r] and hi = OR bm[r + 1 .. 32q + 31].
+// (key 32q + 4j + e in byte e of word j), written to this thread's column cw[j * ld] of shared
+// memory, and the carries for the other keys. Keys c <= r: R = OR bm[c + 1 .. r], scanned from
+// the row down; keys c > r: R = OR bm[r + 1 .. c] (non-causal; count 0 when causal), scanned
+// from the row up. On return lo = OR bm[32q + 1 .. r] and hi = OR bm[r + 1 .. 32q + 31].
 template <typename MaskT, bool kCausal>
-__device__ __forceinline__ void diag_scan(const MaskStage<MaskT>& ms, int q, int r, int s, uint32_t (&cnt)[8],
+__device__ __forceinline__ void diag_scan(const MaskStage<MaskT>& ms, int q, int r, int s, uint32_t* cw, int ld,
                                           MaskT& lo, MaskT& hi) {
   const MaskT* bq = ms.bm + 32 * q;
   const int rr = r - 32 * q;  // the row within the block, 0..31
-#pragma unroll
-  for (int u = 0; u < 8; ++u) cnt[u] = 0u;
   MaskT R = 0;
+#pragma unroll 1
+  for (int j = 7; j >= 0; --j) {
+    uint32_t acc = 0;
 #pragma unroll
-  for (int cc = 31; cc >= 0; --cc) {
-    if (cc < rr) R |= bq[cc + 1];
-    const uint32_t v = (cc <= rr) ? static_cast<uint32_t>(s - popc_m(R)) : 0u;
-    cnt[cc >> 2] |= v << (8 * (cc & 3));
+    for (int e = 3; e >= 0; --e) {
+      const int cc = 4 * j + e;
+      if (cc < rr) R |= bq[cc + 1];
+      acc = (acc << 8) | ((cc <= rr) ? static_cast<uint32_t>(s - popc_m(R)) : 0u);
+    }
+    cw[j * ld] = acc;
   }
   lo = R;
   MaskT R2 = 0;
   if (!kCausal) {
+#pragma unroll 1
+    for (int j = 0; j < 8; ++j) {
+      uint32_t acc = cw[j * ld];
 #pragma unroll
-    for (int cc = 0; cc < 32; ++cc) {
-      if (cc > rr) {
-        R2 |= bq[cc];
-        cnt[cc >> 2] |= static_cast<uint32_t>(s - popc_m(R2)) << (8 * (cc & 3));
+      for (int e = 0; e < 4; ++e) {
+        const int cc = 4 * j + e;
+        if (cc > rr) {
+          R2 |= bq[cc];
+          acc |= static_cast<uint32_t>(s - popc_m(R2)) << (8 * e);
+        }
       }
+      cw[j * ld] = acc;
     }
   }
   hi = R2;
@@ -612,7 +622,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       }
       // range ORs against each warp's 32-row block of the diagonal tile
       if (ti.kind() == 0) {
-#pragma unroll
+#pragma unroll 1
         for (int q = 1; q < 4; ++q) {  // dq[q][c] = OR bm[c + 1 .. 32q], c < 32q
           MaskT v[4];
 #pragma unroll
@@ -628,7 +638,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
           }
         }
         if (!kCausal) {
-#pragma unroll
+#pragma unroll 1
           for (int q = 0; q < 3; ++q) {  // dq[q][c] = OR bm[32q + 32 .. c], c >= 32q + 32
             MaskT v[4];
 #pragma unroll
@@ -706,9 +716,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         l = 0.0f;
       }
       // weights that need only the masks: the diagonal's own block and its carries
-      uint32_t cnt[8];
       MaskT lo = 0, hi = 0;
-      if (kind == 0) diag_scan<MaskT, kCausal>(ms, quarter, r, sw, cnt, lo, hi);
+      if (kind == 0) diag_scan<MaskT, kCausal>(ms, quarter, r, sw, &sm.cw[0][threadIdx.x], kSoftmaxWarps * 32, lo, hi);
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[g & 1], static_cast<uint32_t>(g >> 1) & 1u, abort_flag, err)))
         break;
       tc_fence_after();
@@ -787,7 +796,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
             // the warp's own block on the diagonal: counts from the scan
             uint32_t c4[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) c4[u] = (ch & 1) ? cnt[4 + u] : cnt[u];
+            for (int u = 0; u < 4; ++u) c4[u] = sm.cw[4 * (ch & 1) + u][threadIdx.x];
             lsum += p16_counts(sv, c4, sc, neg_m, pk);
           } else {
             // below: Y | suf[c]; above: Z | bm[0] | pre[c]; diagonal: lo | dq[c] below the warp's
