@@ -60,6 +60,9 @@ def _load() -> ctypes.CDLL:
     lib.plsh_attention_varlen_fwd.restype = i32
     lib.plsh_attention_varlen_fwd.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, i32, vp, vp, vp, i32,
                                               vp, ctypes.c_size_t, vp, vp, vp, vp]
+    lib.plsh_alibi_banded_fwd.restype = i32
+    lib.plsh_alibi_banded_fwd.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, ctypes.c_double, i32, vp, vp,
+                                          vp, vp]
     lib.plsh_attention_varlen_fwd_static.restype = i32
     lib.plsh_attention_varlen_fwd_static.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, i32, vp, vp,
                                                      vp, i32, vp, vp, vp, vp]
@@ -164,8 +167,16 @@ def plsh_attention_varlen_fwd_static(Q, K, V, dtype: int, B: int, H: int, H_kv: 
         _dev_ptr(err_dev, "err_dev"), _stream_ptr(stream)))
 
 
+def plsh_alibi_banded_fwd(Q, K, V, dtype: int, B: int, H: int, H_kv: int, n: int, d: int, sigma_dev, eps: float,
+                          causal: int, O, row_sum, err_dev, stream=None) -> None:
+    _check(_lib.plsh_alibi_banded_fwd(_dev_ptr(Q, "Q"), _dev_ptr(K, "K"), _dev_ptr(V, "V"), dtype, B, H, H_kv, n, d,
+                                      _dev_ptr(sigma_dev, "sigma_dev"), ctypes.c_double(eps), int(causal),
+                                      _dev_ptr(O, "O"), _dev_ptr(row_sum, "row_sum"), _dev_ptr(err_dev, "err_dev"),
+                                      _stream_ptr(stream)))
+
+
 def decode_device_error(word: int) -> list:
     return [name for bit, name in DEVERR_BITS.items() if word & bit]
 
 
-from .api import PlshForward, forward  # noqa: E402,F401
+from .api import PlshForward, fixed_blocks_table, forward  # noqa: E402,F401

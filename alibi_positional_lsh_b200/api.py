@@ -7,6 +7,7 @@ with torch) and runs the whole path:
   a3 plsh_window       (K2)     -> b_max, tile windows, boundary masks
   a4 plsh_attention_fwd (K3)    -> O, row_sum
   a5 plsh_attention_varlen_fwd (K4, the per-sample comparator) -> the same O, row_sum
+  plsh_alibi_banded_fwd (exact banded ALiBi, what the method approximates) -> T*, row_sum
 All arithmetic of a2..a5 runs in libplsh's CUDA kernels.
 """
 from __future__ import annotations
@@ -16,9 +17,9 @@ from typing import Optional, Sequence, Tuple
 import numpy as np
 import torch
 
-from . import (PLSH_BF16, PLSH_F32, PLSH_TILE, PlshError, decode_device_error, plsh_attention_fwd,
-               plsh_attention_varlen_fwd, plsh_draw_table, plsh_sample_bins, plsh_varlen_scratch_bytes,
-               plsh_window)
+from . import (PLSH_BF16, PLSH_F32, PLSH_TILE, PlshError, decode_device_error, plsh_alibi_banded_fwd,
+               plsh_attention_fwd, plsh_attention_varlen_fwd, plsh_draw_table, plsh_sample_bins,
+               plsh_varlen_scratch_bytes, plsh_window)
 
 
 class PlshForward:
@@ -107,6 +108,20 @@ class PlshForward:
                                   self.row_sum, self.err, st)
         return self.O, self.row_sum
 
+    def attend_alibi(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, eps: float = 1e-4,
+                     stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+        """Exact ALiBi attention T* over the band |i - j| <= ceil(sigma_h ln(1/eps)) (needs no prepare())."""
+        B, H, H_kv, n, d = self.B, self.H, self.H_kv, self.n, self.d
+        if q.shape != (B, H, n, d) or k.shape != (B, H_kv, n, d) or v.shape != (B, H_kv, n, d):
+            raise ValueError("q/k/v shapes do not match the plan")
+        for t, nm in ((q, "q"), (k, "k"), (v, "v")):
+            if t.dtype != self.dtype or t.device != self.O.device:
+                raise ValueError(f"{nm} must be {self.dtype} on {self.O.device}")
+        st = torch.cuda.current_stream() if stream is None else stream
+        plsh_alibi_banded_fwd(q, k, v, self.dtype_code, B, H, H_kv, n, d, self.sigma_dev, float(eps),
+                              int(self.causal), self.O, self.row_sum, self.err, st)
+        return self.O, self.row_sum
+
     def __call__(self, q, k, v, stream=None, table=None):
         self.prepare(stream, table)
         return self.attend(q, k, v, stream)
@@ -142,6 +157,18 @@ class PlshForward:
         errs = self.device_errors()
         if errs:
             raise PlshError(-1, "device reported " + ",".join(errs))
+
+
+def fixed_blocks_table(H: int, block: float) -> np.ndarray:
+    """Table of the "fixed blocks" baseline: one hash per head with pitch `block` and offset 0, so
+    positions [k*block, (k+1)*block) form the blocks and every row attends inside its own block
+    (Results, Mistral-7B bullet: the fixed-blocks comparison). Pass it to PlshForward.prepare
+    (table=...) or __call__ with s = 1."""
+    if not block > 0:
+        raise ValueError("block must be > 0")
+    t = np.zeros((H, 1, 2), dtype=np.float64)
+    t[:, 0, 0] = float(block)
+    return t
 
 
 def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, sigma: Sequence[float], s: int, seed: int,

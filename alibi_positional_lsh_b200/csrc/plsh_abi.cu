@@ -1,6 +1,7 @@
 // Entry points of libplsh (declared in include/plsh.h): argument checks,
 // then the launch. Every check that can be made on the host is made here,
 // before anything is enqueued.
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -209,4 +210,31 @@ extern "C" int plsh_attention_varlen_fwd_static(const void* Q, const void* K, co
   plsh::AttnArgs a{Q, K, V, dtype, B, H, H_kv, n, d, s, causal, sigma_dev, table_dev,
                    spans, bmask_dev, O, row_sum, err_dev, 1};
   return plsh::launch_attention(a, st);
+}
+
+// ---------------------------------------------------------------- exact banded ALiBi (the competitor)
+
+extern "C" int plsh_alibi_banded_fwd(const void* Q, const void* K, const void* V, int dtype, int B, int H, int H_kv,
+                                     int n, int d, const double* sigma_dev, double eps, int causal, void* O,
+                                     float* row_sum, uint32_t* err_dev, void* stream) {
+  const char* fn = "plsh_alibi_banded_fwd";
+  if (H < 1 || n < 1) return fail(PLSH_ERR_INVALID_ARG, "%s: need H >= 1 and n >= 1 (H=%d n=%d)", fn, H, n);
+  if (H > 65535) return fail(PLSH_ERR_RANGE, "%s: H=%d exceeds 65535", fn, H);
+  if (n > (1 << 30)) return fail(PLSH_ERR_RANGE, "%s: n=%d exceeds 2^30", fn, n);
+  if (B < 1 || B > 65535) return fail(PLSH_ERR_INVALID_ARG, "%s: need 1 <= B <= 65535 (B=%d)", fn, B);
+  if (H_kv < 1 || H % H_kv != 0)
+    return fail(PLSH_ERR_INVALID_ARG, "%s: H_kv must divide H (H=%d H_kv=%d)", fn, H, H_kv);
+  if (causal != 0 && causal != 1) return fail(PLSH_ERR_INVALID_ARG, "%s: causal must be 0 or 1", fn);
+  if (dtype != PLSH_BF16 && dtype != PLSH_F32) return fail(PLSH_ERR_UNSUPPORTED, "%s: dtype %d", fn, dtype);
+  if (d != 64 && d != 128) return fail(PLSH_ERR_UNSUPPORTED, "%s: head dim %d (64 or 128 supported)", fn, d);
+  if (!(eps > 0.0 && eps < 1.0)) return fail(PLSH_ERR_INVALID_ARG, "%s: need 0 < eps < 1 (eps=%g)", fn, eps);
+  if (!Q || !K || !V || !O || !row_sum || !sigma_dev || !err_dev)
+    return fail(PLSH_ERR_INVALID_ARG, "%s: null pointer", fn);
+  if (!plsh::aligned16(Q) || !plsh::aligned16(K) || !plsh::aligned16(V) || !plsh::aligned16(O))
+    return fail(PLSH_ERR_INVALID_ARG, "%s: Q, K, V and O must be 16-byte aligned", fn);
+  if (static_cast<long long>(B) * H * plsh::ceil_div(n, PLSH_TILE) > 0x7fffffffLL)
+    return fail(PLSH_ERR_RANGE, "%s: too many query tiles", fn);
+  plsh::AttnArgs a{Q, K, V, dtype, B, H, H_kv, n, d, 1, causal, sigma_dev, nullptr,
+                   nullptr, nullptr, O, row_sum, err_dev, 0, 1, -std::log(eps)};
+  return plsh::launch_attention(a, static_cast<cudaStream_t>(stream));
 }

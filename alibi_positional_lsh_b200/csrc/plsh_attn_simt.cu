@@ -69,7 +69,7 @@ attn_simt_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __re
                  int H_kv, int n, int s, int causal, const double* __restrict__ sigma,
                  const double* __restrict__ table, const int32_t* __restrict__ spans,
                  const MaskT* __restrict__ bmask, T* __restrict__ O, float* __restrict__ row_sum,
-                 uint32_t* __restrict__ err, int varlen) {
+                 uint32_t* __restrict__ err, int varlen, int alibi, double log_inv_eps) {
   constexpr int TPR = D / 32;            // threads per query row
   constexpr int NT = kTile * TPR;
   constexpr int F4 = D / 4;              // float4 per row
@@ -113,19 +113,29 @@ attn_simt_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __re
   MaskT Y = 0, Z = 0;
 
   const size_t kv_base = (static_cast<size_t>(b) * H_kv + kvh) * static_cast<size_t>(n) * D;
-  const MaskT* bm_h = bmask + static_cast<size_t>(h) * n;
+  const MaskT* bm_h = alibi ? nullptr : bmask + static_cast<size_t>(h) * n;
   // K3: one pass over the union window with weights c_ij (sw = s). K4 (varlen): one pass per hash k
   // over that hash's window with the hash-k masks alone, so each weight is hash k's 0/1 block
   // indicator (sw = 1); the passes share the running maximum, sum and accumulator.
   const int n_pass = varlen ? s : 1;
   const int sw = varlen ? 1 : s;
+  // exact banded ALiBi: weight exp(-|i - j| / sigma_h) over |i - j| <= ceil(sigma_h ln(1/eps))
+  const float inv_sigma = alibi ? static_cast<float>(1.0 / sigma[h]) : 0.0f;
   const int last_row = min(n, i0 + kTile) - 1;
   for (int pass = 0; pass < n_pass; ++pass) {
     const MaskT bits = varlen ? static_cast<MaskT>(static_cast<MaskT>(1) << pass) : FULL;
     const size_t span_at = varlen ? ((static_cast<size_t>(h) * s + pass) * T_tiles + t) * 2
                                   : (static_cast<size_t>(h) * T_tiles + t) * 2;
-    int lo = spans[span_at];
-    int hi = spans[span_at + 1];
+    int lo, hi;
+    if (alibi) {
+      const double wr = ceil(sigma[h] * log_inv_eps);
+      const int reach = (wr >= static_cast<double>(n) || !(wr >= 0.0)) ? n : static_cast<int>(wr);
+      lo = max(0, i0 - reach);
+      hi = causal ? last_row : min(n - 1, last_row + reach);
+    } else {
+      lo = spans[span_at];
+      hi = spans[span_at + 1];
+    }
     if (lo < 0 || lo > i0 || hi >= n || hi < last_row) {
       flags |= PLSH_DEVERR_WINDOW;
       lo = max(0, min(lo, i0));
@@ -151,7 +161,7 @@ attn_simt_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __re
       }
       for (int c = tid; c <= kTile; c += NT) {
         const int j = j0 + c;
-        sm.bm[c] = static_cast<MaskT>(((j >= 0 && j < n) ? bm_h[j] : FULL) & bits);
+        sm.bm[c] = alibi ? static_cast<MaskT>(0) : static_cast<MaskT>(((j >= 0 && j < n) ? bm_h[j] : FULL) & bits);
       }
       __syncthreads();
       if (tid < kTile) {
@@ -188,7 +198,8 @@ attn_simt_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __re
         for (int cc = 0; cc < 32; ++cc) {
           const int c = chunk * 32 + cc;
           int w;
-          if (kind == 0) w = (causal && c > r) ? 0 : sm.wdiag[r * kDiagStride + c];
+          if (alibi) w = (causal && j0 + c > i) || j0 + c >= n ? 0 : 1;
+          else if (kind == 0) w = (causal && c > r) ? 0 : sm.wdiag[r * kDiagStride + c];
           else if (kind == 1) w = sw - popc_mask(static_cast<MaskT>(sm.suf[c] | Y));
           else w = sw - popc_mask(static_cast<MaskT>(Z | sm.pre[c]));
           float dot = 0.0f;
@@ -202,7 +213,8 @@ attn_simt_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __re
           }
   #pragma unroll
           for (int o = TPR / 2; o >= 1; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-          sv[cc] = w > 0 ? dot * scale : -INFINITY;
+          sv[cc] = w > 0 ? dot * scale - (alibi ? fabsf(static_cast<float>(i - (j0 + c))) * inv_sigma : 0.0f)
+                         : -INFINITY;
           wv[cc] = w;
         }
         float cmax = -INFINITY;
@@ -250,7 +262,7 @@ attn_simt_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __re
       store4(O + o_row + 4 * (part + TPR * m),
              make_float4(acc[4 * m] * inv, acc[4 * m + 1] * inv, acc[4 * m + 2] * inv, acc[4 * m + 3] * inv));
     if (part == 0)
-      row_sum[(static_cast<size_t>(b) * H + h) * n + i] = logf(l_run) + m_run - logf(static_cast<float>(s));
+      row_sum[(static_cast<size_t>(b) * H + h) * n + i] = logf(l_run) + m_run - (alibi ? 0.0f : logf(static_cast<float>(s)));
   }
   if (flags) atomicOr(err, flags);
 }
@@ -265,7 +277,7 @@ int launch_simt_typed(const AttnArgs& a, cudaStream_t st) {
   kern<<<grid, kTile * (D / 32), smem, st>>>(
       static_cast<const T*>(a.Q), static_cast<const T*>(a.K), static_cast<const T*>(a.V), a.H, a.H_kv, a.n, a.s,
       a.causal, a.sigma, a.table, a.spans, static_cast<const MaskT*>(a.bmask), static_cast<T*>(a.O), a.row_sum,
-      a.err, a.varlen);
+      a.err, a.varlen, a.alibi, a.log_inv_eps);
   e = cudaGetLastError();
   return e == cudaSuccess ? PLSH_OK : cuda_fail(e, "attn_simt_kernel launch");
 }

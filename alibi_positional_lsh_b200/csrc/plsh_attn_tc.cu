@@ -53,6 +53,12 @@
 // block-diagonal attention, and the passes share one online softmax, so the
 // result is the same T~ (Methodology 3, Theorem 2.2's construction).
 //
+// Exact banded ALiBi (the kAlibi instantiations, the competitor Positional LSH
+// approximates) runs on the same machinery with weights computed from the
+// positions: x = S log2(e)/sqrt(d) - |i - j| log2(e)/sigma_h - m over the keys
+// within W_h = ceil(sigma_h ln(1/eps)) of the tile's rows; the mask warp then
+// only publishes each tile's descriptor.
+//
 // Every barrier wait is bounded in time (PLSH_DEVERR_TIMEOUT); on timeout all
 // roles leave their loops, in-flight copies and MMAs are drained and TMEM is
 // freed before the CTA returns.
@@ -95,8 +101,8 @@ struct alignas(16) MaskStage {
   // dq[q][c] = OR bm[c + 1 .. 32q] for c < 32q, OR bm[32q + 32 .. c] for c >= 32q + 32
   MaskT dq[4][kTile];
   // the tile as the softmax needs it: valid (0 = end of the CTA's work), kind (0 diagonal,
-  // 1 below, 2 above), first / last tile of its item, item index x
-  int valid, kind, first, last, x, pad0, pad1, pad2;
+  // 1 below, 2 above), first / last tile of its item, item index x, first key j0
+  int valid, kind, first, last, x, j0, pad1, pad2;
 };
 
 template <typename MaskT>
@@ -129,14 +135,24 @@ struct Params {
   // [H][T][2] union windows (K3), or [H][s][T][2] per-hash windows for the comparator (K4, the
   // kVarlen instantiations, which walk every item once per hash)
   const int32_t* spans;
+  // exact banded ALiBi (the kAlibi instantiations): per-head length scales and ln(1/eps); the
+  // window of a query tile reaches W_h = ceil(sigma_h ln(1/eps)) keys past its rows
+  const double* sigma;
+  double log_inv_eps;
 };
+
+// Keys past which exp(-|i - j| / sigma) < eps, clamped to [0, n].
+__device__ __forceinline__ int alibi_reach(double sigma, double log_inv_eps, int n) {
+  const double w = ceil(sigma * log_inv_eps);
+  return (w >= static_cast<double>(n) || !(w >= 0.0)) ? n : static_cast<int>(w);
+}
 
 // The key tiles of a CTA's work items, in the order every role walks them:
 // items x0, x0 + stride, ...; within an item the diagonal tile, then the tiles
 // below, then (non-causal) the tiles above. For the per-sample comparator an
 // item is walked once per hash k (a sub-item), each time over that hash's
 // window. The next (sub-)item's window is fetched one ahead.
-template <bool kVarlen>
+template <bool kVarlen, bool kAlibi = false>
 struct TileIter {
   const Params* p;
   const int16_t* order;
@@ -161,6 +177,13 @@ struct TileIter {
     if (xx < p->items) {
       const int hh = head_of(xx);
       const int tt = (xx % (p->B * p->T)) % p->T;
+      if constexpr (kAlibi) {
+        const int reach = alibi_reach(p->sigma[hh], p->log_inv_eps, p->n);
+        const int i0 = tt * kTile, last_row = min(p->n, i0 + kTile) - 1;
+        lo = max(0, i0 - reach);
+        hi = p->causal ? last_row : min(p->n - 1, last_row + reach);
+        return;
+      }
       const size_t at = kVarlen ? ((static_cast<size_t>(hh) * p->s + sb) * p->T + tt) * 2
                                 : (static_cast<size_t>(hh) * p->T + tt) * 2;
       lo = p->spans[at];
@@ -309,6 +332,29 @@ __device__ __forceinline__ float p16_carry(const uint32_t (&sv)[16], const MaskT
   return (ls[0] + ls[1]) + (ls[2] + ls[3]);
 }
 
+// Exact ALiBi: P = 2^(S sc - m - lam |i - j|) for 16 keys, with t0 = lam (i - j) at the first key
+// (i - j falls by one per key) and keys k > lim dropped (the causal mask, and keys past n, which
+// the tensor map reads as zeros). Returns the sum of P.
+__device__ __forceinline__ float p16_alibi(const uint32_t (&sv)[16], float t0, float lam, int lim, float sc,
+                                           float neg_m, uint32_t (&pk)[8]) {
+  float ls[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+  for (int g4 = 0; g4 < 4; ++g4) {
+    float p[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int k = 4 * g4 + e;
+      const float t = fmaf(-lam, static_cast<float>(k), t0);
+      const float x = fmaf(__uint_as_float(sv[k]), sc, neg_m) - fabsf(t);
+      p[e] = k > lim ? 0.0f : ex2_approx(x);
+      ls[e] += p[e];
+    }
+    pk[2 * g4] = pack_bf16x2(p[0], p[1]);
+    pk[2 * g4 + 1] = pack_bf16x2(p[2], p[3]);
+  }
+  return (ls[0] + ls[1]) + (ls[2] + ls[3]);
+}
+
 // The same with the counts given as bytes: the count of key k in byte k % 4 of c4[k / 4].
 __device__ __forceinline__ float p16_counts(const uint32_t (&sv)[16], const uint32_t (&c4)[4], float sc,
                                             float neg_m, uint32_t (&pk)[8]) {
@@ -369,7 +415,7 @@ __device__ __forceinline__ void diag_scan(const MaskStage<MaskT>& ms, int q, int
   hi = R2;
 }
 
-template <typename MaskT, bool kCausal, bool kVarlen>
+template <typename MaskT, bool kCausal, bool kVarlen, bool kAlibi>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ Params prm,
@@ -403,9 +449,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     const int nsub = kVarlen ? s : 1;
     for (int h = threadIdx.x; h < H; h += kThreads) {
       int w = 0;
-      for (int sb = 0; sb < nsub; ++sb) {
-        const size_t at = (static_cast<size_t>(h) * nsub + sb) * prm.T + tm;
-        w += prm.spans[at * 2 + 1] - prm.spans[at * 2];
+      if constexpr (kAlibi) {
+        w = alibi_reach(prm.sigma[h], prm.log_inv_eps, n);
+      } else {
+        for (int sb = 0; sb < nsub; ++sb) {
+          const size_t at = (static_cast<size_t>(h) * nsub + sb) * prm.T + tm;
+          w += prm.spans[at * 2 + 1] - prm.spans[at * 2];
+        }
       }
       sm.width[h] = w;
     }
@@ -460,7 +510,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       tma_prefetch_desc(&tmap_q);
       tma_prefetch_desc(&tmap_k);
       tma_prefetch_desc(&tmap_v);
-      TileIter<kVarlen> ti;
+      TileIter<kVarlen, kAlibi> ti;
       ti.start(&prm, sm.order);
       int issued_g = 0, issued_v = 0, issued_k = 0;  // K tiles, V tiles and Q items issued
       while (ti.valid) {
@@ -512,7 +562,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         k_desc[i] = smem_desc_sw128(smem_u32(sm.k[i]), 16, 1024);
         v_desc[i] = smem_desc_sw128(smem_u32(sm.v[i]), kChunkBytes, 1024);
       }
-      auto issue_s = [&](const TileIter<kVarlen>& ti) -> bool {
+      auto issue_s = [&](const TileIter<kVarlen, kAlibi>& ti) -> bool {
         const int qb = ti.k & 1;
         if (ti.first() && !mbar_wait(&sm.q_full[qb], (ti.k >> 1) & 1, abort_flag, err)) return false;
         const int st = ti.g % kStages;
@@ -531,7 +581,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         if (ti.last()) mma_commit(&sm.q_empty[qb]);
         return true;
       };
-      auto issue_pv = [&](const TileIter<kVarlen>& ti) -> bool {
+      auto issue_pv = [&](const TileIter<kVarlen, kAlibi>& ti) -> bool {
         const int st = ti.g % kStages;
         if (!mbar_wait(&sm.p_full[ti.g & 1], static_cast<uint32_t>(ti.g >> 1) & 1u, abort_flag, err)) return false;
         if (!mbar_wait(&sm.v_full[st], static_cast<uint32_t>(ti.g / kStages) & 1u, abort_flag, err)) return false;
@@ -550,7 +600,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         mma_commit(&sm.v_empty[st]);
         return true;
       };
-      TileIter<kVarlen> cur, nxt;
+      TileIter<kVarlen, kAlibi> cur, nxt;
       cur.start(&prm, sm.order);
       nxt.start(&prm, sm.order);
       bool ok = !cur.valid || issue_s(cur);
@@ -567,12 +617,51 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     }
   } else if (warp == kWarpMask) {
     // ------------------------------------------------------------ mask warp
-    TileIter<kVarlen> ti, nx;
+    if constexpr (kAlibi) {
+      // exact banded ALiBi needs no masks: the warp only publishes each tile's descriptor
+      TileIter<kVarlen, kAlibi> ti;
+      ti.start(&prm, sm.order);
+      int g_end = 0;
+      bool ok = true;
+      while (ti.valid) {
+        const int st = ti.g % kMaskStages;
+        if (ti.g >= kMaskStages) {
+          ok = mbar_wait(&sm.m_empty[st], (static_cast<uint32_t>(ti.g / kMaskStages) & 1u) ^ 1u, abort_flag, err);
+          if (!__all_sync(0xffffffffu, ok)) {
+            ok = false;
+            break;
+          }
+        }
+        if (lane == 0) {
+          MaskStage<MaskT>& ms = sm.m[st];
+          ms.valid = 1;
+          ms.kind = ti.kind();
+          ms.first = ti.first() ? 1 : 0;
+          ms.last = ti.last() ? 1 : 0;
+          ms.x = ti.x;
+          ms.j0 = ti.j0();
+          mbar_arrive(&sm.m_full[st]);
+        }
+        __syncwarp();
+        g_end = ti.g + 1;
+        ti.next();
+      }
+      if (ok && !*abort_flag) {
+        const int st = g_end % kMaskStages;
+        ok = g_end < kMaskStages ||
+             mbar_wait(&sm.m_empty[st], (static_cast<uint32_t>(g_end / kMaskStages) & 1u) ^ 1u, abort_flag, err);
+        if (__all_sync(0xffffffffu, ok) && lane == 0) {
+          sm.m[st].valid = 0;
+          mbar_arrive(&sm.m_full[st]);
+        }
+      }
+    } else {
+    TileIter<kVarlen, kAlibi> ti, nx;
     ti.start(&prm, sm.order);
     nx.start(&prm, sm.order);
     if (nx.valid) nx.next();
     // the masks of a tile; a comparator sub-item keeps only its own hash's bit
-    auto load_masks = [&](const TileIter<kVarlen>& t, MaskT (&v)[4], MaskT& v128) {
+    auto load_masks = [&](const TileIter<kVarlen, kAlibi>& t, MaskT (&v)[4], MaskT& v128) {
       const MaskT* bm_h = bmask + static_cast<size_t>(t.h) * n;
       const MaskT bits = kVarlen ? static_cast<MaskT>(static_cast<MaskT>(1) << t.sub) : FULL;
       const int j0 = t.j0();
@@ -669,6 +758,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         ms.first = ti.first() ? 1 : 0;
         ms.last = ti.last() ? 1 : 0;
         ms.x = ti.x;
+        ms.j0 = ti.j0();
         if (ti.first() && ti.bad_window) atomicOr(err, PLSH_DEVERR_WINDOW);
       }
       __syncwarp();
@@ -690,6 +780,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         mbar_arrive(&sm.m_full[st]);
       }
     }
+    }  // masks (PLSH) or descriptors only (exact ALiBi)
   } else {
     // ------------------------------------------------------------ softmax: quarter warp & 3, key half warp >> 2
     const int quarter = warp & 3;
@@ -702,6 +793,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     const float cs = 8388608.0f + static_cast<float>(sw);  // 2^23 + sw
     float m2 = -INFINITY, l = 0.0f;
     MaskT Y = 0, Z = 0;
+    float lam = 0.0f;  // exact ALiBi: log2(e) / sigma of the item's head
+    int a_i0 = 0;      // exact ALiBi: the item's first row
     int items = 0;  // items finished by this warp
     for (int g = 0;; ++g) {
       const int st = g % kMaskStages;
@@ -714,10 +807,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       if (first) {
         m2 = -INFINITY;
         l = 0.0f;
+        if constexpr (kAlibi) {
+          const int BT = prm.B * prm.T;
+          const int hh = (H <= kMaxSortedHeads) ? static_cast<int>(sm.order[tx / BT]) : tx / BT;
+          lam = static_cast<float>(1.4426950408889634 / prm.sigma[hh]);
+          a_i0 = ((tx % BT) % prm.T) * kTile;
+        }
       }
       // weights that need only the masks: the diagonal's own block and its carries
       MaskT lo = 0, hi = 0;
-      if (kind == 0) diag_scan<MaskT, kCausal>(ms, quarter, r, sw, &sm.cw[0][threadIdx.x], kSoftmaxWarps * 32, lo, hi);
+      if (!kAlibi && kind == 0) diag_scan<MaskT, kCausal>(ms, quarter, r, sw, &sm.cw[0][threadIdx.x], kSoftmaxWarps * 32, lo, hi);
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[g & 1], static_cast<uint32_t>(g >> 1) & 1u, abort_flag, err)))
         break;
       tc_fence_after();
@@ -792,7 +891,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
           tmem_ld16(s_base + 16u * ch, sv);
           tmem_wait_ld();
           regs_after_wait(sv);
-          if (kind == 0 && (ch >> 1) == quarter) {
+          if constexpr (kAlibi) {
+            // i - j for the chunk's first key; keys past the row (when causal) and past n are dropped
+            const int jc = ms.j0 + 16 * ch;
+            const int d0 = a_i0 + r - jc;
+            lsum += p16_alibi(sv, lam * static_cast<float>(d0), lam, min(kCausal ? d0 : 16, n - 1 - jc), sc, neg_m, pk);
+          } else if (kind == 0 && (ch >> 1) == quarter) {
             // the warp's own block on the diagonal: counts from the scan
             uint32_t c4[4];
 #pragma unroll
@@ -808,7 +912,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         }
         tmem_st8(s_base + 64u * hf + 8u * c, pk);
       }
-      if (kind == 1) {
+      if (kAlibi) {
+      } else if (kind == 1) {
         Y = static_cast<MaskT>(Y | ms.bm[0] | ms.suf[0]);  // OR over [j0, i]
       } else if (kind == 2) {
         Z = static_cast<MaskT>(Zc | ms.pre[kTile - 1]);    // OR over (i, j0 + 127]
@@ -885,7 +990,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         const int i = i0 + r;
         if (hf == 0 && i < n)
           row_sum[(static_cast<size_t>(bb) * H + hh) * n + i] =
-              (log2f(ltot) + m2) * 0.6931471805599453f - logf(static_cast<float>(s));
+              (log2f(ltot) + m2) * 0.6931471805599453f - (kAlibi ? 0.0f : logf(static_cast<float>(s)));
         ++items;
       }
     }
@@ -940,7 +1045,7 @@ int sm_count() {
   return count;
 }
 
-template <typename MaskT, bool kCausal, bool kVarlen>
+template <typename MaskT, bool kCausal, bool kVarlen, bool kAlibi>
 int launch_tc_typed(const AttnArgs& a, cudaStream_t st) {
   CUtensorMap mq, mk, mv;
   if (int rc = make_map(&mq, a.Q, a.n, a.B * a.H)) return rc;
@@ -956,7 +1061,9 @@ int launch_tc_typed(const AttnArgs& a, cudaStream_t st) {
   prm.T = ceil_div(a.n, kTile);
   prm.items = a.B * a.H * prm.T;
   prm.spans = a.spans;
-  auto kern = attn_tc_kernel<MaskT, kCausal, kVarlen>;
+  prm.sigma = a.sigma;
+  prm.log_inv_eps = a.log_inv_eps;
+  auto kern = attn_tc_kernel<MaskT, kCausal, kVarlen, kAlibi>;
   const size_t smem = sizeof(TcSmem<MaskT>) + 1024;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_tc_kernel)");
@@ -972,18 +1079,21 @@ int launch_tc_typed(const AttnArgs& a, cudaStream_t st) {
 int launch_attention_tc(const AttnArgs& a, cudaStream_t st) {
   if (static_cast<long long>(a.B) * a.H * ceil_div(a.n, kTile) > 0x7fffffffLL)
     return fail(PLSH_ERR_RANGE, "plsh_attention_fwd: too many query tiles");
+  if (a.alibi)
+    return a.causal ? launch_tc_typed<uint32_t, true, false, true>(a, st)
+                    : launch_tc_typed<uint32_t, false, false, true>(a, st);
   if (a.varlen) {
     if (a.causal)
-      return a.s <= 32 ? launch_tc_typed<uint32_t, true, true>(a, st)
-                       : launch_tc_typed<unsigned long long, true, true>(a, st);
-    return a.s <= 32 ? launch_tc_typed<uint32_t, false, true>(a, st)
-                     : launch_tc_typed<unsigned long long, false, true>(a, st);
+      return a.s <= 32 ? launch_tc_typed<uint32_t, true, true, false>(a, st)
+                       : launch_tc_typed<unsigned long long, true, true, false>(a, st);
+    return a.s <= 32 ? launch_tc_typed<uint32_t, false, true, false>(a, st)
+                     : launch_tc_typed<unsigned long long, false, true, false>(a, st);
   }
   if (a.causal)
-    return a.s <= 32 ? launch_tc_typed<uint32_t, true, false>(a, st)
-                     : launch_tc_typed<unsigned long long, true, false>(a, st);
-  return a.s <= 32 ? launch_tc_typed<uint32_t, false, false>(a, st)
-                   : launch_tc_typed<unsigned long long, false, false>(a, st);
+    return a.s <= 32 ? launch_tc_typed<uint32_t, true, false, false>(a, st)
+                     : launch_tc_typed<unsigned long long, true, false, false>(a, st);
+  return a.s <= 32 ? launch_tc_typed<uint32_t, false, false, false>(a, st)
+                   : launch_tc_typed<unsigned long long, false, false, false>(a, st);
 }
 
 }  // namespace plsh

@@ -32,6 +32,10 @@ struct AttnArgs {
   // 0: K3 (spans = [H][T][2] union windows, weights c_ij). 1: K4, the per-sample comparator
   // (spans = [H][s][T][2] per-hash windows; each sample's block indicator, summed over samples).
   int varlen;
+  // 1: exact banded ALiBi instead of Positional LSH (spans, bmask, table unused): weights
+  // exp(-|i - j| / sigma_h) over |i - j| <= ceil(sigma_h ln(1/eps)), with log_inv_eps = ln(1/eps)
+  int alibi;
+  double log_inv_eps;
 };
 int launch_varlen_spans(const int32_t* ids, int H, int s, int n, int causal, int32_t* spans, cudaStream_t st);
 int launch_attention_simt(const AttnArgs& a, cudaStream_t st);

@@ -129,6 +129,18 @@ class ClockSampler:
                 "samples": len(self.samples), "source": "nvml, every 2 ms during the timed region"}
 
 
+def alibi_spans(sigma, eps: float, n: int, causal: bool) -> np.ndarray:
+    """[H][T][2] key windows of exact banded ALiBi (the kernel's own rule)."""
+    T = (n + TILE - 1) // TILE
+    out = np.empty((len(sigma), T, 2), dtype=np.int64)
+    for h, sg in enumerate(sigma):
+        reach = min(n, int(np.ceil(sg * np.log(1.0 / eps))))
+        for t in range(T):
+            i0, last = t * TILE, min(n, (t + 1) * TILE) - 1
+            out[h, t] = (max(0, i0 - reach), last if causal else min(n - 1, last + reach))
+    return out
+
+
 def issued_tiles(spans: np.ndarray, causal: bool) -> int:
     """Key tiles of 128 the fused kernel's window covers, summed over heads and query tiles:
     ceil((hi - lo + 1) / 128) per query tile (the span rounded to the MMA N granularity)."""
@@ -260,15 +272,19 @@ def run_ours(args, rank, world, local):
     stream = torch.cuda.current_stream()
 
     varlen = args.path == "varlen"
+    alibi = args.path == "alibi"
 
     def attend():
         if varlen:
             plan.attend_varlen(q, k, v, stream)
+        elif alibi:
+            plan.attend_alibi(q, k, v, args.eps, stream)
         else:
             plan.attend(q, k, v, stream)
 
     def step(ev=None):
-        plan.prepare(stream)
+        if not alibi:       # exact banded ALiBi needs no table, ids or masks
+            plan.prepare(stream)
         if ev is not None:
             ev[0].record(stream)
         attend()
@@ -284,6 +300,8 @@ def run_ours(args, rank, world, local):
     if varlen:   # per-hash windows [H][s][T][2]: every hash's window is visited
         T = (w.n + TILE - 1) // TILE
         spans = plan.scratch.cpu().numpy()[: w.H * w.s * T * 2].reshape(w.H * w.s, T, 2)
+    elif alibi:  # bands |i - j| <= ceil(sigma_h ln(1/eps)) around each query tile
+        spans = alibi_spans(w.sigmas(), args.eps, w.n, w.causal)
     else:
         spans = plan.spans.cpu().numpy()
     tiles_min = issued_tiles(spans, w.causal)
@@ -319,8 +337,20 @@ def run_ours(args, rank, world, local):
     oh = torch.empty_like(plan.O, device="cpu").pin_memory()
     rh = torch.empty_like(plan.row_sum, device="cpu").pin_memory()
     qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def run_host(qh_, kh_, vh_, qd_, kd_, vd_, oh_, rh_):
+        if alibi:   # no table or masks: copy in, attend, copy out
+            with torch.cuda.stream(stream):
+                qd_.copy_(qh_, non_blocking=True)
+                kd_.copy_(kh_, non_blocking=True)
+                vd_.copy_(vh_, non_blocking=True)
+                plan.attend_alibi(qd_, kd_, vd_, args.eps, stream)
+                oh_.copy_(plan.O, non_blocking=True)
+                rh_.copy_(plan.row_sum, non_blocking=True)
+        else:
+            plan.run_host(qh_, kh_, vh_, qd_, kd_, vd_, oh_, rh_, stream, varlen=varlen)
     for _ in range(3):
-        plan.run_host(qh, kh, vh, qd, kd, vd, oh, rh, stream, varlen=varlen)
+        run_host(qh, kh, vh, qd, kd, vd, oh, rh)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     Ke = max(3, min(K, 20))
@@ -328,7 +358,7 @@ def run_ours(args, rank, world, local):
     torch.cuda.synchronize()
     e0.record(stream)
     for _ in range(Ke):
-        plan.run_host(qh, kh, vh, qd, kd, vd, oh, rh, stream, varlen=varlen)
+        run_host(qh, kh, vh, qd, kd, vd, oh, rh)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
@@ -337,29 +367,33 @@ def run_ours(args, rank, world, local):
     d2h = oh.numel() * oh.element_size() + rh.numel() * 4
 
     # the other attention path on the same plan and inputs, for comparison (not part of the step)
-    other = None
+    # the other attention paths on the same plan and inputs, for comparison (not part of the step)
+    others = []
     if world == 1:
-        def other_attend():
-            if varlen:
-                plan.attend(q, k, v, stream)
-            else:
-                plan.attend_varlen(q, k, v, stream)
-        for _ in range(2):
-            other_attend()
-        ts = []
-        for _ in range(5):
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            other_attend()
-            b.record(stream)
-            torch.cuda.synchronize()
-            ts.append(a.elapsed_time(b))
-        errs = plan.device_errors()
-        if errs:
-            raise RuntimeError(f"device errors in the comparison path: {errs}")
-        other = {"path": "fused (plsh_attention_fwd)" if varlen else "per-sample comparator (plsh_attention_varlen_fwd)",
-                 "attention_ms": float(np.median(ts)),
-                 "this_path_speedup": float(np.median(ts)) / attn_avg}
+        paths = {"fused": ("fused (plsh_attention_fwd)", lambda: plan.attend(q, k, v, stream)),
+                 "varlen": ("per-sample comparator (plsh_attention_varlen_fwd)",
+                            lambda: plan.attend_varlen(q, k, v, stream)),
+                 "alibi": (f"exact banded ALiBi, eps={args.eps:g} (plsh_alibi_banded_fwd)",
+                           lambda: plan.attend_alibi(q, k, v, args.eps, stream))}
+        plan.prepare(stream)
+        for key, (label, run) in paths.items():
+            if key == args.path:
+                continue
+            for _ in range(2):
+                run()
+            ts = []
+            for _ in range(5):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                run()
+                b.record(stream)
+                torch.cuda.synchronize()
+                ts.append(a.elapsed_time(b))
+            errs = plan.device_errors()
+            if errs:
+                raise RuntimeError(f"device errors in the comparison path {key}: {errs}")
+            others.append({"path": label, "attention_ms": float(np.median(ts)),
+                           "this_path_speedup": float(np.median(ts)) / attn_avg})
 
     tokens = w.B * w.n * world
     value = job_value(w.B * w.n, world, ms_step)
@@ -393,7 +427,9 @@ def run_ours(args, rank, world, local):
 
     line = {
         "metric": "PLSH-ALiBi fwd query-tokens/s at n=32k, s=20; achieved % of roofline",
-        "path": "per-sample comparator (plsh_attention_varlen_fwd)" if varlen else "fused (plsh_attention_fwd)",
+        "path": ("per-sample comparator (plsh_attention_varlen_fwd)" if varlen else
+                 f"exact banded ALiBi, eps={args.eps:g} (plsh_alibi_banded_fwd)" if alibi else
+                 "fused (plsh_attention_fwd)"),
         "value": value,
         "unit": "query-tokens/s",
         "n_gpus": world,
@@ -409,16 +445,18 @@ def run_ours(args, rank, world, local):
         "roofline": roof,
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "query-tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "path": "PlshForward.run_host: pinned host Q/K/V -> device -> table, K1, K2, "
-                        + ("K4" if varlen else "K3") + " -> host O, row_sum"},
-        "gpu_launches": (5 if varlen else 4) * K,
-        "gpu_launches_per_step": dict({"sample_bins_kernel": 1, "mask_bmax_kernel": 1, "spans_kernel": 1,
-                                       roof["kernel"]: 1}, **({"varlen_spans_kernel": 1} if varlen else {})),
+                "path": ("pinned host Q/K/V -> device -> exact banded ALiBi -> host O, row_sum" if alibi else
+                         "PlshForward.run_host: pinned host Q/K/V -> device -> table, K1, K2, "
+                         + ("K4" if varlen else "K3") + " -> host O, row_sum")},
+        "gpu_launches": (1 if alibi else 5 if varlen else 4) * K,
+        "gpu_launches_per_step": ({roof["kernel"]: 1} if alibi else
+                                  dict({"sample_bins_kernel": 1, "mask_bmax_kernel": 1, "spans_kernel": 1,
+                                        roof["kernel"]: 1}, **({"varlen_spans_kernel": 1} if varlen else {}))),
         "step_breakdown_ms": {"attention": attn_avg, "table+bins+window": ms_step - attn_avg},
         "clocks": clocks,
     }
-    if other is not None:
-        line["comparison"] = other
+    if others:
+        line["comparison"] = others
     if rank == 0 and not args.no_cpu_baseline:
         sampler = OracleSampler(w)
         rate, desc = sampler.run(args.cpu_seconds)
@@ -474,8 +512,11 @@ def main(argv=None):
     ap.add_argument("--workload", default=workloads.HEADLINE, choices=list(workloads.WORKLOADS))
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--path", choices=["fused", "varlen"], default="fused",
-                    help="attention path timed: the fused kernel (K3) or the per-sample comparator (K4)")
+    ap.add_argument("--path", choices=["fused", "varlen", "alibi"], default="fused",
+                    help="attention path timed: the fused kernel (K3), the per-sample comparator (K4) or "
+                         "exact banded ALiBi")
+    ap.add_argument("--eps", type=float, default=1e-4,
+                    help="band cut-off of exact banded ALiBi (keys lighter than eps are left out)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller cases for profiling)")
     args = ap.parse_args(argv)

@@ -252,6 +252,26 @@ PLSH_API int plsh_attention_varlen_fwd_static(const void* Q, const void* K, cons
                                               const void* bmask_dev, int causal, void* O, float* row_sum,
                                               uint32_t* err_dev, void* stream);
 
+/*
+ * plsh_alibi_banded_fwd -- exact ALiBi attention, the computation Positional
+ * LSH approximates (technical summary, Methodology 1: L*_ij = e^{-|i-j|/sigma}
+ * as the ALiBi bias matrix; Results: the approximation error ||T* - T~||),
+ * restricted to a band: per query head h with KV head h / (H/H_kv),
+ *   O_i       = sum_j w_ij e^{S_ij} V_j / sum_j w_ij e^{S_ij},  S = Q K^T / sqrt d,
+ *   row_sum_i = ln( sum_j w_ij e^{S_ij} ),   w_ij = e^{-|i-j| / sigma_h},
+ * over every key in the 128-key tiles that cover |i - j| <= ceil(sigma_h ln(1/eps))
+ * (and j <= i when causal). Keys outside that band weigh less than eps each
+ * relative to the diagonal and are left out. No table, ids or masks are used.
+ *
+ *   Arguments as plsh_attention_fwd, plus
+ *   sigma_dev  [H] doubles, the ALiBi length scales (1 / slope); required.
+ *   eps        the band's cut-off, 0 < eps < 1.
+ * Every pointer must be 16-byte aligned.
+ */
+PLSH_API int plsh_alibi_banded_fwd(const void* Q, const void* K, const void* V, int dtype, int B, int H, int H_kv,
+                                   int n, int d, const double* sigma_dev, double eps, int causal, void* O,
+                                   float* row_sum, uint32_t* err_dev, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

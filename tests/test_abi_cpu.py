@@ -102,3 +102,35 @@ def test_entry_points_reject_bad_sizes_before_any_launch(plsh):
     rc = lib.plsh_attention_fwd(fake, fake, fake, 7, 1, 1, 1, 128, 128, null, 4, null, fake, fake, 0, fake, fake,
                                 fake, null)
     assert rc == 2
+
+
+def test_banded_alibi_rejects_bad_arguments_before_any_launch(plsh):
+    lib = plsh._lib
+    null = None
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the checks fail first
+    args = lambda eps, sigma=fake, d=128, causal=1: (fake, fake, fake, 0, 1, 2, 1, 256, d, sigma,
+                                                     ctypes.c_double(eps), causal, fake, fake, fake, null)
+    assert lib.plsh_alibi_banded_fwd(*args(0.0)) == 1 and "eps" in plsh.plsh_last_error()
+    assert lib.plsh_alibi_banded_fwd(*args(1.0)) == 1
+    assert lib.plsh_alibi_banded_fwd(*args(float("nan"))) == 1
+    assert lib.plsh_alibi_banded_fwd(*args(1e-4, sigma=null)) == 1 and "null" in plsh.plsh_last_error()
+    assert lib.plsh_alibi_banded_fwd(*args(1e-4, d=96)) == 2
+    assert lib.plsh_alibi_banded_fwd(*args(1e-4, causal=3)) == 1
+
+
+def test_varlen_entry_points_reject_bad_arguments_before_any_launch(plsh):
+    lib = plsh._lib
+    null = None
+    fake = ctypes.c_void_p(1 << 20)
+    assert lib.plsh_varlen_scratch_bytes(16, 20, 32768) == 8 * 16 * 20 * 256
+    assert lib.plsh_varlen_scratch_bytes(0, 20, 32768) == 0
+    assert lib.plsh_varlen_spans(null, 1, 4, 100, 0, fake, null) == 1
+    assert lib.plsh_varlen_spans(fake, 1, 4, 100, 2, fake, null) == 1
+    # scratch smaller than needed
+    rc = lib.plsh_attention_varlen_fwd(fake, fake, fake, 0, 1, 1, 1, 300, 128, null, 5, null, fake, fake, 1, fake,
+                                       ctypes.c_size_t(8), fake, fake, fake, null)
+    assert rc == 1 and "scratch" in plsh.plsh_last_error()
+    # the static-buffer entry point refuses windows larger than its buffer
+    rc = lib.plsh_attention_varlen_fwd_static(fake, fake, fake, 0, 1, 40, 8, 131072, 128, null, 64, null, fake,
+                                              fake, 1, fake, fake, fake, null)
+    assert rc == 3 and "static buffer" in plsh.plsh_last_error()

@@ -173,3 +173,31 @@ def test_mistral_s_sweep_sampled_rows():
         O, R = PH.oracle_rows(q, k, v, gpu["table"], True, rows)
         to, tr = PH.tolerance(base.torch_dtype, v)
         PH.assert_close(gpu["O"][:, :, rows], gpu["row_sum"][:, :, rows], O, R, to, tr, f"s={s}")
+
+
+# ---------------------------------------------------------------- the fixed-blocks baseline
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fixed_blocks_baseline(causal):
+    """A deterministic table (s = 1, pitch = block, offset 0) through the same kernels: each row
+    attends inside its own block of `block` positions (the fixed-blocks comparison)."""
+    from alibi_positional_lsh_b200 import fixed_blocks_table
+    B, H, H_kv, n, d, block = 1, 2, 1, 1000, 128, 96
+    q, k, v = _inputs(B, H, H_kv, n, d, torch.bfloat16, 77)
+    table = fixed_blocks_table(H, block)
+    gpu = PH.run_gpu(B, H, H_kv, n, d, 1, causal, [float(block)] * H, 0, q, k, v, table=table)
+    assert gpu["errors"] == []
+    ids = oracle.bin_ids(table, n)
+    assert np.array_equal(ids[0, 0], np.arange(n) // block)
+    PH.oracle_window_checks(table, n, causal, gpu)
+    O, R = PH.oracle_rows(q, k, v, table, causal, None)
+    to, tr = PH.tolerance(torch.bfloat16, v)
+    PH.assert_close(gpu["O"], gpu["row_sum"], O, R, to, tr, "fixed blocks")
+    # per-block softmax, written out directly
+    Qf, Kf, Vf = PH.f64(q)[0, 0], PH.f64(k)[0, 0], PH.f64(v)[0, 0]
+    for i in (0, block - 1, block, n - 1):
+        lo = (i // block) * block
+        hi = i if causal else min(n, lo + block) - 1
+        sc = Qf[i] @ Kf[lo:hi + 1].T / math.sqrt(d)
+        w = np.exp(sc - sc.max())
+        assert np.abs(gpu["O"][0, 0, i] - (w @ Vf[lo:hi + 1]) / w.sum()).max() <= to
