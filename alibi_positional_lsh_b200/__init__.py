@@ -25,7 +25,7 @@ PLSH_F32 = 1
 PLSH_TILE = 128
 PLSH_MAX_S = 64
 PLSH_VARLEN_STATIC_SCRATCH_BYTES = 4 << 20
-DEVERR_BITS = {1: "RANGE", 2: "TABLE", 4: "WINDOW", 8: "TIMEOUT", 16: "SIGMA"}
+DEVERR_BITS = {1: "RANGE", 2: "TABLE", 4: "WINDOW", 8: "TIMEOUT", 16: "SIGMA", 32: "POSITION"}
 
 
 class PlshError(RuntimeError):
@@ -66,6 +66,8 @@ def _load() -> ctypes.CDLL:
     lib.plsh_attention_varlen_fwd_static.restype = i32
     lib.plsh_attention_varlen_fwd_static.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, i32, vp, vp,
                                                      vp, i32, vp, vp, vp, vp]
+    lib.plsh_decode_fwd.restype = i32
+    lib.plsh_decode_fwd.argtypes = [vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, i32, vp, vp, vp, vp]
     return lib
 
 
@@ -173,6 +175,14 @@ def plsh_alibi_banded_fwd(Q, K, V, dtype: int, B: int, H: int, H_kv: int, n: int
                                       _dev_ptr(sigma_dev, "sigma_dev"), ctypes.c_double(eps), int(causal),
                                       _dev_ptr(O, "O"), _dev_ptr(row_sum, "row_sum"), _dev_ptr(err_dev, "err_dev"),
                                       _stream_ptr(stream)))
+
+
+def plsh_decode_fwd(Q, pos_dev, m: int, K, V, dtype: int, B: int, H: int, H_kv: int, n: int, d: int, s: int,
+                    bmask_dev, causal: int, O, row_sum, err_dev, stream=None) -> None:
+    _check(_lib.plsh_decode_fwd(_dev_ptr(Q, "Q"), _dev_ptr(pos_dev, "pos_dev"), m, _dev_ptr(K, "K"),
+                                _dev_ptr(V, "V"), dtype, B, H, H_kv, n, d, s, _dev_ptr(bmask_dev, "bmask_dev"),
+                                int(causal), _dev_ptr(O, "O"), _dev_ptr(row_sum, "row_sum"),
+                                _dev_ptr(err_dev, "err_dev"), _stream_ptr(stream)))
 
 
 def decode_device_error(word: int) -> list:

@@ -7,6 +7,7 @@ with torch) and runs the whole path:
   a3 plsh_window       (K2)     -> b_max, tile windows, boundary masks
   a4 plsh_attention_fwd (K3)    -> O, row_sum
   a5 plsh_attention_varlen_fwd (K4, the per-sample comparator) -> the same O, row_sum
+  plsh_decode_fwd (single query rows against the cached K, V) -> rows of T~, row_sum
   plsh_alibi_banded_fwd (exact banded ALiBi, what the method approximates) -> T*, row_sum
 All arithmetic of a2..a5 runs in libplsh's CUDA kernels.
 """
@@ -18,7 +19,7 @@ import numpy as np
 import torch
 
 from . import (PLSH_BF16, PLSH_F32, PLSH_TILE, PlshError, decode_device_error, plsh_alibi_banded_fwd,
-               plsh_attention_fwd, plsh_attention_varlen_fwd, plsh_draw_table, plsh_sample_bins,
+               plsh_attention_fwd, plsh_attention_varlen_fwd, plsh_decode_fwd, plsh_draw_table, plsh_sample_bins,
                plsh_varlen_scratch_bytes, plsh_window)
 
 
@@ -121,6 +122,26 @@ class PlshForward:
         plsh_alibi_banded_fwd(q, k, v, self.dtype_code, B, H, H_kv, n, d, self.sigma_dev, float(eps),
                               int(self.causal), self.O, self.row_sum, self.err, st)
         return self.O, self.row_sum
+
+    def decode(self, q_rows: torch.Tensor, pos: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+               stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+        """Rows pos (int32 [m] on the device) of T~ for query rows q_rows [B,H,m,d] against the cache k, v
+        [B,H_kv,n,d], with the masks of the last prepare(). Returns new tensors O [B,H,m,d], row_sum [B,H,m]."""
+        B, H, H_kv, n, d = self.B, self.H, self.H_kv, self.n, self.d
+        m = int(pos.shape[0]) if pos.dim() == 1 else -1
+        if m < 1 or pos.dtype != torch.int32 or pos.device != self.O.device:
+            raise ValueError(f"pos must be a non-empty int32 vector on {self.O.device}")
+        if q_rows.shape != (B, H, m, d) or k.shape != (B, H_kv, n, d) or v.shape != (B, H_kv, n, d):
+            raise ValueError("q_rows/k/v shapes do not match the plan")
+        for t, nm in ((q_rows, "q_rows"), (k, "k"), (v, "v")):
+            if t.dtype != self.dtype or t.device != self.O.device:
+                raise ValueError(f"{nm} must be {self.dtype} on {self.O.device}")
+        O = torch.empty((B, H, m, d), dtype=self.dtype, device=self.O.device)
+        R = torch.empty((B, H, m), dtype=torch.float32, device=self.O.device)
+        st = torch.cuda.current_stream() if stream is None else stream
+        plsh_decode_fwd(q_rows, pos, m, k, v, self.dtype_code, B, H, H_kv, n, d, self.s, self.bmask,
+                        int(self.causal), O, R, self.err, st)
+        return O, R
 
     def __call__(self, q, k, v, stream=None, table=None):
         self.prepare(stream, table)

@@ -28,6 +28,7 @@ SOURCES = [
     "plsh_attn_simt.cu",
     "plsh_attn_tc.cu",
     "plsh_varlen.cu",
+    "plsh_decode.cu",
 ]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -238,3 +238,18 @@ extern "C" int plsh_alibi_banded_fwd(const void* Q, const void* K, const void* V
                    nullptr, nullptr, O, row_sum, err_dev, 0, 1, -std::log(eps)};
   return plsh::launch_attention(a, static_cast<cudaStream_t>(stream));
 }
+
+// ---------------------------------------------------------------- decode
+
+extern "C" int plsh_decode_fwd(const void* Q, const int32_t* pos_dev, int m, const void* K, const void* V, int dtype,
+                               int B, int H, int H_kv, int n, int d, int s, const void* bmask_dev, int causal,
+                               void* O, float* row_sum, uint32_t* err_dev, void* stream) {
+  const char* fn = "plsh_decode_fwd";
+  if (int rc = plsh::check_attention(fn, Q, K, V, dtype, B, H, H_kv, n, d, s, causal, bmask_dev, O, row_sum,
+                                     err_dev))
+    return rc;
+  if (m < 1) return fail(PLSH_ERR_INVALID_ARG, "%s: need m >= 1 (m=%d)", fn, m);
+  if (!pos_dev) return fail(PLSH_ERR_INVALID_ARG, "%s: null pointer", fn);
+  plsh::DecodeArgs a{Q, pos_dev, m, K, V, dtype, B, H, H_kv, n, d, s, causal, bmask_dev, O, row_sum, err_dev};
+  return plsh::launch_decode(a, static_cast<cudaStream_t>(stream));
+}

@@ -37,6 +37,15 @@ struct AttnArgs {
   int alibi;
   double log_inv_eps;
 };
+// Decode: query rows Q [B][H][m][d] at positions pos [m] against K, V [B][H_kv][n][d].
+struct DecodeArgs {
+  const void* Q; const int32_t* pos; int m;
+  const void* K; const void* V;
+  int dtype, B, H, H_kv, n, d, s, causal;
+  const void* bmask;
+  void* O; float* row_sum; uint32_t* err;
+};
+int launch_decode(const DecodeArgs& a, cudaStream_t st);
 int launch_varlen_spans(const int32_t* ids, int H, int s, int n, int causal, int32_t* spans, cudaStream_t st);
 int launch_attention_simt(const AttnArgs& a, cudaStream_t st);
 int launch_attention_tc(const AttnArgs& a, cudaStream_t st);

@@ -257,6 +257,52 @@ class OracleSampler:
 
 # ---------------------------------------------------------------- our arm
 
+def decode_keys(bmask: np.ndarray, s: int, i: int, causal: bool) -> int:
+    """Keys with a nonzero count c_ij for the query at position i, summed over heads: the rows of K
+    and V plsh_decode_fwd reads. c_ij = s - popcount(OR of the masks over (min, max])."""
+    H, n = bmask.shape
+    full = (1 << s) - 1
+    total = 0
+    for h in range(H):
+        bm = bmask[h].astype(np.uint64)
+        below = np.bitwise_or.accumulate(bm[i:0:-1]) if i > 0 else np.zeros(0, np.uint64)   # keys i-1 .. 0
+        total += 1 + int(np.count_nonzero(below != full))
+        if not causal and i + 1 < n:
+            above = np.bitwise_or.accumulate(bm[i + 1:])                                        # keys i+1 .. n-1
+            total += int(np.count_nonzero(above != full))
+    return total
+
+
+def decode_timing(plan, q, k, v, stream, w):
+    """plsh_decode_fwd on the newest position (one query row per (b, h) at i = n-1) against the whole
+    cache: device time per call and the K/V bytes it must read (the weighted keys' rows)."""
+    i = w.n - 1
+    pos = torch.tensor([i], dtype=torch.int32, device=q.device)
+    q1 = q[:, :, i:i + 1].contiguous()
+    for _ in range(3):
+        plan.decode(q1, pos, k, v, stream)
+    ts = []
+    for _ in range(20):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        plan.decode(q1, pos, k, v, stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    errs = plan.device_errors()
+    if errs:
+        raise RuntimeError(f"device errors in decode: {errs}")
+    bm = plan.bmask.cpu().numpy()
+    bm = bm.view(np.uint32) if w.s <= 32 else bm.view(np.uint64)
+    keys = decode_keys(bm, w.s, i, w.causal) * w.B
+    elt = 2 if w.dtype == "bf16" else 4
+    kv_bytes = keys * 2 * w.d * elt
+    us = float(np.median(ts)) * 1e3
+    return {"path": "decode (plsh_decode_fwd), one query row per (b, h) at position n-1, whole cache",
+            "kernel": "decode_kernel", "us_per_call": us, "weighted_keys": keys, "kv_bytes": kv_bytes,
+            "achieved_GBps": kv_bytes / (us * 1e-6) / 1e9}
+
+
 def run_ours(args, rank, world, local):
     from alibi_positional_lsh_b200 import PlshForward
     import alibi_positional_lsh_b200 as plsh_mod  # noqa: F401
@@ -366,7 +412,6 @@ def run_ours(args, rank, world, local):
     h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh)) + plan.table_host.numel() * 8
     d2h = oh.numel() * oh.element_size() + rh.numel() * 4
 
-    # the other attention path on the same plan and inputs, for comparison (not part of the step)
     # the other attention paths on the same plan and inputs, for comparison (not part of the step)
     others = []
     if world == 1:
@@ -394,6 +439,8 @@ def run_ours(args, rank, world, local):
                 raise RuntimeError(f"device errors in the comparison path {key}: {errs}")
             others.append({"path": label, "attention_ms": float(np.median(ts)),
                            "this_path_speedup": float(np.median(ts)) / attn_avg})
+
+    decode = decode_timing(plan, q, k, v, stream, w) if (world == 1 and not alibi) else None
 
     tokens = w.B * w.n * world
     value = job_value(w.B * w.n, world, ms_step)
@@ -457,6 +504,8 @@ def run_ours(args, rank, world, local):
     }
     if others:
         line["comparison"] = others
+    if decode:
+        line["decode"] = decode
     if rank == 0 and not args.no_cpu_baseline:
         sampler = OracleSampler(w)
         rate, desc = sampler.run(args.cpu_seconds)

@@ -63,6 +63,7 @@ extern "C" {
 #define PLSH_DEVERR_WINDOW   4u  /* a tile window outside [0, n) or not covering the tile's own rows */
 #define PLSH_DEVERR_TIMEOUT  8u  /* a bounded wait on a barrier gave up (the kernel returned early) */
 #define PLSH_DEVERR_SIGMA   16u  /* a per-head sigma not finite and > 0 */
+#define PLSH_DEVERR_POSITION 32u /* a decode query position outside [0, n) */
 
 #define PLSH_TILE   128   /* query/key tile height of the windows */
 #define PLSH_MAX_S  64    /* most hashes per head (one bit each in a 64-bit boundary mask) */
@@ -271,6 +272,39 @@ PLSH_API int plsh_attention_varlen_fwd_static(const void* Q, const void* K, cons
 PLSH_API int plsh_alibi_banded_fwd(const void* Q, const void* K, const void* V, int dtype, int B, int H, int H_kv,
                                    int n, int d, const double* sigma_dev, double eps, int causal, void* O,
                                    float* row_sum, uint32_t* err_dev, void* stream);
+
+/*
+ * plsh_decode_fwd -- single query rows against cached keys and values: row i
+ * of the same T~ as plsh_attention_fwd, for a handful of rows at a time
+ * (autoregressive decoding, where the new token at position i attends to
+ * the cached keys 0..i).
+ *
+ * Cites: Methodology 2 (M~ = (1/s) sum_k M(h_k)), Methodology 3 (attention
+ * restricted to short random blocks) and Methodology 1, structure (blocks
+ * are contiguous, so c_ij only falls as j moves away from i and the key walk
+ * can stop at the first stretch where it is 0 for every key). For query row
+ * t of (b, h) at position i = pos[t], with KV head h / (H/H_kv):
+ *   O[b][h][t]       = sum_j c_ij e^{S_ij} V_j / sum_j c_ij e^{S_ij},
+ *   row_sum[b][h][t] = ln( sum_j (c_ij / s) e^{S_ij} ),
+ *   S_ij = Q[b][h][t] . K[b][h_kv][j] / sqrt d,
+ * c_ij = s - popcount(OR of bmask over (min(i,j), max(i,j)]), over j <= i
+ * when causal, every j in [0, n) otherwise.
+ *
+ *   Q          [B][H][m][d] query rows; O like Q (out).
+ *   pos_dev    [m] int32 device positions, each in [0, n); a position
+ *              outside sets PLSH_DEVERR_POSITION and leaves that row's
+ *              O and row_sum unwritten. Positions may repeat.
+ *   m          rows per (b, h), >= 1.
+ *   K, V       [B][H_kv][n][d] the cache, n positions.
+ *   dtype, d, s, causal, bmask_dev, err_dev   as plsh_attention_fwd; the
+ *              masks are plsh_window's for this n (with causal, only the
+ *              entries at positions <= max(pos) are read).
+ *   row_sum    [B][H][m] float32 out.
+ * Q, K, V and O must be 16-byte aligned.
+ */
+PLSH_API int plsh_decode_fwd(const void* Q, const int32_t* pos_dev, int m, const void* K, const void* V, int dtype,
+                             int B, int H, int H_kv, int n, int d, int s, const void* bmask_dev, int causal,
+                             void* O, float* row_sum, uint32_t* err_dev, void* stream);
 
 #ifdef __cplusplus
 }

@@ -134,3 +134,16 @@ def test_varlen_entry_points_reject_bad_arguments_before_any_launch(plsh):
     rc = lib.plsh_attention_varlen_fwd_static(fake, fake, fake, 0, 1, 40, 8, 131072, 128, null, 64, null, fake,
                                               fake, 1, fake, fake, fake, null)
     assert rc == 3 and "static buffer" in plsh.plsh_last_error()
+
+
+def test_decode_rejects_bad_arguments_before_any_launch(plsh):
+    lib = plsh._lib
+    null = None
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the checks fail first
+    args = lambda m=4, pos=fake, d=128, H_kv=1, causal=1: (fake, pos, m, fake, fake, 0, 1, 2, H_kv, 256, d, 20, fake,
+                                                           causal, fake, fake, fake, null)
+    assert lib.plsh_decode_fwd(*args(m=0)) == 1 and "m >= 1" in plsh.plsh_last_error()
+    assert lib.plsh_decode_fwd(*args(pos=null)) == 1 and "null" in plsh.plsh_last_error()
+    assert lib.plsh_decode_fwd(*args(d=96)) == 2
+    assert lib.plsh_decode_fwd(*args(H_kv=3)) == 1
+    assert lib.plsh_decode_fwd(*args(causal=2)) == 1
