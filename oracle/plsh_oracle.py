@@ -41,6 +41,7 @@ __all__ = [
     "bins", "bin_ids", "hash_mask", "match_counts", "mean_mask", "counts_rows",
     "boundary_bits", "block_lengths", "bmax", "tile_spans", "varlen_spans", "alibi_matrix",
     "approx_attention", "exact_attention", "forward", "forward_exact",
+    "approx_attention_grad", "backward",
     "COUNTER_HEAD_SHIFT", "TILE",
 ]
 
@@ -356,3 +357,64 @@ def forward_exact(Q: np.ndarray, K: np.ndarray, V: np.ndarray, sigma: Sequence[f
             O[b, h], _ = exact_attention(Q[b, h], K[b, h // group], V[b, h // group],
                                          float(sigma[h]), causal, rows)
     return O
+
+
+# ---------------------------------------------------------------------------
+# Gradients of T~ (training with Positional LSH in place of ALiBi)
+# ---------------------------------------------------------------------------
+
+def approx_attention_grad(q: np.ndarray, k: np.ndarray, v: np.ndarray, do: np.ndarray, ids_hs: np.ndarray,
+                          causal: bool) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """dQ, dK, dV of <dO, T~> for one query head (float64), the table held fixed.
+
+    The pages train and fine-tune models with Positional LSH in the attention
+    ([nl R], experimental validation: Qwen3 from scratch, Mistral-7B
+    fine-tuning), which needs these gradients; they follow from T~ by the
+    chain rule. With P_ij = M~_ij e^{S_ij} / sum_l M~_il e^{S_il} (the row
+    weights of T~ = P V, [nl M2], [nl M3]) and S = q k^T / sqrt d:
+        dV = P^T dO,  dP = dO V^T,  D_i = sum_j P_ij dP_ij (= dO_i . T~_i),
+        dS = P o (dP - D 1^T),  dQ = dS K / sqrt d,  dK = dS^T Q / sqrt d.
+    The M~ weights only scale P; entries with M~_ij = 0 (and j > i when
+    causal) carry no gradient.
+    """
+    n, d = k.shape
+    S = (q @ k.T) / math.sqrt(d)
+    W = match_counts(ids_hs).astype(np.float64) / ids_hs.shape[0]
+    if causal:
+        W[np.arange(n)[None, :] > np.arange(n)[:, None]] = 0.0
+    valid = W > 0
+    m = np.where(valid, S, -np.inf).max(axis=1)
+    A = np.where(valid, np.exp(np.where(valid, S - m[:, None], 0.0)), 0.0) * W
+    P = A / A.sum(axis=1)[:, None]
+    O = P @ v
+    dV = P.T @ do
+    dP = do @ v.T
+    Dv = (do * O).sum(axis=1)
+    dS = P * (dP - Dv[:, None])
+    dQ = dS @ k / math.sqrt(d)
+    dK = dS.T @ q / math.sqrt(d)
+    return dQ, dK, dV
+
+
+def backward(Q: np.ndarray, K: np.ndarray, V: np.ndarray, dO: np.ndarray, table: np.ndarray,
+             causal: bool) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Multi-head gradients, layout as forward(): dQ like Q, dK and dV like K.
+
+    Grouped-query attention: KV head g collects the gradients of every query
+    head h with h // (H / H_kv) == g.
+    """
+    B, H, n, d = Q.shape
+    H_kv = K.shape[1]
+    group = H // H_kv
+    ids = bin_ids(table, n)
+    dQ = np.zeros_like(Q, dtype=np.float64)
+    dK = np.zeros(K.shape, dtype=np.float64)
+    dV = np.zeros(V.shape, dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            g = h // group
+            dq, dk, dv = approx_attention_grad(Q[b, h], K[b, g], V[b, g], dO[b, h], ids[h], causal)
+            dQ[b, h] = dq
+            dK[b, g] += dk
+            dV[b, g] += dv
+    return dQ, dK, dV

@@ -398,3 +398,81 @@ def check_rows_and_gqa(orc, n=160, d=8):
         # head 1 reads KV head 0, head 2 reads KV head 1
         O1, _ = orc.approx_attention(Q[0, 2], K[0, 1], V[0, 1], orc.bin_ids(table, n)[2], causal)
         np.testing.assert_allclose(O[0, 2], O1, rtol=1e-13, atol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# Gradients
+# ---------------------------------------------------------------------------
+
+def _counts_by_definition(ids_hs):
+    """c_ij = number of hashes putting positions i and j in one bin, by direct comparison."""
+    return sum((row[:, None] == row[None, :]).astype(np.float64) for row in ids_hs)
+
+
+def check_grad_autograd(orc, n=150, d=8):
+    """Gradients against torch autograd of softmax(S + ln c) V: T~ is that softmax attention for
+    any table (ln 0 = -inf drops the pair), so the library's reverse mode gives the exact answer."""
+    r = np.random.default_rng(21)
+    q, k, v, do = (r.standard_normal((n, d)) for _ in range(4))
+    for sigma, s in ((3.0, 5), (20.0, 12), (0.7, 3)):
+        ids = orc.bin_ids(orc.draw_table(31 + s, [sigma], s), n)[0]
+        W = _counts_by_definition(ids)
+        for causal in (False, True):
+            Wc = np.tril(W) if causal else W
+            tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+            bias = torch.from_numpy(np.where(Wc > 0, np.log(np.where(Wc > 0, Wc, 1.0)), -np.inf))
+            att = torch.softmax(tq @ tk.T / math.sqrt(d) + bias, dim=1)
+            (att @ tv).backward(torch.from_numpy(do))
+            dq, dk, dv = orc.approx_attention_grad(q, k, v, do, ids, causal)
+            np.testing.assert_allclose(dq, tq.grad.numpy(), rtol=1e-10, atol=1e-12)
+            np.testing.assert_allclose(dk, tk.grad.numpy(), rtol=1e-10, atol=1e-12)
+            np.testing.assert_allclose(dv, tv.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def check_grad_finite_differences(orc, n=12, d=3, eps=1e-6):
+    """Central differences of f = <dO, T~> computed with the oracle's forward."""
+    r = np.random.default_rng(22)
+    q, k, v, do = (r.standard_normal((n, d)) for _ in range(4))
+    ids = orc.bin_ids(orc.draw_table(5, [2.5], 4), n)[0]
+    for causal in (False, True):
+        grads = orc.approx_attention_grad(q, k, v, do, ids, causal)
+        for which in range(3):
+            for (i, e) in ((0, 0), (5, 1), (11, 2), (7, 0)):
+                xs = [q.copy(), k.copy(), v.copy()]
+                xs[which][i, e] += eps
+                fp = (orc.approx_attention(*xs, ids, causal)[0] * do).sum()
+                xs[which][i, e] -= 2 * eps
+                fm = (orc.approx_attention(*xs, ids, causal)[0] * do).sum()
+                fd = (fp - fm) / (2 * eps)
+                assert abs(fd - grads[which][i, e]) <= 1e-7 * max(1.0, abs(fd)), (which, i, e, fd,
+                                                                                  grads[which][i, e])
+
+
+def check_grad_singleton_bins(orc, n=60, d=8):
+    """delta < 1: T~ = V whatever Q and K are, so dV = dO and dQ = dK = 0."""
+    r = np.random.default_rng(23)
+    q, k, v, do = (r.standard_normal((n, d)) for _ in range(4))
+    ids = orc.bin_ids(np.array([[[0.5, 0.25], [0.9, 0.1]]]), n)[0]
+    for causal in (False, True):
+        dq, dk, dv = orc.approx_attention_grad(q, k, v, do, ids, causal)
+        np.testing.assert_allclose(dv, do, rtol=0, atol=1e-14)
+        assert np.abs(dq).max() <= 1e-14 and np.abs(dk).max() <= 1e-14
+
+
+def check_backward_gqa(orc, n=90, d=6):
+    """Multi-head gradients: GQA equals MHA on repeated K/V with the group's dK, dV summed."""
+    r = np.random.default_rng(24)
+    B, H, Hkv = 2, 4, 2
+    Q, dO = r.standard_normal((B, H, n, d)), r.standard_normal((B, H, n, d))
+    K, V = r.standard_normal((B, Hkv, n, d)), r.standard_normal((B, Hkv, n, d))
+    table = orc.draw_table(25, [2.0, 5.0, 11.0, 30.0], 6)
+    for causal in (False, True):
+        dQ, dK, dV = orc.backward(Q, K, V, dO, table, causal)
+        dQr, dKr, dVr = orc.backward(Q, np.repeat(K, 2, axis=1), np.repeat(V, 2, axis=1), dO, table, causal)
+        np.testing.assert_allclose(dQ, dQr, rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(dK, dKr[:, 0::2] + dKr[:, 1::2], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(dV, dVr[:, 0::2] + dVr[:, 1::2], rtol=1e-12, atol=1e-13)
+        # query head 3 reads KV head 1
+        ids3 = orc.bin_ids(table, n)[3]
+        dq3, _, _ = orc.approx_attention_grad(Q[1, 3], K[1, 1], V[1, 1], dO[1, 3], ids3, causal)
+        np.testing.assert_allclose(dQ[1, 3], dq3, rtol=1e-13, atol=1e-13)

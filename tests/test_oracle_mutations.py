@@ -154,6 +154,42 @@ def _bmax_interior_only(ids_hs):
     return int(max(O.block_lengths(ids_hs[k])[1:-1].max(initial=1) for k in range(ids_hs.shape[0])))
 
 
+def _grad_no_row_term(q, k, v, do, ids_hs, causal):
+    # drops D_i from dS = P o (dP - D)
+    n, d = k.shape
+    S = (q @ k.T) / math.sqrt(d)
+    W = O.match_counts(ids_hs).astype(np.float64)
+    if causal:
+        W = np.tril(W)
+    A = np.where(W > 0, np.exp(S - S.max(axis=1, keepdims=True)), 0.0) * W
+    P_ = A / A.sum(axis=1, keepdims=True)
+    dS = P_ * (do @ v.T)
+    return dS @ k / math.sqrt(d), dS.T @ q / math.sqrt(d), P_.T @ do
+
+
+def _grad_dk_unscaled(q, k, v, do, ids_hs, causal):
+    dq, dk, dv = _ORIG_GRAD(q, k, v, do, ids_hs, causal)
+    return dq, dk * math.sqrt(k.shape[1]), dv
+
+
+def _backward_wrong_gqa(Q, K, V, dO, table, causal):
+    # query head h reads KV head h % H_kv instead of h // (H / H_kv)
+    B, H, n, d = Q.shape
+    H_kv = K.shape[1]
+    ids = O.bin_ids(table, n)
+    dQ, dK, dV = np.zeros(Q.shape), np.zeros(K.shape), np.zeros(V.shape)
+    for b in range(B):
+        for h in range(H):
+            g = h % H_kv
+            dq, dk, dv = O.approx_attention_grad(Q[b, h], K[b, g], V[b, g], dO[b, h], ids[h], causal)
+            dQ[b, h] = dq
+            dK[b, g] += dk
+            dV[b, g] += dv
+    return dQ, dK, dV
+
+
+_ORIG_GRAD = O.approx_attention_grad
+
 MUTATIONS = [
     ("draw_table", _draw_table_shape1, [P.check_table_moments, P.check_table_laws]),
     ("draw_table", _draw_table_scale_rate, [P.check_table_moments]),
@@ -171,6 +207,9 @@ MUTATIONS = [
     ("bmax", _bmax_interior_only, [P.check_bins_worked]),
     ("varlen_spans", _varlen_union_window, [P.check_bins_worked, P.check_varlen_spans_from_blocks]),
     ("varlen_spans", _varlen_shared_row, [P.check_bins_worked, P.check_varlen_spans_from_blocks]),
+    ("approx_attention_grad", _grad_no_row_term, [P.check_grad_autograd, P.check_grad_finite_differences]),
+    ("approx_attention_grad", _grad_dk_unscaled, [P.check_grad_autograd, P.check_grad_finite_differences]),
+    ("backward", _backward_wrong_gqa, [P.check_backward_gqa]),
 ]
 
 

@@ -87,3 +87,19 @@ def test_convergence_in_s():
 
 def test_sampled_rows_and_gqa():
     P.check_rows_and_gqa(oracle)
+
+
+def test_gradients_match_autograd_of_log_count_bias():
+    P.check_grad_autograd(oracle)
+
+
+def test_gradients_match_finite_differences():
+    P.check_grad_finite_differences(oracle)
+
+
+def test_gradients_of_singleton_bins():
+    P.check_grad_singleton_bins(oracle)
+
+
+def test_backward_gqa():
+    P.check_backward_gqa(oracle)
