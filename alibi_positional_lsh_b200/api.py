@@ -8,6 +8,7 @@ with torch) and runs the whole path:
   a4 plsh_attention_fwd (K3)    -> O, row_sum
   a5 plsh_attention_varlen_fwd (K4, the per-sample comparator) -> the same O, row_sum
   plsh_decode_fwd (single query rows against the cached K, V) -> rows of T~, row_sum
+  plsh_attention_bwd (training) -> dQ, dK, dV of T~ with the table fixed
   plsh_alibi_banded_fwd (exact banded ALiBi, what the method approximates) -> T*, row_sum
 All arithmetic of a2..a5 runs in libplsh's CUDA kernels.
 """
@@ -19,7 +20,7 @@ import numpy as np
 import torch
 
 from . import (PLSH_BF16, PLSH_F32, PLSH_TILE, PlshError, decode_device_error, plsh_alibi_banded_fwd,
-               plsh_attention_fwd, plsh_attention_varlen_fwd, plsh_decode_fwd, plsh_draw_table, plsh_sample_bins,
+               plsh_attention_bwd, plsh_attention_fwd, plsh_attention_varlen_fwd, plsh_decode_fwd, plsh_draw_table, plsh_sample_bins,
                plsh_varlen_scratch_bytes, plsh_window)
 
 
@@ -54,6 +55,7 @@ class PlshForward:
         self.O = torch.empty((B, H, n, d), dtype=dtype, device=dev)
         self.row_sum = torch.empty((B, H, n), dtype=torch.float32, device=dev)
         self.scratch = None  # per-hash windows of the comparator, allocated on first use
+        self.grads = None    # (delta, dQ, dK, dV) of backward(), allocated on first use
 
     # a1 + a2 + a3
     def prepare(self, stream: Optional[torch.cuda.Stream] = None, table: Optional[np.ndarray] = None) -> None:
@@ -122,6 +124,27 @@ class PlshForward:
         plsh_alibi_banded_fwd(q, k, v, self.dtype_code, B, H, H_kv, n, d, self.sigma_dev, float(eps),
                               int(self.causal), self.O, self.row_sum, self.err, st)
         return self.O, self.row_sum
+
+    def backward(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dO: torch.Tensor,
+                 stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+        """dQ, dK, dV of <dO, T~> for the inputs of the last attend() (its O and row_sum, the same table)."""
+        B, H, H_kv, n, d = self.B, self.H, self.H_kv, self.n, self.d
+        if q.shape != (B, H, n, d) or dO.shape != (B, H, n, d) or k.shape != (B, H_kv, n, d) \
+                or v.shape != (B, H_kv, n, d):
+            raise ValueError("q/k/v/dO shapes do not match the plan")
+        for t, nm in ((q, "q"), (k, "k"), (v, "v"), (dO, "dO")):
+            if t.dtype != self.dtype or t.device != self.O.device:
+                raise ValueError(f"{nm} must be {self.dtype} on {self.O.device}")
+        if self.grads is None:
+            dev = self.O.device
+            self.grads = (torch.empty((B, H, n), dtype=torch.float32, device=dev), torch.empty_like(self.O),
+                          torch.empty((B, H_kv, n, d), dtype=self.dtype, device=dev),
+                          torch.empty((B, H_kv, n, d), dtype=self.dtype, device=dev))
+        delta, dQ, dK, dV = self.grads
+        st = torch.cuda.current_stream() if stream is None else stream
+        plsh_attention_bwd(q, k, v, self.O, dO, self.row_sum, self.dtype_code, B, H, H_kv, n, d, self.s, self.ids,
+                           int(self.causal), delta, dQ, dK, dV, self.err, st)
+        return dQ, dK, dV
 
     def decode(self, q_rows: torch.Tensor, pos: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:

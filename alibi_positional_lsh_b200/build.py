@@ -29,6 +29,7 @@ SOURCES = [
     "plsh_attn_tc.cu",
     "plsh_varlen.cu",
     "plsh_decode.cu",
+    "plsh_bwd.cu",
 ]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -253,3 +253,28 @@ extern "C" int plsh_decode_fwd(const void* Q, const int32_t* pos_dev, int m, con
   plsh::DecodeArgs a{Q, pos_dev, m, K, V, dtype, B, H, H_kv, n, d, s, causal, bmask_dev, O, row_sum, err_dev};
   return plsh::launch_decode(a, static_cast<cudaStream_t>(stream));
 }
+
+// ---------------------------------------------------------------- backward
+
+extern "C" int plsh_attention_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                                  const float* row_sum, int dtype, int B, int H, int H_kv, int n, int d, int s,
+                                  const int32_t* ids_dev, int causal, float* delta_dev, void* dQ, void* dK,
+                                  void* dV, uint32_t* err_dev, void* stream) {
+  const char* fn = "plsh_attention_bwd";
+  if (int rc = plsh::check_sizes(fn, H, s, n)) return rc;
+  if (B < 1 || B > 65535) return fail(PLSH_ERR_INVALID_ARG, "%s: need 1 <= B <= 65535 (B=%d)", fn, B);
+  if (H_kv < 1 || H % H_kv != 0)
+    return fail(PLSH_ERR_INVALID_ARG, "%s: H_kv must divide H (H=%d H_kv=%d)", fn, H, H_kv);
+  if (causal != 0 && causal != 1) return fail(PLSH_ERR_INVALID_ARG, "%s: causal must be 0 or 1", fn);
+  if (dtype != PLSH_BF16 && dtype != PLSH_F32) return fail(PLSH_ERR_UNSUPPORTED, "%s: dtype %d", fn, dtype);
+  if (d != 64 && d != 128) return fail(PLSH_ERR_UNSUPPORTED, "%s: head dim %d (64 or 128 supported)", fn, d);
+  if (!Q || !K || !V || !O || !dO || !row_sum || !ids_dev || !delta_dev || !dQ || !dK || !dV || !err_dev)
+    return fail(PLSH_ERR_INVALID_ARG, "%s: null pointer", fn);
+  if (!plsh::aligned16(Q) || !plsh::aligned16(K) || !plsh::aligned16(V) || !plsh::aligned16(O) ||
+      !plsh::aligned16(dO))
+    return fail(PLSH_ERR_INVALID_ARG, "%s: Q, K, V, O and dO must be 16-byte aligned", fn);
+  if (static_cast<size_t>(B) * H * n > (size_t{1} << 31))
+    return fail(PLSH_ERR_RANGE, "%s: B*H*n exceeds 2^31", fn);
+  plsh::BwdArgs a{Q, K, V, O, dO, row_sum, ids_dev, dtype, B, H, H_kv, n, d, s, causal, delta_dev, dQ, dK, dV};
+  return plsh::launch_bwd(a, static_cast<cudaStream_t>(stream));
+}

@@ -46,6 +46,15 @@ struct DecodeArgs {
   void* O; float* row_sum; uint32_t* err;
 };
 int launch_decode(const DecodeArgs& a, cudaStream_t st);
+// Backward: dQ, dK, dV of T~ (Q, O, dO, dQ [B][H][n][d]; K, V, dK, dV [B][H_kv][n][d]).
+struct BwdArgs {
+  const void* Q; const void* K; const void* V; const void* O; const void* dO;
+  const float* row_sum; const int32_t* ids;
+  int dtype, B, H, H_kv, n, d, s, causal;
+  float* delta;
+  void* dQ; void* dK; void* dV;
+};
+int launch_bwd(const BwdArgs& a, cudaStream_t st);
 int launch_varlen_spans(const int32_t* ids, int H, int s, int n, int causal, int32_t* spans, cudaStream_t st);
 int launch_attention_simt(const AttnArgs& a, cudaStream_t st);
 int launch_attention_tc(const AttnArgs& a, cudaStream_t st);

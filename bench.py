@@ -273,6 +273,70 @@ def decode_keys(bmask: np.ndarray, s: int, i: int, causal: bool) -> int:
     return total
 
 
+BWD_TILE = 64
+FP32_LANES_PER_SM = 128   # fp32 FMA lanes per SM (4 sub-partitions x 32)
+
+
+def bwd_chunk_pairs(ids: np.ndarray, causal: bool, group: int) -> tuple:
+    """(query-tile x key-chunk pairs of bwd_dq_kernel, key-tile x query-chunk pairs of bwd_dkdv_kernel) for one
+    batch element: per 64-position tile the range of positions sharing a block with it in some hash (first
+    position of the first row's block to the last of the last row's block, widest over the hashes), walked in
+    chunks of 64. ids: [H][s][n]."""
+    H, s, n = ids.shape
+    T = (n + BWD_TILE - 1) // BWD_TILE
+    a = np.arange(T) * BWD_TILE
+    b = np.minimum(n - 1, a + BWD_TILE - 1)
+    dq = dkdv = 0
+    for h in range(H):
+        lo = np.full(T, n, np.int64)
+        hi = np.full(T, -1, np.int64)
+        for k in range(s):
+            row = ids[h, k]
+            lo = np.minimum(lo, np.searchsorted(row, row[a], "left"))
+            hi = np.maximum(hi, np.searchsorted(row, row[b], "right") - 1)
+        hq = np.minimum(hi, b) if causal else hi          # dQ: keys j <= i
+        lk = np.maximum(lo, a) if causal else lo          # dK, dV: rows i >= j
+        dq += int(((hq - lo) // BWD_TILE + 1).sum())
+        dkdv += int(((hi - lk) // BWD_TILE + 1).sum())
+    return dq, dkdv
+
+
+def bwd_timing(plan, q, k, v, stream, w, sm_count: int, sm_max_mhz: float):
+    """plsh_attention_bwd on the step's inputs with a seeded dO: device time per call and its issued fp32
+    FLOPs (per 64 x 64 pair: S, dP and dQ in the dQ kernel, S, dP, dV and dK in the dK/dV kernel, 2d each)
+    against the CUDA-core fp32 FMA peak derived from the SM count and the maximum SM clock."""
+    g = torch.Generator(device=q.device).manual_seed(w.seed + 99)
+    dO = torch.randn(q.shape, generator=g, device=q.device, dtype=torch.float32).to(q.dtype)
+    plan.attend(q, k, v, stream)             # O and row_sum of these inputs
+    for _ in range(2):
+        plan.backward(q, k, v, dO, stream)
+    ts = []
+    for _ in range(5):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        plan.backward(q, k, v, dO, stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    errs = plan.device_errors()
+    if errs:
+        raise RuntimeError(f"device errors in backward: {errs}")
+    ids = plan.ids.cpu().numpy()
+    dq_pairs, dkdv_pairs = bwd_chunk_pairs(ids, w.causal, w.H // w.H_kv)
+    per_pair = 2.0 * w.d * BWD_TILE * BWD_TILE
+    flops = (3 * dq_pairs + 4 * dkdv_pairs) * per_pair * w.B
+    ms = float(np.median(ts))
+    peak = sm_count * FP32_LANES_PER_SM * 2 * sm_max_mhz * 1e6 / 1e12
+    achieved = flops / (ms * 1e-3) / 1e12
+    return {"path": "backward (plsh_attention_bwd): dQ, dK, dV of T~, fp32 CUDA-core arithmetic",
+            "kernels": ["bwd_delta_kernel", "bwd_dkdv_kernel", "bwd_dq_kernel"], "ms_per_call": ms,
+            "issued_fp32_flops": flops, "achieved_TFLOPs": achieved,
+            "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak,
+                         "peak_source": f"derived: {sm_count} SMs x {FP32_LANES_PER_SM} fp32 lanes x 2 x "
+                                        f"{sm_max_mhz:.0f} MHz"}}
+
+
 def decode_timing(plan, q, k, v, stream, w):
     """plsh_decode_fwd on the newest position (one query row per (b, h) at i = n-1) against the whole
     cache: device time per call and the K/V bytes it must read (the weighted keys' rows)."""
@@ -441,6 +505,11 @@ def run_ours(args, rank, world, local):
                            "this_path_speedup": float(np.median(ts)) / attn_avg})
 
     decode = decode_timing(plan, q, k, v, stream, w) if (world == 1 and not alibi) else None
+    bwd = None
+    if world == 1 and not alibi and not args.no_backward:
+        props = torch.cuda.get_device_properties(local)
+        bwd = bwd_timing(plan, q, k, v, stream, w, props.multi_processor_count,
+                         float(clocks.get("sm_max_mhz") or 1965))
 
     tokens = w.B * w.n * world
     value = job_value(w.B * w.n, world, ms_step)
@@ -506,6 +575,8 @@ def run_ours(args, rank, world, local):
         line["comparison"] = others
     if decode:
         line["decode"] = decode
+    if bwd:
+        line["backward"] = bwd
     if rank == 0 and not args.no_cpu_baseline:
         sampler = OracleSampler(w)
         rate, desc = sampler.run(args.cpu_seconds)
@@ -561,6 +632,7 @@ def main(argv=None):
     ap.add_argument("--workload", default=workloads.HEADLINE, choices=list(workloads.WORKLOADS))
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-backward", action="store_true", help="skip timing plsh_attention_bwd beside the step")
     ap.add_argument("--path", choices=["fused", "varlen", "alibi"], default="fused",
                     help="attention path timed: the fused kernel (K3), the per-sample comparator (K4) or "
                          "exact banded ALiBi")

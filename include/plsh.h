@@ -306,6 +306,40 @@ PLSH_API int plsh_decode_fwd(const void* Q, const int32_t* pos_dev, int m, const
                              int B, int H, int H_kv, int n, int d, int s, const void* bmask_dev, int causal,
                              void* O, float* row_sum, uint32_t* err_dev, void* stream);
 
+/*
+ * plsh_attention_bwd -- gradients of T~ for training: dQ, dK, dV of
+ * <dO, O> with the (delta, u) table, and so the bins, held fixed.
+ *
+ * Cites: Methodology 2 and 3 (T~ = P V with row weights P_ij = M~_ij e^{S_ij}
+ * / sum_l M~_il e^{S_il}) and the Results' experimental validation (models
+ * trained from scratch and fine-tuned with Positional LSH in the attention,
+ * which needs these gradients). With the forward's row_sum L_i,
+ * P_ij = (c_ij / s) e^{S_ij - L_i} is recomputed, and
+ *   dV = P^T dO,  D_i = dO_i . O_i,  dS = P o (dO V^T - D),
+ *   dQ = dS K / sqrt d,  dK = dS^T Q / sqrt d,
+ * restricted to j <= i when causal. For grouped-query attention dK and dV of
+ * KV head g sum the query heads h with h / (H/H_kv) == g.
+ *
+ *   Q, O, dO       [B][H][n][d]; O and row_sum are plsh_attention_fwd's
+ *                  outputs for the same inputs, table and causal flag.
+ *   K, V           [B][H_kv][n][d].
+ *   row_sum        [B][H][n] float32, the forward's.
+ *   dtype, d, s    as plsh_attention_fwd (both dtypes compute in fp32 on
+ *                  CUDA cores).
+ *   ids_dev        [H][s][n] int32 bin ids from plsh_sample_bins (the
+ *                  key and query ranges of every tile come from them; no
+ *                  masks or windows are needed).
+ *   delta_dev      [B][H][n] float32 scratch (written: D_i).
+ *   dQ             [B][H][n][d] out; dK, dV [B][H_kv][n][d] out, each row
+ *                  written once (no accumulation into the caller's buffers).
+ *   err_dev        device error word (no bit is set today).
+ * Q, K, V, O and dO must be 16-byte aligned.
+ */
+PLSH_API int plsh_attention_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                                const float* row_sum, int dtype, int B, int H, int H_kv, int n, int d, int s,
+                                const int32_t* ids_dev, int causal, float* delta_dev, void* dQ, void* dK,
+                                void* dV, uint32_t* err_dev, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

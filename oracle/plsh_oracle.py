@@ -41,7 +41,7 @@ __all__ = [
     "bins", "bin_ids", "hash_mask", "match_counts", "mean_mask", "counts_rows",
     "boundary_bits", "block_lengths", "bmax", "tile_spans", "varlen_spans", "alibi_matrix",
     "approx_attention", "exact_attention", "forward", "forward_exact",
-    "approx_attention_grad", "backward",
+    "approx_attention_grad", "approx_attention_grad_sampled", "backward",
     "COUNTER_HEAD_SHIFT", "TILE",
 ]
 
@@ -393,6 +393,60 @@ def approx_attention_grad(q: np.ndarray, k: np.ndarray, v: np.ndarray, do: np.nd
     dS = P * (dP - Dv[:, None])
     dQ = dS @ k / math.sqrt(d)
     dK = dS.T @ q / math.sqrt(d)
+    return dQ, dK, dV
+
+
+def approx_attention_grad_sampled(q: np.ndarray, k: np.ndarray, v: np.ndarray, do: np.ndarray,
+                                  ids_hs: np.ndarray, causal: bool, rows: Sequence[int], keys: Sequence[int],
+                                  chunk: int = 256) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """dQ on `rows` and dK, dV on `keys` of approx_attention_grad, for long sequences (float64).
+
+    The same formulas, evaluated only where they are needed: a query row's
+    dQ needs its own row of P and dS; a key's dK and dV collect P_ij and
+    dS_ij over the rows i that give it weight (c_ij > 0, and i >= j when
+    causal), and each of those rows needs its whole row of P (for D_i).
+    Rows are processed `chunk` at a time, each over the keys its rows weight.
+    """
+    n, d = k.shape
+    sq = math.sqrt(d)
+    s = ids_hs.shape[0]
+
+    def rows_pass(r):
+        W = counts_rows(ids_hs, r).astype(np.float64) / s
+        if causal:
+            W[np.arange(n)[None, :] > r[:, None]] = 0.0
+        cols = np.nonzero((W > 0).any(axis=0))[0]
+        Wc = W[:, cols]
+        S = (q[r] @ k[cols].T) / sq
+        valid = Wc > 0
+        m = np.where(valid, S, -np.inf).max(axis=1)
+        A = np.where(valid, np.exp(np.where(valid, S - m[:, None], 0.0)), 0.0) * Wc
+        P = A / A.sum(axis=1)[:, None]
+        Dv = (do[r] * (P @ v[cols])).sum(axis=1)
+        dS = P * (do[r] @ v[cols].T - Dv[:, None])
+        return cols, P, dS
+
+    rows = np.asarray(rows, dtype=np.int64)
+    keys = np.asarray(keys, dtype=np.int64)
+    dQ = np.zeros((0, d))
+    if len(rows):
+        cols, _, dS = rows_pass(rows)
+        dQ = dS @ k[cols] / sq
+    # rows reaching the keys: c_ij = c_ji, so they are the positions the keys weight
+    reach = (counts_rows(ids_hs, keys) > 0)
+    if causal:
+        reach &= np.arange(n)[None, :] >= keys[:, None]
+    R = np.nonzero(reach.any(axis=0))[0]
+    dK = np.zeros((len(keys), d))
+    dV = np.zeros((len(keys), d))
+    for c0 in range(0, len(R), chunk):
+        r = R[c0:c0 + chunk]
+        cols, P, dS = rows_pass(r)
+        at = np.searchsorted(cols, keys)
+        hit = (at < len(cols)) & (cols[np.minimum(at, len(cols) - 1)] == keys)
+        for t in np.nonzero(hit)[0]:
+            dK[t] += dS[:, at[t]] @ q[r] / sq
+            dV[t] += P[:, at[t]] @ do[r]
     return dQ, dK, dV
 
 

@@ -476,3 +476,20 @@ def check_backward_gqa(orc, n=90, d=6):
         ids3 = orc.bin_ids(table, n)[3]
         dq3, _, _ = orc.approx_attention_grad(Q[1, 3], K[1, 1], V[1, 1], dO[1, 3], ids3, causal)
         np.testing.assert_allclose(dQ[1, 3], dq3, rtol=1e-13, atol=1e-13)
+
+
+def check_grad_sampled_equals_full(orc, n=700, d=8):
+    """The sampled gradients equal the full ones on the same rows and keys (small chunks force
+    several passes over the reaching rows)."""
+    r = np.random.default_rng(26)
+    q, k, v, do = (r.standard_normal((n, d)) for _ in range(4))
+    rows = [0, 1, 128, 350, 699]
+    keys = [0, 5, 300, 640, 699]
+    for sigma in (3.0, 40.0):
+        ids = orc.bin_ids(orc.draw_table(27, [sigma], 7), n)[0]
+        for causal in (False, True):
+            dq, dk, dv = orc.approx_attention_grad(q, k, v, do, ids, causal)
+            sq_, sk, sv = orc.approx_attention_grad_sampled(q, k, v, do, ids, causal, rows, keys, chunk=64)
+            np.testing.assert_allclose(sq_, dq[rows], rtol=1e-10, atol=1e-12)
+            np.testing.assert_allclose(sk, dk[keys], rtol=1e-10, atol=1e-12)
+            np.testing.assert_allclose(sv, dv[keys], rtol=1e-10, atol=1e-12)

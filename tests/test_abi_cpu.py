@@ -147,3 +147,18 @@ def test_decode_rejects_bad_arguments_before_any_launch(plsh):
     assert lib.plsh_decode_fwd(*args(d=96)) == 2
     assert lib.plsh_decode_fwd(*args(H_kv=3)) == 1
     assert lib.plsh_decode_fwd(*args(causal=2)) == 1
+
+
+def test_backward_rejects_bad_arguments_before_any_launch(plsh):
+    lib = plsh._lib
+    null = None
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the checks fail first
+    args = lambda d=128, H_kv=1, causal=1, ids=fake, dtype=0, Q=fake: (Q, fake, fake, fake, fake, fake, dtype, 1, 2,
+                                                                        H_kv, 256, d, 20, ids, causal, fake, fake,
+                                                                        fake, fake, fake, null)
+    assert lib.plsh_attention_bwd(*args(ids=null)) == 1 and "null" in plsh.plsh_last_error()
+    assert lib.plsh_attention_bwd(*args(d=96)) == 2
+    assert lib.plsh_attention_bwd(*args(H_kv=3)) == 1
+    assert lib.plsh_attention_bwd(*args(causal=2)) == 1
+    assert lib.plsh_attention_bwd(*args(dtype=9)) == 2
+    assert lib.plsh_attention_bwd(*args(Q=ctypes.c_void_p((1 << 20) + 4))) == 1 and "aligned" in plsh.plsh_last_error()

@@ -189,6 +189,14 @@ def _backward_wrong_gqa(Q, K, V, dO, table, causal):
 
 
 _ORIG_GRAD = O.approx_attention_grad
+_ORIG_SAMPLED = O.approx_attention_grad_sampled
+
+
+def _sampled_reach_ignores_causal(q, k, v, do, ids_hs, causal, rows, keys, chunk=256):
+    # collects dK, dV from the non-causal rows' P (rows above the key are skipped, but P is not causal)
+    dq, _, _ = _ORIG_SAMPLED(q, k, v, do, ids_hs, causal, rows, keys, chunk)
+    _, dk, dv = _ORIG_SAMPLED(q, k, v, do, ids_hs, False, rows, keys, chunk)
+    return dq, dk, dv
 
 MUTATIONS = [
     ("draw_table", _draw_table_shape1, [P.check_table_moments, P.check_table_laws]),
@@ -210,6 +218,7 @@ MUTATIONS = [
     ("approx_attention_grad", _grad_no_row_term, [P.check_grad_autograd, P.check_grad_finite_differences]),
     ("approx_attention_grad", _grad_dk_unscaled, [P.check_grad_autograd, P.check_grad_finite_differences]),
     ("backward", _backward_wrong_gqa, [P.check_backward_gqa]),
+    ("approx_attention_grad_sampled", _sampled_reach_ignores_causal, [P.check_grad_sampled_equals_full]),
 ]
 
 

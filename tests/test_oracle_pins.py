@@ -103,3 +103,7 @@ def test_gradients_of_singleton_bins():
 
 def test_backward_gqa():
     P.check_backward_gqa(oracle)
+
+
+def test_sampled_gradients_equal_full():
+    P.check_grad_sampled_equals_full(oracle)
