@@ -201,4 +201,4 @@ def decode_device_error(word: int) -> list:
     return [name for bit, name in DEVERR_BITS.items() if word & bit]
 
 
-from .api import PlshForward, fixed_blocks_table, forward  # noqa: E402,F401
+from .api import HostPipeline, PlshForward, fixed_blocks_table, forward  # noqa: E402,F401

@@ -203,6 +203,67 @@ class PlshForward:
             raise PlshError(-1, "device reported " + ",".join(errs))
 
 
+class HostPipeline:
+    """T~ for a stream of batches that live in pinned host memory, with the copies overlapped.
+
+    Each step copies one batch's Q, K, V in, runs the table draw, K1, K2 and K3,
+    and copies O and row_sum out. Two device buffer sets alternate, so the
+    host->device copy of step t+1 runs while step t computes and while its
+    outputs travel device->host (the link carries both directions at once).
+    Every step draws its table from the plan's seed, as PlshForward.run_host does.
+    """
+
+    def __init__(self, plan: PlshForward):
+        self.plan = plan
+        dev = plan.O.device
+        B, H, H_kv, n, d = plan.B, plan.H, plan.H_kv, plan.n, plan.d
+        self.sets = [dict(q=torch.empty((B, H, n, d), dtype=plan.dtype, device=dev),
+                          k=torch.empty((B, H_kv, n, d), dtype=plan.dtype, device=dev),
+                          v=torch.empty((B, H_kv, n, d), dtype=plan.dtype, device=dev),
+                          O=torch.empty_like(plan.O), R=torch.empty_like(plan.row_sum)) for _ in range(2)]
+        self.copy_in = torch.cuda.Stream(dev)
+        self.copy_out = torch.cuda.Stream(dev)
+        self.inputs_ready = [torch.cuda.Event() for _ in range(2)]
+        self.computed = [torch.cuda.Event() for _ in range(2)]
+        self.copied_out = [torch.cuda.Event() for _ in range(2)]
+        self.t = 0
+
+    def step(self, q_host: torch.Tensor, k_host: torch.Tensor, v_host: torch.Tensor, o_host: torch.Tensor,
+             rs_host: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None) -> None:
+        """Enqueues one batch: pinned host Q, K, V in; O (and row_sum) written to the pinned host buffers once the
+        step's copy-out has run (after synchronize(), or after the next steps' events)."""
+        plan, i = self.plan, self.t % 2
+        buf = self.sets[i]
+        compute = torch.cuda.current_stream() if stream is None else stream
+        if self.t >= 2:
+            self.copy_in.wait_event(self.computed[i])   # step t-2 has finished reading this set's inputs
+            compute.wait_event(self.copied_out[i])      # and copied this set's outputs out
+        with torch.cuda.stream(self.copy_in):
+            buf["q"].copy_(q_host, non_blocking=True)
+            buf["k"].copy_(k_host, non_blocking=True)
+            buf["v"].copy_(v_host, non_blocking=True)
+            self.inputs_ready[i].record(self.copy_in)
+        compute.wait_event(self.inputs_ready[i])
+        plan.prepare(compute)
+        plsh_attention_fwd(buf["q"], buf["k"], buf["v"], plan.dtype_code, plan.B, plan.H, plan.H_kv, plan.n, plan.d,
+                           plan.sigma_dev, plan.s, plan.table_dev, plan.spans, plan.bmask, int(plan.causal),
+                           buf["O"], buf["R"], plan.err, compute)
+        self.computed[i].record(compute)
+        self.copy_out.wait_event(self.computed[i])
+        with torch.cuda.stream(self.copy_out):
+            o_host.copy_(buf["O"], non_blocking=True)
+            if rs_host is not None:
+                rs_host.copy_(buf["R"], non_blocking=True)
+            self.copied_out[i].record(self.copy_out)
+        self.t += 1
+
+    def wait(self, stream: Optional[torch.cuda.Stream] = None) -> None:
+        """Makes `stream` (default: the current stream) wait for every enqueued step's copy-out."""
+        st = torch.cuda.current_stream() if stream is None else stream
+        for t in range(max(0, self.t - 2), self.t):
+            st.wait_event(self.copied_out[t % 2])
+
+
 def fixed_blocks_table(H: int, block: float) -> np.ndarray:
     """Table of the "fixed blocks" baseline: one hash per head with pitch `block` and offset 0, so
     positions [k*block, (k+1)*block) form the blocks and every row attends inside its own block

@@ -37,11 +37,11 @@ __device__ __forceinline__ int popc_mask(MaskT m) {
 
 __device__ __forceinline__ float to_f(float x) { return x; }
 
-// q . row for one key row (q in shared memory), 16-byte loads.
+// q . row for one key row (q in shared memory), 16-byte loads, all issued before the first FMA.
 template <int D>
 __device__ __forceinline__ float dot_row(const float* q, const float* row) {
   float acc = 0.0f;
-#pragma unroll 4
+#pragma unroll
   for (int e = 0; e < D; e += 4) {
     const float4 k4 = *reinterpret_cast<const float4*>(row + e);
     acc = fmaf(q[e], k4.x, fmaf(q[e + 1], k4.y, fmaf(q[e + 2], k4.z, fmaf(q[e + 3], k4.w, acc))));
@@ -51,7 +51,7 @@ __device__ __forceinline__ float dot_row(const float* q, const float* row) {
 template <int D>
 __device__ __forceinline__ float dot_row(const float* q, const __nv_bfloat16* row) {
   float acc = 0.0f;
-#pragma unroll 2
+#pragma unroll
   for (int e = 0; e < D; e += 8) {
     const uint4 u = *reinterpret_cast<const uint4*>(row + e);
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -151,15 +151,25 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const T* __restrict__ 
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, o);
     lw += psum;
-    // O += p_j V_j over the warp's keys, lanes over dims
-    for (int kk = 0; kk < 32; ++kk) {
-      const float pk = __shfl_sync(0xffffffffu, p, kk);
-      const int jk = __shfl_sync(0xffffffffu, j, kk);
-      if (pk == 0.0f) continue;
-      float vv[DPL];
-      load_n<DPL>(Vh + static_cast<size_t>(jk) * D + lane * DPL, vv);
+    // O += p_j V_j over the warp's keys, lanes over dims; 8 keys at a time, their loads issued together
+#pragma unroll 1
+    for (int k0 = 0; k0 < 32; k0 += 8) {
+      float pk[8], vv[8][DPL];
 #pragma unroll
-      for (int e = 0; e < DPL; ++e) ow[e] = fmaf(pk, vv[e], ow[e]);
+      for (int u = 0; u < 8; ++u) {
+        pk[u] = __shfl_sync(0xffffffffu, p, k0 + u);
+        const int jk = __shfl_sync(0xffffffffu, j, k0 + u);
+        if (pk[u] != 0.0f) {
+          load_n<DPL>(Vh + static_cast<size_t>(jk) * D + lane * DPL, vv[u]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < DPL; ++e) vv[u][e] = 0.0f;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) ow[e] = fmaf(pk[u], vv[u][e], ow[e]);
     }
   };
 

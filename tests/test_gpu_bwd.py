@@ -103,7 +103,8 @@ def test_backward_singleton_bins_give_dv_equal_do():
     bound = 4 * d * 2.0 ** -24 * float(dO.abs().max() * v.abs().max()) * float(max(q.abs().max(), k.abs().max()))
     bound /= d ** 0.5
     assert float(dQ.abs().max()) <= bound and float(dK.abs().max()) <= bound, bound
-    torch.testing.assert_close(dV[:, 0], dO.sum(dim=1), rtol=1e-6, atol=1e-6)
+    # P_ii = exp(S_ii / sqrt d - L_i) = 1 up to the fp32 rounding of the forward's row_sum L_i = S_ii / sqrt d
+    torch.testing.assert_close(dV[:, 0], dO.sum(dim=1), rtol=2e-5, atol=2e-5)
 
 
 def test_backward_headline_sampled():
