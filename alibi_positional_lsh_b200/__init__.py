@@ -70,7 +70,10 @@ def _load() -> ctypes.CDLL:
     lib.plsh_attention_bwd.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, i32, vp, vp,
                                        vp, vp, vp, vp]
     lib.plsh_decode_fwd.restype = i32
-    lib.plsh_decode_fwd.argtypes = [vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, i32, vp, vp, vp, vp]
+    lib.plsh_decode_fwd.argtypes = [vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, i32, vp,
+                                    ctypes.c_size_t, vp, vp, vp, vp]
+    lib.plsh_decode_scratch_bytes.restype = ctypes.c_size_t
+    lib.plsh_decode_scratch_bytes.argtypes = [i32, i32, i32, i32]
     return lib
 
 
@@ -180,12 +183,18 @@ def plsh_alibi_banded_fwd(Q, K, V, dtype: int, B: int, H: int, H_kv: int, n: int
                                       _stream_ptr(stream)))
 
 
+def plsh_decode_scratch_bytes(B: int, H: int, m: int, d: int) -> int:
+    return int(_lib.plsh_decode_scratch_bytes(B, H, m, d))
+
+
 def plsh_decode_fwd(Q, pos_dev, m: int, K, V, dtype: int, B: int, H: int, H_kv: int, n: int, d: int, s: int,
-                    bmask_dev, causal: int, O, row_sum, err_dev, stream=None) -> None:
+                    bmask_dev, causal: int, scratch_dev, O, row_sum, err_dev, stream=None) -> None:
+    nbytes = 0 if scratch_dev is None else scratch_dev.numel() * scratch_dev.element_size()
     _check(_lib.plsh_decode_fwd(_dev_ptr(Q, "Q"), _dev_ptr(pos_dev, "pos_dev"), m, _dev_ptr(K, "K"),
                                 _dev_ptr(V, "V"), dtype, B, H, H_kv, n, d, s, _dev_ptr(bmask_dev, "bmask_dev"),
-                                int(causal), _dev_ptr(O, "O"), _dev_ptr(row_sum, "row_sum"),
-                                _dev_ptr(err_dev, "err_dev"), _stream_ptr(stream)))
+                                int(causal), _dev_ptr(scratch_dev, "scratch_dev"), ctypes.c_size_t(nbytes),
+                                _dev_ptr(O, "O"), _dev_ptr(row_sum, "row_sum"), _dev_ptr(err_dev, "err_dev"),
+                                _stream_ptr(stream)))
 
 
 def plsh_attention_bwd(Q, K, V, O, dO, row_sum, dtype: int, B: int, H: int, H_kv: int, n: int, d: int, s: int,

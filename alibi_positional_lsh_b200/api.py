@@ -20,7 +20,8 @@ import numpy as np
 import torch
 
 from . import (PLSH_BF16, PLSH_F32, PLSH_TILE, PlshError, decode_device_error, plsh_alibi_banded_fwd,
-               plsh_attention_bwd, plsh_attention_fwd, plsh_attention_varlen_fwd, plsh_decode_fwd, plsh_draw_table, plsh_sample_bins,
+               plsh_attention_bwd, plsh_attention_fwd, plsh_attention_varlen_fwd, plsh_decode_fwd,
+               plsh_decode_scratch_bytes, plsh_draw_table, plsh_sample_bins,
                plsh_varlen_scratch_bytes, plsh_window)
 
 
@@ -56,6 +57,7 @@ class PlshForward:
         self.row_sum = torch.empty((B, H, n), dtype=torch.float32, device=dev)
         self.scratch = None  # per-hash windows of the comparator, allocated on first use
         self.grads = None    # (delta, dQ, dK, dV) of backward(), allocated on first use
+        self.decode_scratch = None  # partial results of decode(), grown on demand
 
     # a1 + a2 + a3
     def prepare(self, stream: Optional[torch.cuda.Stream] = None, table: Optional[np.ndarray] = None) -> None:
@@ -161,9 +163,12 @@ class PlshForward:
                 raise ValueError(f"{nm} must be {self.dtype} on {self.O.device}")
         O = torch.empty((B, H, m, d), dtype=self.dtype, device=self.O.device)
         R = torch.empty((B, H, m), dtype=torch.float32, device=self.O.device)
+        need = plsh_decode_scratch_bytes(B, H, m, d)
+        if self.decode_scratch is None or self.decode_scratch.numel() * 4 < need:
+            self.decode_scratch = torch.empty((need // 4,), dtype=torch.float32, device=self.O.device)
         st = torch.cuda.current_stream() if stream is None else stream
         plsh_decode_fwd(q_rows, pos, m, k, v, self.dtype_code, B, H, H_kv, n, d, self.s, self.bmask,
-                        int(self.causal), O, R, self.err, st)
+                        int(self.causal), self.decode_scratch, O, R, self.err, st)
         return O, R
 
     def __call__(self, q, k, v, stream=None, table=None):

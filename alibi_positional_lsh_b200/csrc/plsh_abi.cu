@@ -241,16 +241,28 @@ extern "C" int plsh_alibi_banded_fwd(const void* Q, const void* K, const void* V
 
 // ---------------------------------------------------------------- decode
 
+extern "C" size_t plsh_decode_scratch_bytes(int B, int H, int m, int d) {
+  if (B < 1 || H < 1 || m < 1 || d < 1) return 0;
+  return sizeof(float) * static_cast<size_t>(B) * H * m * plsh::kDecodeMaxSplit * (static_cast<size_t>(d) + 2);
+}
+
 extern "C" int plsh_decode_fwd(const void* Q, const int32_t* pos_dev, int m, const void* K, const void* V, int dtype,
                                int B, int H, int H_kv, int n, int d, int s, const void* bmask_dev, int causal,
-                               void* O, float* row_sum, uint32_t* err_dev, void* stream) {
+                               void* scratch_dev, size_t scratch_bytes, void* O, float* row_sum, uint32_t* err_dev,
+                               void* stream) {
   const char* fn = "plsh_decode_fwd";
   if (int rc = plsh::check_attention(fn, Q, K, V, dtype, B, H, H_kv, n, d, s, causal, bmask_dev, O, row_sum,
                                      err_dev))
     return rc;
   if (m < 1) return fail(PLSH_ERR_INVALID_ARG, "%s: need m >= 1 (m=%d)", fn, m);
-  if (!pos_dev) return fail(PLSH_ERR_INVALID_ARG, "%s: null pointer", fn);
-  plsh::DecodeArgs a{Q, pos_dev, m, K, V, dtype, B, H, H_kv, n, d, s, causal, bmask_dev, O, row_sum, err_dev};
+  if (!pos_dev || !scratch_dev) return fail(PLSH_ERR_INVALID_ARG, "%s: null pointer", fn);
+  if (static_cast<size_t>(m) * plsh::kDecodeMaxSplit > (size_t{1} << 31) - 1)
+    return fail(PLSH_ERR_RANGE, "%s: m=%d too large", fn, m);
+  const size_t need = plsh_decode_scratch_bytes(B, H, m, d);
+  if (scratch_bytes < need)
+    return fail(PLSH_ERR_INVALID_ARG, "%s: scratch holds %zu bytes, %zu needed", fn, scratch_bytes, need);
+  plsh::DecodeArgs a{Q, pos_dev, m, K, V, dtype, B, H, H_kv, n, d, s, causal, bmask_dev, O, row_sum, err_dev,
+                     static_cast<float*>(scratch_dev)};
   return plsh::launch_decode(a, static_cast<cudaStream_t>(stream));
 }
 

@@ -10,13 +10,17 @@
 // of keys whose counts are all zero. Only the keys sharing a block with i in
 // some hash are read, so the kernel is bound by reading their K and V rows.
 //
-// One CTA of 256 threads per (b, h, t). Keys are taken in chunks of 256 on
-// each side of i (i and below, then above when not causal): thread k of the
-// CTA owns key i - k (below) or i + 1 + k (above) of the chunk; a CTA-wide
-// OR-scan of the boundary masks gives every key its count. Each warp then
+// Each query row's walk is spread over G CTAs of 256 threads (G chosen so the
+// grid covers the SMs about twice, at most 8). Keys are taken in chunks of 256
+// on each side of i (i and below, then above when not causal); CTA g of a row
+// takes chunks g, g + G, g + 2G, ... Its carry -- the OR of the masks between
+// i and its chunk -- is OR-reduced from the masks of the chunks in between,
+// and a CTA-wide OR-scan inside the chunk gives every key its count. Each warp
 // scores its 32 keys (lane = key, q from shared memory), keeps a running
-// maximum, sum and 128-wide output (lane = 4 dims), and the 8 warps are
-// merged at the end.
+// maximum, sum and output row (lanes over dims), and the CTA writes the merge
+// of its warps as a partial result (maximum, sum, unnormalised row) to caller
+// scratch. decode_combine_kernel then merges each row's G partials.
+#include <algorithm>
 #include <cmath>
 
 #include <cuda_bf16.h>
@@ -93,32 +97,73 @@ __device__ __forceinline__ void from_f(__nv_bfloat16& y, float x) { y = __float2
 template <typename T, int D, typename MaskT>
 struct DecodeSmem {
   float q[D];
-  MaskT wsum[kWarps];          // OR of each warp's masks in the current chunk
+  MaskT wsum[kWarps];          // OR of each warp's masks
   float wm[kWarps], wl[kWarps];
   float wo[kWarps][D];
   int live;                    // some key of the chunk carries weight
 };
 
+// The mask the walk's key at offset kk from i contributes on `side` (0: i and below, 1: above), and
+// that key. Below, key j needs the masks over (j, i], i.e. bm[j + 1 .. i] (none for j = i, which has
+// count s); above, over (i, j], bm[i + 1 .. j]. Keys outside [0, n) contribute every hash.
+template <typename MaskT>
+__device__ __forceinline__ MaskT walk_mask(const MaskT* bm, int i, int n, int side, int kk, MaskT full, int& j,
+                                           bool& in) {
+  j = side == 0 ? i - kk : i + 1 + kk;
+  in = j >= 0 && j < n;
+  return !in ? full : side == 1 ? bm[j] : j == i ? static_cast<MaskT>(0) : bm[j + 1];
+}
+
+// OR of v over the CTA (every thread gets it).
+template <typename MaskT>
+__device__ __forceinline__ MaskT cta_or(MaskT v, MaskT* wsum, int lane, int warp) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v |= __shfl_xor_sync(0xffffffffu, v, o);
+  if (lane == 0) wsum[warp] = v;
+  __syncthreads();
+  MaskT all = 0;
+#pragma unroll
+  for (int w2 = 0; w2 < kWarps; ++w2) all |= wsum[w2];
+  __syncthreads();
+  return all;
+}
+
+// OR of the walk masks at offsets [k0, k1) on `side`.
+template <typename MaskT>
+__device__ __forceinline__ MaskT walk_or(const MaskT* bm, int i, int n, int side, int k0, int k1, MaskT full,
+                                         MaskT* wsum, int lane, int warp) {
+  MaskT acc = 0;
+#pragma unroll 8
+  for (int kk = k0 + static_cast<int>(threadIdx.x); kk < k1; kk += kThreads) {
+    int j;
+    bool in;
+    acc |= walk_mask(bm, i, n, side, kk, full, j, in);
+  }
+  return cta_or(acc, wsum, lane, warp);
+}
+
+// One of G CTAs of query row t of (b, h): the chunks g, g + G, g + 2G, ... of each side's walk. Its
+// partial result -- running maximum, sum and unnormalised output row -- goes to part.
 template <typename T, int D, typename MaskT>
-__global__ void __launch_bounds__(kThreads) decode_kernel(const T* __restrict__ Q, const int32_t* __restrict__ pos,
-                                                          int m, const T* __restrict__ K, const T* __restrict__ V,
-                                                          int H, int H_kv, int n, int s, int causal,
-                                                          const MaskT* __restrict__ bmask, T* __restrict__ O,
-                                                          float* __restrict__ row_sum, uint32_t* __restrict__ err) {
+__global__ void __launch_bounds__(kThreads) decode_partial_kernel(
+    const T* __restrict__ Q, const int32_t* __restrict__ pos, int m, const T* __restrict__ K,
+    const T* __restrict__ V, int H, int H_kv, int n, int s, int causal, const MaskT* __restrict__ bmask, int G,
+    float* __restrict__ part, uint32_t* __restrict__ err) {
   constexpr int DPL = D / 32;  // output dims per lane
   __shared__ DecodeSmem<T, D, MaskT> sm;
-  const int t = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int t = blockIdx.x / G, g = blockIdx.x % G, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int i = pos[t];
   if (i < 0 || i >= n) {
-    if (tid == 0) atomicOr(err, PLSH_DEVERR_POSITION);
+    if (tid == 0 && g == 0) atomicOr(err, PLSH_DEVERR_POSITION);
     return;
   }
   const int kvh = h / (H / H_kv);
   const MaskT FULL = (s >= static_cast<int>(8 * sizeof(MaskT))) ? static_cast<MaskT>(~static_cast<MaskT>(0))
                                                               : static_cast<MaskT>((static_cast<MaskT>(1) << s) - 1);
   const MaskT* bm = bmask + static_cast<size_t>(h) * n;
-  const T* qrow = Q + ((static_cast<size_t>(b) * H + h) * m + t) * D;
+  const size_t row = (static_cast<size_t>(b) * H + h) * m + t;
+  const T* qrow = Q + row * D;
   for (int e = tid; e < D; e += kThreads) sm.q[e] = to_f(qrow[e]);
   const T* Kh = K + (static_cast<size_t>(b) * H_kv + kvh) * static_cast<size_t>(n) * D;
   const T* Vh = V + (static_cast<size_t>(b) * H_kv + kvh) * static_cast<size_t>(n) * D;
@@ -151,12 +196,12 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const T* __restrict__ 
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, o);
     lw += psum;
-    // O += p_j V_j over the warp's keys, lanes over dims; 8 keys at a time, their loads issued together
+    // O += p_j V_j over the warp's keys, lanes over dims; 16 keys at a time, their loads issued together
 #pragma unroll 1
-    for (int k0 = 0; k0 < 32; k0 += 8) {
-      float pk[8], vv[8][DPL];
+    for (int k0 = 0; k0 < 32; k0 += 16) {
+      float pk[16], vv[16][DPL];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < 16; ++u) {
         pk[u] = __shfl_sync(0xffffffffu, p, k0 + u);
         const int jk = __shfl_sync(0xffffffffu, j, k0 + u);
         if (pk[u] != 0.0f) {
@@ -167,21 +212,19 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const T* __restrict__ 
         }
       }
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
+      for (int u = 0; u < 16; ++u)
 #pragma unroll
         for (int e = 0; e < DPL; ++e) ow[e] = fmaf(pk[u], vv[u][e], ow[e]);
     }
   };
 
-  // i and below (j <= i), then above (j > i, non-causal): chunks of kThreads keys walking away from i
   for (int side = 0; side < (causal ? 1 : 2); ++side) {
-    MaskT carry = 0;  // OR of the masks between i and the chunk's nearest key
-    for (int base = 0;; base += kThreads) {
-      const int j = side == 0 ? i - base - tid : i + 1 + base + tid;
-      const bool in = j >= 0 && j < n;
-      // below: key j needs the masks over (j, i], i.e. bm[j + 1 .. i] (none for j = i, which has count s);
-      // above: over (i, j], bm[i + 1 .. j]
-      const MaskT mine = !in ? FULL : side == 1 ? bm[j] : j == i ? static_cast<MaskT>(0) : bm[j + 1];
+    // OR of the masks between i and the nearest key of chunk g
+    MaskT carry = walk_or(bm, i, n, side, 0, g * kThreads, FULL, sm.wsum, lane, warp);
+    for (int c = g; carry != FULL; c += G) {   // a carry holding every hash leaves no key any weight
+      int j;
+      bool in;
+      const MaskT mine = walk_mask(bm, i, n, side, c * kThreads + tid, FULL, j, in);
       // inclusive OR-scan over the CTA in walking order
       MaskT v = mine;
 #pragma unroll
@@ -196,20 +239,21 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const T* __restrict__ 
       MaskT all = carry;
       for (int w2 = 0; w2 < kWarps; ++w2) all |= sm.wsum[w2];
       const MaskT R = before | v;
-      const int c = in ? s - popc_mask(R) : 0;
+      const int cnt = in ? s - popc_mask(R) : 0;
       if (tid == 0) sm.live = 0;
       __syncthreads();
-      if (c > 0) sm.live = 1;
+      if (cnt > 0) sm.live = 1;
       __syncthreads();
       const bool live = sm.live != 0;
       __syncthreads();
-      if (!live) break;
-      fold(j, c);
-      carry = all;
+      if (!live) break;   // the OR only grows along the walk: no later key has weight
+      fold(j, cnt);
+      // through chunk c, then the chunks the other CTAs of the row take before chunk c + G
+      carry = all | walk_or(bm, i, n, side, (c + 1) * kThreads, (c + G) * kThreads, FULL, sm.wsum, lane, warp);
     }
   }
 
-  // merge the warps
+  // merge the warps into the CTA's partial result
   if (lane == 0) {
     sm.wm[warp] = mw;
     sm.wl[warp] = lw;
@@ -230,35 +274,81 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const T* __restrict__ 
 #pragma unroll
       for (int e = 0; e < DPL; ++e) ot[e] += sm.wo[w2][lane * DPL + e] * f;
     }
-    const float inv = 1.0f / lt;
-    T* orow = O + ((static_cast<size_t>(b) * H + h) * m + t) * D;
+    float* pr = part + (row * G + g) * (D + 2);
 #pragma unroll
-    for (int e = 0; e < DPL; ++e) from_f(orow[lane * DPL + e], ot[e] * inv);
-    if (lane == 0) row_sum[(static_cast<size_t>(b) * H + h) * m + t] = logf(lt) + mt - logf(static_cast<float>(s));
+    for (int e = 0; e < DPL; ++e) pr[2 + lane * DPL + e] = ot[e];
+    if (lane == 0) {
+      pr[0] = mt;
+      pr[1] = lt;
+    }
   }
 }
 
+// One warp per query row: merges the row's G partial results into O and row_sum.
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads) decode_combine_kernel(const float* __restrict__ part,
+                                                                  const int32_t* __restrict__ pos, int m, int n,
+                                                                  int s, int G, size_t rows, T* __restrict__ O,
+                                                                  float* __restrict__ row_sum) {
+  constexpr int DPL = D / 32;
+  const size_t row = static_cast<size_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const int i = pos[row % m];
+  if (i < 0 || i >= n) return;   // reported by the partial kernel; the row stays unwritten
+  const float* pr = part + row * G * (D + 2);
+  float mt = -INFINITY;
+  for (int g = 0; g < G; ++g) mt = fmaxf(mt, pr[g * (D + 2)]);
+  float lt = 0.0f, ot[DPL];
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) ot[e] = 0.0f;
+  for (int g = 0; g < G; ++g) {
+    const float* q = pr + g * (D + 2);
+    if (q[0] == -INFINITY) continue;
+    const float f = expf(q[0] - mt);
+    lt += q[1] * f;
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) ot[e] += q[2 + lane * DPL + e] * f;
+  }
+  const float inv = 1.0f / lt;
+  T* orow = O + row * D;
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) from_f(orow[lane * DPL + e], ot[e] * inv);
+  if (lane == 0) row_sum[row] = logf(lt) + mt - logf(static_cast<float>(s));
+}
+
 template <typename T, int D, typename MaskT>
-int launch_decode_typed(const DecodeArgs& a, cudaStream_t st) {
-  dim3 grid(a.m, a.H, a.B);
-  decode_kernel<T, D, MaskT><<<grid, kThreads, 0, st>>>(
+int launch_decode_typed(const DecodeArgs& a, int G, cudaStream_t st) {
+  decode_partial_kernel<T, D, MaskT><<<dim3(a.m * G, a.H, a.B), kThreads, 0, st>>>(
       static_cast<const T*>(a.Q), a.pos, a.m, static_cast<const T*>(a.K), static_cast<const T*>(a.V), a.H, a.H_kv,
-      a.n, a.s, a.causal, static_cast<const MaskT*>(a.bmask), static_cast<T*>(a.O), a.row_sum, a.err);
-  const cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? PLSH_OK : cuda_fail(e, "decode_kernel launch");
+      a.n, a.s, a.causal, static_cast<const MaskT*>(a.bmask), G, a.part, a.err);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "decode_partial_kernel launch");
+  const size_t rows = static_cast<size_t>(a.B) * a.H * a.m;
+  decode_combine_kernel<T, D><<<static_cast<unsigned>((rows + kWarps - 1) / kWarps), kThreads, 0, st>>>(
+      a.part, a.pos, a.m, a.n, a.s, G, rows, static_cast<T*>(a.O), a.row_sum);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? PLSH_OK : cuda_fail(e, "decode_combine_kernel launch");
 }
 
 template <typename T, int D>
-int launch_decode_mask(const DecodeArgs& a, cudaStream_t st) {
-  return a.s <= 32 ? launch_decode_typed<T, D, uint32_t>(a, st) : launch_decode_typed<T, D, unsigned long long>(a, st);
+int launch_decode_mask(const DecodeArgs& a, int G, cudaStream_t st) {
+  return a.s <= 32 ? launch_decode_typed<T, D, uint32_t>(a, G, st)
+                   : launch_decode_typed<T, D, unsigned long long>(a, G, st);
 }
 
 }  // namespace
 
 int launch_decode(const DecodeArgs& a, cudaStream_t st) {
+  // CTAs per row: enough for about two CTAs per SM over all rows, at most kDecodeMaxSplit
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    sms = 148;
+  const long long rows = static_cast<long long>(a.B) * a.H * a.m;
+  const int G = static_cast<int>(std::min<long long>(kDecodeMaxSplit, std::max<long long>(1, (2LL * sms + rows - 1) / rows)));
   if (a.dtype == PLSH_F32)
-    return a.d == 64 ? launch_decode_mask<float, 64>(a, st) : launch_decode_mask<float, 128>(a, st);
-  return a.d == 64 ? launch_decode_mask<__nv_bfloat16, 64>(a, st) : launch_decode_mask<__nv_bfloat16, 128>(a, st);
+    return a.d == 64 ? launch_decode_mask<float, 64>(a, G, st) : launch_decode_mask<float, 128>(a, G, st);
+  return a.d == 64 ? launch_decode_mask<__nv_bfloat16, 64>(a, G, st) : launch_decode_mask<__nv_bfloat16, 128>(a, G, st);
 }
 
 }  // namespace plsh

@@ -38,12 +38,15 @@ struct AttnArgs {
   double log_inv_eps;
 };
 // Decode: query rows Q [B][H][m][d] at positions pos [m] against K, V [B][H_kv][n][d].
+// part: caller scratch of B*H*m*kDecodeMaxSplit*(d+2) floats for the per-CTA partial results.
+constexpr int kDecodeMaxSplit = 8;
 struct DecodeArgs {
   const void* Q; const int32_t* pos; int m;
   const void* K; const void* V;
   int dtype, B, H, H_kv, n, d, s, causal;
   const void* bmask;
   void* O; float* row_sum; uint32_t* err;
+  float* part;
 };
 int launch_decode(const DecodeArgs& a, cudaStream_t st);
 // Backward: dQ, dK, dV of T~ (Q, O, dO, dQ [B][H][n][d]; K, V, dK, dV [B][H_kv][n][d]).

@@ -299,12 +299,24 @@ PLSH_API int plsh_alibi_banded_fwd(const void* Q, const void* K, const void* V, 
  *   dtype, d, s, causal, bmask_dev, err_dev   as plsh_attention_fwd; the
  *              masks are plsh_window's for this n (with causal, only the
  *              entries at positions <= max(pos) are read).
+ *   scratch_dev    device scratch for the partial results of the CTAs that
+ *                  share a row's walk (up to 8 per row), nothing needs to be
+ *                  zero; scratch_bytes its size, at least
+ *                  plsh_decode_scratch_bytes(B, H, m, d), else
+ *                  PLSH_ERR_INVALID_ARG.
  *   row_sum    [B][H][m] float32 out.
  * Q, K, V and O must be 16-byte aligned.
  */
 PLSH_API int plsh_decode_fwd(const void* Q, const int32_t* pos_dev, int m, const void* K, const void* V, int dtype,
                              int B, int H, int H_kv, int n, int d, int s, const void* bmask_dev, int causal,
-                             void* O, float* row_sum, uint32_t* err_dev, void* stream);
+                             void* scratch_dev, size_t scratch_bytes, void* O, float* row_sum, uint32_t* err_dev,
+                             void* stream);
+
+/*
+ * plsh_decode_scratch_bytes -- bytes of scratch plsh_decode_fwd needs:
+ * 4 * B * H * m * 8 * (d + 2). Returns 0 for a non-positive size.
+ */
+PLSH_API size_t plsh_decode_scratch_bytes(int B, int H, int m, int d);
 
 /*
  * plsh_attention_bwd -- gradients of T~ for training: dQ, dK, dV of
