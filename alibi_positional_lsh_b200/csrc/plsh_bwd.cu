@@ -35,7 +35,14 @@ namespace {
 
 constexpr int kT = 64;          // rows per query tile and keys per key tile
 constexpr int kThreads = 256;   // 16 x 16 threads; each owns 4 x 4 (row, key) pairs
-constexpr int kSP = kT + 1;     // padded pitch of the 64 x 64 score tiles
+constexpr int kSP = kT + 4;     // pitch of the 64 x 64 score tiles (16-byte rows, spread over the banks)
+template <int D>
+__host__ __device__ constexpr int pitch() { return D + 4; }   // pitch of the 64 x D row tiles (16-byte rows)
+
+__device__ __forceinline__ float4 lds4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ float comp(const float4& v, int u) {
+  return u == 0 ? v.x : (u == 1 ? v.y : (u == 2 ? v.z : v.w));
+}
 
 __device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
 __device__ __forceinline__ float4 ld4(const __nv_bfloat16* p) {
@@ -46,7 +53,7 @@ __device__ __forceinline__ float4 ld4(const __nv_bfloat16* p) {
 __device__ __forceinline__ void st1(float* p, float x) { *p = x; }
 __device__ __forceinline__ void st1(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
 
-// rows [r0, r0 + 64) of a [n][D] matrix into fp32 shared memory of pitch D + 1 (zeros past `last`)
+// rows [r0, r0 + 64) of a [n][D] matrix into fp32 shared memory of pitch D + 4 (zeros past `last`)
 template <typename T, int D>
 __device__ __forceinline__ void load_rows(float* dst, const T* src, int r0, int last) {
   constexpr int F4 = D / 4;
@@ -54,8 +61,7 @@ __device__ __forceinline__ void load_rows(float* dst, const T* src, int r0, int 
     const int r = x / F4, c = (x % F4) * 4;
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
     if (r0 + r <= last) v = ld4(src + static_cast<size_t>(r0 + r) * D + c);
-    float* o = dst + r * (D + 1) + c;
-    o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+    *reinterpret_cast<float4*>(dst + r * pitch<D>() + c) = v;
   }
 }
 
@@ -90,34 +96,37 @@ __device__ __forceinline__ void block_range(int* range, const int32_t* ids_h, in
   atomicMax(&range[1], lo);
 }
 
-// S = q k^T and dP = dO v^T for the thread's 4 x 4 pairs (rows ty + 16a, keys tx + 16b)
+// S = q k^T and dP = dO v^T for the thread's 4 x 4 pairs (rows ty + 16a, keys tx + 16b), four
+// dims per step through 16-byte shared loads
 template <int D>
 __device__ __forceinline__ void scores(const float* qs, const float* dos, const float* ks, const float* vs,
                                        int ty, int tx, float (&sacc)[4][4], float (&pacc)[4][4]) {
-  constexpr int P = D + 1;
+  constexpr int P = pitch<D>();
 #pragma unroll
   for (int a = 0; a < 4; ++a)
 #pragma unroll
     for (int b = 0; b < 4; ++b) sacc[a][b] = pacc[a][b] = 0.0f;
-#pragma unroll 4
-  for (int e = 0; e < D; ++e) {
-    float qa[4], oa[4], kb[4], vb[4];
+#pragma unroll 2
+  for (int e = 0; e < D; e += 4) {
+    float4 qa[4], oa[4], kb[4], vb[4];
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
-      qa[a] = qs[(ty + 16 * a) * P + e];
-      oa[a] = dos[(ty + 16 * a) * P + e];
+      qa[a] = lds4(qs + (ty + 16 * a) * P + e);
+      oa[a] = lds4(dos + (ty + 16 * a) * P + e);
     }
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
-      kb[b] = ks[(tx + 16 * b) * P + e];
-      vb[b] = vs[(tx + 16 * b) * P + e];
+      kb[b] = lds4(ks + (tx + 16 * b) * P + e);
+      vb[b] = lds4(vs + (tx + 16 * b) * P + e);
     }
 #pragma unroll
     for (int a = 0; a < 4; ++a)
 #pragma unroll
       for (int b = 0; b < 4; ++b) {
-        sacc[a][b] = fmaf(qa[a], kb[b], sacc[a][b]);
-        pacc[a][b] = fmaf(oa[a], vb[b], pacc[a][b]);
+        sacc[a][b] = fmaf(qa[a].x, kb[b].x, fmaf(qa[a].y, kb[b].y, fmaf(qa[a].z, kb[b].z, fmaf(qa[a].w, kb[b].w,
+                          sacc[a][b]))));
+        pacc[a][b] = fmaf(oa[a].x, vb[b].x, fmaf(oa[a].y, vb[b].y, fmaf(oa[a].z, vb[b].z, fmaf(oa[a].w, vb[b].w,
+                          pacc[a][b]))));
       }
   }
 }
@@ -162,9 +171,9 @@ struct BwdParams {
 };
 
 template <int D>
-constexpr size_t dq_smem_floats() { return 4 * kT * (D + 1) + kT * kSP + 2 * kT; }
+__host__ __device__ constexpr size_t dq_smem_floats() { return 4 * kT * pitch<D>() + kT * kSP + 2 * kT; }
 template <int D>
-constexpr size_t dkdv_smem_floats() { return 4 * kT * (D + 1) + 2 * kT * kSP + 2 * kT; }
+__host__ __device__ constexpr size_t dkdv_smem_floats() { return 4 * kT * pitch<D>() + 2 * kT * kSP + 2 * kT; }
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(const T* __restrict__ Q, const T* __restrict__ K,
@@ -173,8 +182,8 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(const T* __restrict__ 
                                                           const float* __restrict__ delta,
                                                           const int32_t* __restrict__ ids, BwdParams p,
                                                           T* __restrict__ dQ) {
-  constexpr int P = D + 1;
-  constexpr int NB = D / 16;   // output dims per thread
+  constexpr int P = pitch<D>();
+  constexpr int NB = D / 16;   // output dims per thread: tx * NB .. tx * NB + NB - 1
   extern __shared__ __align__(16) float smf[];
   float* qs = smf;
   float* dos = qs + kT * P;
@@ -244,26 +253,37 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(const T* __restrict__ 
       }
     }
     __syncthreads();
-#pragma unroll 4
-    for (int j = 0; j < kT; ++j) {
-      float dv[4], kv[NB];
+#pragma unroll 1
+    for (int j = 0; j < kT; j += 4) {
+      float4 dv[4];
 #pragma unroll
-      for (int a = 0; a < 4; ++a) dv[a] = ds[(ty + 16 * a) * kSP + j];
+      for (int a = 0; a < 4; ++a) dv[a] = lds4(ds + (ty + 16 * a) * kSP + j);
 #pragma unroll
-      for (int c = 0; c < NB; ++c) kv[c] = ks[j * P + tx + 16 * c];
+      for (int u = 0; u < 4; ++u) {
+        float4 kv[NB / 4];
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
+        for (int c4 = 0; c4 < NB / 4; ++c4) kv[c4] = lds4(ks + (j + u) * P + tx * NB + 4 * c4);
 #pragma unroll
-        for (int c = 0; c < NB; ++c) acc[a][c] = fmaf(dv[a], kv[c], acc[a][c]);
+        for (int a = 0; a < 4; ++a) {
+          const float w = comp(dv[a], u);
+#pragma unroll
+          for (int c4 = 0; c4 < NB / 4; ++c4) {
+            acc[a][4 * c4] = fmaf(w, kv[c4].x, acc[a][4 * c4]);
+            acc[a][4 * c4 + 1] = fmaf(w, kv[c4].y, acc[a][4 * c4 + 1]);
+            acc[a][4 * c4 + 2] = fmaf(w, kv[c4].z, acc[a][4 * c4 + 2]);
+            acc[a][4 * c4 + 3] = fmaf(w, kv[c4].w, acc[a][4 * c4 + 3]);
+          }
+        }
+      }
     }
   }
 #pragma unroll
   for (int a = 0; a < 4; ++a) {
     const int i = r0 + ty + 16 * a;
     if (i > r1) continue;
-    T* out = dQ + (bh * n + i) * D;
+    T* out = dQ + (bh * n + i) * D + tx * NB;
 #pragma unroll
-    for (int c = 0; c < NB; ++c) st1(out + tx + 16 * c, acc[a][c] * scale);
+    for (int c = 0; c < NB; ++c) st1(out + c, acc[a][c] * scale);
   }
 }
 
@@ -274,8 +294,8 @@ __global__ void __launch_bounds__(kThreads) bwd_dkdv_kernel(const T* __restrict_
                                                             const float* __restrict__ delta,
                                                             const int32_t* __restrict__ ids, BwdParams p,
                                                             T* __restrict__ dK, T* __restrict__ dV) {
-  constexpr int P = D + 1;
-  constexpr int NB = D / 16;
+  constexpr int P = pitch<D>();
+  constexpr int NB = D / 16;   // output dims per thread: tx * NB .. tx * NB + NB - 1
   extern __shared__ __align__(16) float smf[];
   float* ks = smf;
   float* vs = ks + kT * P;
@@ -345,31 +365,45 @@ __global__ void __launch_bounds__(kThreads) bwd_dkdv_kernel(const T* __restrict_
             pij = static_cast<float>(cnt[a][bb]) * inv_s * expf(sacc[a][bb] * scale - Ls[ty + 16 * a]);
             dsv = pij * (pacc[a][bb] - Ds[ty + 16 * a]);
           }
-          ps[(ty + 16 * a) * kSP + tx + 16 * bb] = pij;
-          dss[(ty + 16 * a) * kSP + tx + 16 * bb] = dsv;
+          // transposed, [key][row], so that a key's 4 consecutive rows are one 16-byte load
+          ps[(tx + 16 * bb) * kSP + ty + 16 * a] = pij;
+          dss[(tx + 16 * bb) * kSP + ty + 16 * a] = dsv;
         }
       }
       __syncthreads();
-#pragma unroll 2
-      for (int i = 0; i < kT; ++i) {
-        float pv[4], dv[4], ov[NB], qv[NB];
+      // keys ty + 16a of the tile, dims tx * NB ..: four query rows per step
+#pragma unroll 1
+      for (int i = 0; i < kT; i += 4) {
+        float4 pv[4], dv[4];
 #pragma unroll
         for (int a = 0; a < 4; ++a) {
-          pv[a] = ps[i * kSP + ty + 16 * a];
-          dv[a] = dss[i * kSP + ty + 16 * a];
+          pv[a] = lds4(ps + (ty + 16 * a) * kSP + i);
+          dv[a] = lds4(dss + (ty + 16 * a) * kSP + i);
         }
 #pragma unroll
-        for (int c = 0; c < NB; ++c) {
-          ov[c] = dos[i * P + tx + 16 * c];
-          qv[c] = qs[i * P + tx + 16 * c];
-        }
+        for (int u = 0; u < 4; ++u) {
+          float4 ov[NB / 4], qv[NB / 4];
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-          for (int c = 0; c < NB; ++c) {
-            accV[a][c] = fmaf(pv[a], ov[c], accV[a][c]);
-            accK[a][c] = fmaf(dv[a], qv[c], accK[a][c]);
+          for (int c4 = 0; c4 < NB / 4; ++c4) {
+            ov[c4] = lds4(dos + (i + u) * P + tx * NB + 4 * c4);
+            qv[c4] = lds4(qs + (i + u) * P + tx * NB + 4 * c4);
           }
+#pragma unroll
+          for (int a = 0; a < 4; ++a) {
+            const float wp = comp(pv[a], u), wd = comp(dv[a], u);
+#pragma unroll
+            for (int c4 = 0; c4 < NB / 4; ++c4) {
+              accV[a][4 * c4] = fmaf(wp, ov[c4].x, accV[a][4 * c4]);
+              accV[a][4 * c4 + 1] = fmaf(wp, ov[c4].y, accV[a][4 * c4 + 1]);
+              accV[a][4 * c4 + 2] = fmaf(wp, ov[c4].z, accV[a][4 * c4 + 2]);
+              accV[a][4 * c4 + 3] = fmaf(wp, ov[c4].w, accV[a][4 * c4 + 3]);
+              accK[a][4 * c4] = fmaf(wd, qv[c4].x, accK[a][4 * c4]);
+              accK[a][4 * c4 + 1] = fmaf(wd, qv[c4].y, accK[a][4 * c4 + 1]);
+              accK[a][4 * c4 + 2] = fmaf(wd, qv[c4].z, accK[a][4 * c4 + 2]);
+              accK[a][4 * c4 + 3] = fmaf(wd, qv[c4].w, accK[a][4 * c4 + 3]);
+            }
+          }
+        }
       }
     }
   }
@@ -377,12 +411,12 @@ __global__ void __launch_bounds__(kThreads) bwd_dkdv_kernel(const T* __restrict_
   for (int a = 0; a < 4; ++a) {
     const int j = j0 + ty + 16 * a;
     if (j > j1) continue;
-    T* ok = dK + (bg * n + j) * D;
-    T* ov = dV + (bg * n + j) * D;
+    T* ok = dK + (bg * n + j) * D + tx * NB;
+    T* ov = dV + (bg * n + j) * D + tx * NB;
 #pragma unroll
     for (int c = 0; c < NB; ++c) {
-      st1(ok + tx + 16 * c, accK[a][c] * scale);
-      st1(ov + tx + 16 * c, accV[a][c]);
+      st1(ok + c, accK[a][c] * scale);
+      st1(ov + c, accV[a][c]);
     }
   }
 }
