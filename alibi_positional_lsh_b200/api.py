@@ -165,7 +165,8 @@ class PlshForward:
         R = torch.empty((B, H, m), dtype=torch.float32, device=self.O.device)
         need = plsh_decode_scratch_bytes(B, H, m, d)
         if self.decode_scratch is None or self.decode_scratch.numel() * 4 < need:
-            self.decode_scratch = torch.empty((need // 4,), dtype=torch.float32, device=self.O.device)
+            # zero once: the per-row counters at its end must start at zero (every call leaves them so)
+            self.decode_scratch = torch.zeros((need // 4,), dtype=torch.float32, device=self.O.device)
         st = torch.cuda.current_stream() if stream is None else stream
         plsh_decode_fwd(q_rows, pos, m, k, v, self.dtype_code, B, H, H_kv, n, d, self.s, self.bmask,
                         int(self.causal), self.decode_scratch, O, R, self.err, st)

@@ -19,7 +19,9 @@
 // scores its 32 keys (lane = key, q from shared memory), keeps a running
 // maximum, sum and output row (lanes over dims), and the CTA writes the merge
 // of its warps as a partial result (maximum, sum, unnormalised row) to caller
-// scratch. decode_combine_kernel then merges each row's G partials.
+// scratch. The last of a row's G CTAs to finish (a ticket from a per-row
+// counter in the same scratch) merges the G partials into O and row_sum and
+// resets the counter.
 #include <algorithm>
 #include <cmath>
 
@@ -148,7 +150,8 @@ template <typename T, int D, typename MaskT>
 __global__ void __launch_bounds__(kThreads) decode_partial_kernel(
     const T* __restrict__ Q, const int32_t* __restrict__ pos, int m, const T* __restrict__ K,
     const T* __restrict__ V, int H, int H_kv, int n, int s, int causal, const MaskT* __restrict__ bmask, int G,
-    float* __restrict__ part, uint32_t* __restrict__ err) {
+    float* __restrict__ part, unsigned* __restrict__ done, T* __restrict__ O, float* __restrict__ row_sum,
+    uint32_t* __restrict__ err) {
   constexpr int DPL = D / 32;  // output dims per lane
   __shared__ DecodeSmem<T, D, MaskT> sm;
   const int t = blockIdx.x / G, g = blockIdx.x % G, h = blockIdx.y, b = blockIdx.z;
@@ -281,54 +284,52 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(
       pr[0] = mt;
       pr[1] = lt;
     }
+    // the row's last CTA to finish merges the G partial results (the others' writes are visible to it
+    // once its ticket shows they have all been published) and leaves the row's counter at zero again
+    __threadfence();
+    __syncwarp();
+    unsigned ticket = 0;
+    if (lane == 0) ticket = atomicAdd(&done[row], 1u);
+    ticket = __shfl_sync(0xffffffffu, ticket, 0);
+    if (ticket == static_cast<unsigned>(G - 1)) {
+      __threadfence();
+      const float* p0 = part + row * G * (D + 2);
+      float M = -INFINITY;
+      for (int g2 = 0; g2 < G; ++g2) M = fmaxf(M, __ldcg(p0 + g2 * (D + 2)));
+      float L = 0.0f, acc[DPL];
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) acc[e] = 0.0f;
+      for (int g2 = 0; g2 < G; ++g2) {
+        const float* q2 = p0 + g2 * (D + 2);
+        const float m2 = __ldcg(q2);
+        if (m2 == -INFINITY) continue;
+        const float f = expf(m2 - M);
+        L += __ldcg(q2 + 1) * f;
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) acc[e] += __ldcg(q2 + 2 + lane * DPL + e) * f;
+      }
+      const float inv = 1.0f / L;
+      T* orow = O + row * D;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) from_f(orow[lane * DPL + e], acc[e] * inv);
+      if (lane == 0) {
+        row_sum[row] = logf(L) + M - logf(static_cast<float>(s));
+        done[row] = 0u;
+      }
+    }
   }
-}
-
-// One warp per query row: merges the row's G partial results into O and row_sum.
-template <typename T, int D>
-__global__ void __launch_bounds__(kThreads) decode_combine_kernel(const float* __restrict__ part,
-                                                                  const int32_t* __restrict__ pos, int m, int n,
-                                                                  int s, int G, size_t rows, T* __restrict__ O,
-                                                                  float* __restrict__ row_sum) {
-  constexpr int DPL = D / 32;
-  const size_t row = static_cast<size_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= rows) return;
-  const int i = pos[row % m];
-  if (i < 0 || i >= n) return;   // reported by the partial kernel; the row stays unwritten
-  const float* pr = part + row * G * (D + 2);
-  float mt = -INFINITY;
-  for (int g = 0; g < G; ++g) mt = fmaxf(mt, pr[g * (D + 2)]);
-  float lt = 0.0f, ot[DPL];
-#pragma unroll
-  for (int e = 0; e < DPL; ++e) ot[e] = 0.0f;
-  for (int g = 0; g < G; ++g) {
-    const float* q = pr + g * (D + 2);
-    if (q[0] == -INFINITY) continue;
-    const float f = expf(q[0] - mt);
-    lt += q[1] * f;
-#pragma unroll
-    for (int e = 0; e < DPL; ++e) ot[e] += q[2 + lane * DPL + e] * f;
-  }
-  const float inv = 1.0f / lt;
-  T* orow = O + row * D;
-#pragma unroll
-  for (int e = 0; e < DPL; ++e) from_f(orow[lane * DPL + e], ot[e] * inv);
-  if (lane == 0) row_sum[row] = logf(lt) + mt - logf(static_cast<float>(s));
 }
 
 template <typename T, int D, typename MaskT>
 int launch_decode_typed(const DecodeArgs& a, int G, cudaStream_t st) {
+  const size_t rows = static_cast<size_t>(a.B) * a.H * a.m;
+  unsigned* done = reinterpret_cast<unsigned*>(a.part + rows * kDecodeMaxSplit * (a.d + 2));
   decode_partial_kernel<T, D, MaskT><<<dim3(a.m * G, a.H, a.B), kThreads, 0, st>>>(
       static_cast<const T*>(a.Q), a.pos, a.m, static_cast<const T*>(a.K), static_cast<const T*>(a.V), a.H, a.H_kv,
-      a.n, a.s, a.causal, static_cast<const MaskT*>(a.bmask), G, a.part, a.err);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "decode_partial_kernel launch");
-  const size_t rows = static_cast<size_t>(a.B) * a.H * a.m;
-  decode_combine_kernel<T, D><<<static_cast<unsigned>((rows + kWarps - 1) / kWarps), kThreads, 0, st>>>(
-      a.part, a.pos, a.m, a.n, a.s, G, rows, static_cast<T*>(a.O), a.row_sum);
-  e = cudaGetLastError();
-  return e == cudaSuccess ? PLSH_OK : cuda_fail(e, "decode_combine_kernel launch");
+      a.n, a.s, a.causal, static_cast<const MaskT*>(a.bmask), G, a.part, done, static_cast<T*>(a.O), a.row_sum,
+      a.err);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? PLSH_OK : cuda_fail(e, "decode_partial_kernel launch");
 }
 
 template <typename T, int D>

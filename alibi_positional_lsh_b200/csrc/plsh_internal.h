@@ -38,7 +38,8 @@ struct AttnArgs {
   double log_inv_eps;
 };
 // Decode: query rows Q [B][H][m][d] at positions pos [m] against K, V [B][H_kv][n][d].
-// part: caller scratch of B*H*m*kDecodeMaxSplit*(d+2) floats for the per-CTA partial results.
+// part: caller scratch of B*H*m*kDecodeMaxSplit*(d+2) floats for the per-CTA partial results, then one
+// unsigned counter per row (zero before the first call; every completed call leaves them zero).
 constexpr int kDecodeMaxSplit = 8;
 struct DecodeArgs {
   const void* Q; const int32_t* pos; int m;

@@ -299,9 +299,13 @@ PLSH_API int plsh_alibi_banded_fwd(const void* Q, const void* K, const void* V, 
  *   dtype, d, s, causal, bmask_dev, err_dev   as plsh_attention_fwd; the
  *              masks are plsh_window's for this n (with causal, only the
  *              entries at positions <= max(pos) are read).
- *   scratch_dev    device scratch for the partial results of the CTAs that
- *                  share a row's walk (up to 8 per row), nothing needs to be
- *                  zero; scratch_bytes its size, at least
+ *   scratch_dev    device scratch: the partial results of the CTAs that
+ *                  share a row's walk (up to 8 per row), then one counter
+ *                  per row. Zero the whole buffer once before its first use
+ *                  (for example with cudaMemsetAsync). Every call that runs
+ *                  to completion leaves the counters at zero again; after a
+ *                  call that did not (a CUDA error), zero it again.
+ *                  scratch_bytes is its size, at least
  *                  plsh_decode_scratch_bytes(B, H, m, d), else
  *                  PLSH_ERR_INVALID_ARG.
  *   row_sum    [B][H][m] float32 out.
@@ -314,7 +318,7 @@ PLSH_API int plsh_decode_fwd(const void* Q, const int32_t* pos_dev, int m, const
 
 /*
  * plsh_decode_scratch_bytes -- bytes of scratch plsh_decode_fwd needs:
- * 4 * B * H * m * 8 * (d + 2). Returns 0 for a non-positive size.
+ * 4 * B * H * m * (8 * (d + 2) + 1). Returns 0 for a non-positive size.
  */
 PLSH_API size_t plsh_decode_scratch_bytes(int B, int H, int m, int d);
 

@@ -101,3 +101,28 @@ def test_decode_position_out_of_range_sets_error_bit():
     assert plan.device_errors() == ["POSITION"]
     plan.reset_errors()
     assert bool(torch.isfinite(O[:, :, 0].float()).all())
+
+
+def test_decode_repeated_calls_agree_and_leave_counters_zero():
+    """The last CTA of each row merges the partials and resets the row's counter: repeated calls give the
+    same rows bit for bit, and the counters at the end of the scratch are zero after every call."""
+    from alibi_positional_lsh_b200 import PlshForward, plsh_decode_scratch_bytes
+    n, H, d = 2000, 4, 128
+    w = workloads.Workload("case", 1, H, 2, n, d, "bf16", True, 20, 31)
+    q, k, v = (t.cuda() for t in workloads.make_qkv(w))
+    plan = PlshForward(1, H, 2, n, d, 20, True, _sigmas(H), 4, torch.bfloat16, "cuda:0")
+    plan.prepare()
+    rows = [n - 1, 1000, 3]
+    pos = torch.tensor(rows, dtype=torch.int32, device="cuda:0")
+    qr = q[:, :, rows].contiguous()
+    first = plan.decode(qr, pos, k, v)
+    first = (first[0].clone(), first[1].clone())
+    m = len(rows)
+    n_rows = 1 * H * m
+    for _ in range(3):
+        O, R = plan.decode(qr, pos, k, v)
+        torch.cuda.synchronize()
+        assert torch.equal(O, first[0]) and torch.equal(R, first[1])
+        counters = plan.decode_scratch[plsh_decode_scratch_bytes(1, H, m, d) // 4 - n_rows:]
+        assert int(counters.view(torch.int32).abs().max()) == 0
+    assert plan.device_errors() == []
