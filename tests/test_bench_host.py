@@ -1,0 +1,49 @@
+"""bench.py's host-side work counts against brute force from the oracle's definitions (no GPU).
+
+The decode and backward roofline figures divide counted work by measured
+time: decode_keys counts the keys a decode row gives weight to, and
+bwd_chunk_pairs the 64 x 64 tile pairs the backward kernels walk. Both are
+recounted here from c_ij by direct comparison of bin ids.
+"""
+import numpy as np
+import pytest
+
+import bench
+import oracle
+
+
+def _table_ids(n, sigmas, s, seed):
+    return oracle.bin_ids(oracle.draw_table(seed, sigmas, s), n)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_decode_keys_counts_weighted_keys(causal):
+    n, s = 500, 6
+    ids = _table_ids(n, [2.0, 30.0, 7.0], s, 3)
+    bm = np.stack([oracle.boundary_bits(ids[h]) for h in range(ids.shape[0])])
+    for i in (0, 1, 250, 499):
+        want = 0
+        for h in range(ids.shape[0]):
+            c = (ids[h][:, i][:, None] == ids[h]).sum(axis=0)
+            if causal:
+                c[i + 1:] = 0
+            want += int((c > 0).sum())
+        assert bench.decode_keys(bm, s, i, causal) == want
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_bwd_chunk_pairs_match_block_ranges(causal):
+    n = 700
+    ids = _table_ids(n, [2.0, 30.0, 5.0], 6, 4)
+    dq = dkdv = 0
+    for h in range(ids.shape[0]):
+        C = oracle.match_counts(ids[h])
+        for t in range(0, n, bench.BWD_TILE):
+            rows = np.arange(t, min(n, t + bench.BWD_TILE))
+            nz = np.nonzero(C[rows].sum(axis=0))[0]
+            lo, hi = int(nz.min()), int(nz.max())
+            hq = min(hi, int(rows[-1])) if causal else hi        # dQ: keys j <= i
+            lk = max(lo, t) if causal else lo                    # dK, dV: rows i >= j
+            dq += (hq - lo) // bench.BWD_TILE + 1
+            dkdv += (hi - lk) // bench.BWD_TILE + 1
+    assert bench.bwd_chunk_pairs(ids, causal, 1) == (dq, dkdv)
