@@ -50,6 +50,8 @@ def _load() -> ctypes.CDLL:
     lib.plsh_sample_bins.argtypes = [vp, i32, i32, i32, vp, vp, vp]
     lib.plsh_window.restype = i32
     lib.plsh_window.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp]
+    lib.plsh_window_from_table.restype = i32
+    lib.plsh_window_from_table.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp]
     lib.plsh_attention_fwd.restype = i32
     lib.plsh_attention_fwd.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, i32, vp, vp, vp, i32,
                                        vp, vp, vp, vp]
@@ -131,6 +133,14 @@ def plsh_window(ids_dev, H: int, s: int, n: int, causal: int, bmax_dev, tile_spa
     _check(_lib.plsh_window(_dev_ptr(ids_dev, "ids_dev"), H, s, n, int(causal), _dev_ptr(bmax_dev, "bmax_dev"),
                             _dev_ptr(tile_span_dev, "tile_span_dev"), _dev_ptr(bmask_dev, "bmask_dev"),
                             _dev_ptr(err_dev, "err_dev"), _stream_ptr(stream)))
+
+
+def plsh_window_from_table(table_dev, H: int, s: int, n: int, causal: int, bmax_dev, spans_dev, bmask_dev, err_dev,
+                           stream=None) -> None:
+    _check(_lib.plsh_window_from_table(_dev_ptr(table_dev, "table_dev"), H, s, n, int(causal),
+                                       _dev_ptr(bmax_dev, "bmax_dev"), _dev_ptr(spans_dev, "spans_dev"),
+                                       _dev_ptr(bmask_dev, "bmask_dev"), _dev_ptr(err_dev, "err_dev"),
+                                       _stream_ptr(stream)))
 
 
 def plsh_attention_fwd(Q, K, V, dtype: int, B: int, H: int, H_kv: int, n: int, d: int, sigma_dev, s: int,

@@ -3,8 +3,9 @@
 PlshForward owns the device buffers of one problem shape (allocated once
 with torch) and runs the whole path:
   a1 plsh_draw_table   (host)   -> (delta, u) table, copied to the device
-  a2 plsh_sample_bins  (K1)     -> bin ids
-  a3 plsh_window       (K2)     -> b_max, tile windows, boundary masks
+  a2+a3 plsh_window_from_table (K1 + K2 fused) -> b_max, tile windows, boundary masks
+  a2 plsh_sample_bins  (K1)     -> bin ids, computed when something needs them (the comparator,
+                                   the backward, a caller reading .ids)
   a4 plsh_attention_fwd (K3)    -> O, row_sum
   a5 plsh_attention_varlen_fwd (K4, the per-sample comparator) -> the same O, row_sum
   plsh_decode_fwd (single query rows against the cached K, V) -> rows of T~, row_sum
@@ -21,8 +22,8 @@ import torch
 
 from . import (PLSH_BF16, PLSH_F32, PLSH_TILE, PlshError, decode_device_error, plsh_alibi_banded_fwd,
                plsh_attention_bwd, plsh_attention_fwd, plsh_attention_varlen_fwd, plsh_decode_fwd,
-               plsh_decode_scratch_bytes, plsh_draw_table, plsh_sample_bins,
-               plsh_varlen_scratch_bytes, plsh_window)
+               plsh_decode_scratch_bytes, plsh_draw_table, plsh_sample_bins, plsh_window_from_table,
+               plsh_varlen_scratch_bytes)
 
 
 class PlshForward:
@@ -48,7 +49,8 @@ class PlshForward:
         self._table_copied = None  # event after the last host->device table copy
         self.table_dev = torch.empty((H, s, 2), dtype=torch.float64, device=dev)
         self.sigma_dev = torch.from_numpy(self.sigma_host.copy()).to(dev)
-        self.ids = torch.empty((H, s, n), dtype=torch.int32, device=dev)
+        self._ids = torch.empty((H, s, n), dtype=torch.int32, device=dev)
+        self._ids_ok = False  # whether _ids holds the bin ids of the current table
         self.bmax = torch.empty((H,), dtype=torch.int32, device=dev)
         self.spans = torch.empty((H, T, 2), dtype=torch.int32, device=dev)
         self.bmask = torch.empty((H, n), dtype=torch.int32 if s <= 32 else torch.int64, device=dev)
@@ -76,9 +78,21 @@ class PlshForward:
             self.table_dev.copy_(self.table_host, non_blocking=True)
             self._table_copied = torch.cuda.Event()
             self._table_copied.record(st)
-        plsh_sample_bins(self.table_dev, self.H, self.s, self.n, self.ids, self.err, st)
-        plsh_window(self.ids, self.H, self.s, self.n, int(self.causal), self.bmax, self.spans, self.bmask,
-                    self.err, st)
+        plsh_window_from_table(self.table_dev, self.H, self.s, self.n, int(self.causal), self.bmax, self.spans,
+                               self.bmask, self.err, st)
+        self._ids_ok = False
+
+    def ensure_ids(self, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+        """The bin ids [H][s][n] of the current table (K1, run on `stream` the first time they are needed)."""
+        if not self._ids_ok:
+            st = torch.cuda.current_stream() if stream is None else stream
+            plsh_sample_bins(self.table_dev, self.H, self.s, self.n, self._ids, self.err, st)
+            self._ids_ok = True
+        return self._ids
+
+    @property
+    def ids(self) -> torch.Tensor:
+        return self.ensure_ids()
 
     # a4
     def attend(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
@@ -109,8 +123,8 @@ class PlshForward:
             self.scratch = torch.empty((nbytes // 4,), dtype=torch.int32, device=self.O.device)
         st = torch.cuda.current_stream() if stream is None else stream
         plsh_attention_varlen_fwd(q, k, v, self.dtype_code, B, H, H_kv, n, d, self.sigma_dev, self.s,
-                                  self.table_dev, self.ids, self.bmask, int(self.causal), self.scratch, self.O,
-                                  self.row_sum, self.err, st)
+                                  self.table_dev, self.ensure_ids(st), self.bmask, int(self.causal), self.scratch,
+                                  self.O, self.row_sum, self.err, st)
         return self.O, self.row_sum
 
     def attend_alibi(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, eps: float = 1e-4,
@@ -144,7 +158,8 @@ class PlshForward:
                           torch.empty((B, H_kv, n, d), dtype=self.dtype, device=dev))
         delta, dQ, dK, dV = self.grads
         st = torch.cuda.current_stream() if stream is None else stream
-        plsh_attention_bwd(q, k, v, self.O, dO, self.row_sum, self.dtype_code, B, H, H_kv, n, d, self.s, self.ids,
+        plsh_attention_bwd(q, k, v, self.O, dO, self.row_sum, self.dtype_code, B, H, H_kv, n, d, self.s,
+                           self.ensure_ids(st),
                            int(self.causal), delta, dQ, dK, dV, self.err, st)
         return dQ, dK, dV
 
@@ -212,7 +227,7 @@ class PlshForward:
 class HostPipeline:
     """T~ for a stream of batches that live in pinned host memory, with the copies overlapped.
 
-    Each step copies one batch's Q, K, V in, runs the table draw, K1, K2 and K3,
+    Each step copies one batch's Q, K, V in, runs the table draw, fused K1 + K2 and K3,
     and copies O and row_sum out. Two device buffer sets alternate, so the
     host->device copy of step t+1 runs while step t computes and while its
     outputs travel device->host (the link carries both directions at once).

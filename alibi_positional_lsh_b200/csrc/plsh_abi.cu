@@ -66,6 +66,17 @@ extern "C" int plsh_window(const int32_t* ids_dev, int H, int s, int n, int caus
                              static_cast<cudaStream_t>(stream));
 }
 
+extern "C" int plsh_window_from_table(const double* table_dev, int H, int s, int n, int causal, int32_t* bmax_dev,
+                                      int32_t* tile_span_dev, void* bmask_dev, uint32_t* err_dev, void* stream) {
+  if (int rc = plsh::check_sizes("plsh_window_from_table", H, s, n)) return rc;
+  if (!table_dev || !bmax_dev || !tile_span_dev || !bmask_dev || !err_dev)
+    return fail(PLSH_ERR_INVALID_ARG, "plsh_window_from_table: null pointer");
+  if (causal != 0 && causal != 1)
+    return fail(PLSH_ERR_INVALID_ARG, "plsh_window_from_table: causal must be 0 or 1");
+  return plsh::launch_window_from_table(table_dev, H, s, n, causal, bmax_dev, tile_span_dev, bmask_dev, err_dev,
+                                        static_cast<cudaStream_t>(stream));
+}
+
 namespace plsh {
 namespace {
 

@@ -10,11 +10,12 @@
 //
 // HBM-bound: 4 bytes written per (head, hash, position), no reads beyond
 // the 16-byte table entry; the quotient is a multiply by the reciprocal with
-// an exactness test (floor_quotient), so the float64 divide runs only near
-// bin boundaries. Each thread writes 4 consecutive ids (one 16-byte
+// an exactness test (floor_quotient in plsh_binid.cuh, shared with the fused
+// window path), so the float64 divide runs only near bin boundaries. Each thread writes 4 consecutive ids (one 16-byte
 // store) when the row is 16-byte aligned.
 #include <cmath>
 
+#include "plsh_binid.cuh"
 #include "plsh_internal.h"
 
 namespace plsh {
@@ -22,30 +23,6 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kPerThread = 4;
-
-// floor(RN((pos + u) / delta)) without a division for almost every position. With
-// a = RN(pos + u) and rcp = RN(1 / delta), xa = RN(a * rcp) is within 3 * 2^-53 * xa of
-// q = RN(a / delta) (each of the three roundings is relative 2^-53). If xa lies more than
-// 2^-50 * xa from both integers around it, q lies strictly between them too and
-// floor(q) = floor(xa); otherwise the exact quotient is taken.
-__device__ __forceinline__ double floor_quotient(double pos, double u, double delta, double rcp) {
-  const double a = __dadd_rn(pos, u);
-  const double xa = __dmul_rn(a, rcp);
-  const double fl = floor(xa);
-  const double tol = xa * 0x1p-50;
-  if (xa - fl > tol && (fl + 1.0) - xa > tol) return fl;
-  return floor(__ddiv_rn(a, delta));
-}
-
-__device__ __forceinline__ int32_t bin_id(double pos, double u, double delta, double rcp, double base,
-                                          uint32_t& flags) {
-  const double id = floor_quotient(pos, u, delta, rcp) - base;
-  if (!(id >= 0.0 && id <= 2147483647.0)) {
-    flags |= PLSH_DEVERR_RANGE;
-    return 2147483647;
-  }
-  return static_cast<int32_t>(id);
-}
 
 __global__ void __launch_bounds__(kThreads) sample_bins_kernel(const double* __restrict__ table, int s,
                                                                int n, int32_t* __restrict__ ids,

@@ -22,6 +22,8 @@ int launch_sample_bins(const double* table, int H, int s, int n, int32_t* ids, u
                        cudaStream_t st);
 int launch_window(const int32_t* ids, int H, int s, int n, int causal, int32_t* bmax,
                   int32_t* spans, void* bmask, uint32_t* err, cudaStream_t st);
+int launch_window_from_table(const double* table, int H, int s, int n, int causal, int32_t* bmax,
+                             int32_t* spans, void* bmask, uint32_t* err, cudaStream_t st);
 
 struct AttnArgs {
   const void* Q; const void* K; const void* V;

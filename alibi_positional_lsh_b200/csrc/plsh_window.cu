@@ -17,6 +17,13 @@
 // (block lengths via a CTA-wide scan of block starts); only the block
 // holding each CTA's first position, and the window ends, are found by an
 // exponential-then-binary search on the non-decreasing ids.
+//
+// The ids come either from memory (plsh_window, after K1) or straight from
+// the (delta, u) table (plsh_window_from_table): each id is then evaluated
+// where it is needed with K1's own float64 steps (plsh_binid.cuh), so the
+// outputs are the same bit for bit and the [H][s][n] ids are never written
+// or read.
+#include "plsh_binid.cuh"
 #include "plsh_internal.h"
 
 namespace plsh {
@@ -24,38 +31,46 @@ namespace {
 
 constexpr int kThreads = 256;
 
-// First position of the run of value `a` that contains position p (row[p] == a).
-__device__ __forceinline__ int block_start(const int32_t* __restrict__ row, int p, int32_t a) {
+// The ids of one (head, hash) read from memory; Binning (plsh_binid.cuh) evaluates them from the table.
+struct MemRow {
+  const int32_t* row;
+  __device__ __forceinline__ int32_t at(int p) const { return row[p]; }
+};
+
+// First position of the run of value `a` that contains position p (row.at(p) == a).
+template <typename Row>
+__device__ __forceinline__ int block_start(const Row& row, int p, int32_t a) {
   int good = p, bad = -1, step = 1;
   while (true) {
     const int q = p - step;
     if (q < 0) { bad = -1; break; }
-    if (row[q] != a) { bad = q; break; }
+    if (row.at(q) != a) { bad = q; break; }
     good = q;
     if (step > (1 << 29)) { bad = -1; break; }
     step <<= 1;
   }
   while (good - bad > 1) {
     const int mid = bad + (good - bad) / 2;
-    if (row[mid] == a) good = mid; else bad = mid;
+    if (row.at(mid) == a) good = mid; else bad = mid;
   }
   return good;
 }
 
-// Last position of the run of value `a` that contains position p (row[p] == a).
-__device__ __forceinline__ int block_end(const int32_t* __restrict__ row, int p, int32_t a, int n) {
+// Last position of the run of value `a` that contains position p (row.at(p) == a).
+template <typename Row>
+__device__ __forceinline__ int block_end(const Row& row, int p, int32_t a, int n) {
   int good = p, bad = n, step = 1;
   while (true) {
     const int q = p + step;
     if (q >= n) { bad = n; break; }
-    if (row[q] != a) { bad = q; break; }
+    if (row.at(q) != a) { bad = q; break; }
     good = q;
     if (step > (1 << 29)) { bad = n; break; }
     step <<= 1;
   }
   while (bad - good > 1) {
     const int mid = good + (bad - good) / 2;
-    if (row[mid] == a) good = mid; else bad = mid;
+    if (row.at(mid) == a) good = mid; else bad = mid;
   }
   return good;
 }
@@ -66,22 +81,34 @@ __device__ __forceinline__ int block_end(const int32_t* __restrict__ row, int p,
 // block start at or before it: within the thread, else from earlier threads of the CTA (a
 // CTA-wide max-scan of the threads' last starts), else the block began before the CTA's first
 // position p0 and its start is carry[k], found once per CTA and hash by a search.
-template <typename MaskT>
-__global__ void __launch_bounds__(kThreads) mask_bmax_kernel(const int32_t* __restrict__ ids, int s, int n,
+template <typename MaskT, bool kFromTable>
+__global__ void __launch_bounds__(kThreads) mask_bmax_kernel(const int32_t* __restrict__ ids,
+                                                             const double* __restrict__ table, int s, int n,
                                                              MaskT* __restrict__ bmask,
-                                                             int32_t* __restrict__ bmax) {
+                                                             int32_t* __restrict__ bmax, uint32_t* __restrict__ err) {
   constexpr int kPer = 4;
   constexpr int kSpan = kThreads * kPer;
   constexpr int kWarps = kThreads / 32;
   __shared__ int carry[PLSH_MAX_S];
   __shared__ int warp_last[kWarps];
+  __shared__ Binning bins[kFromTable ? PLSH_MAX_S : 1];
   const int h = blockIdx.y;
   const int p0 = blockIdx.x * kSpan;
   const int t = threadIdx.x, lane = t & 31, w = t >> 5;
-  const int32_t* base = ids + static_cast<size_t>(h) * s * n;
+  const int32_t* base = kFromTable ? nullptr : ids + static_cast<size_t>(h) * s * n;
   if (t < s) {
-    const int32_t* row = base + static_cast<size_t>(t) * n;
-    carry[t] = block_start(row, p0, row[p0]);
+    if constexpr (kFromTable) {
+      const Binning b = Binning::from_table(table + (static_cast<size_t>(h) * s + t) * 2);
+      bins[t] = b;
+      if (blockIdx.x == 0) {
+        const uint32_t f = b.flags(n);
+        if (f) atomicOr(err, f);
+      }
+      carry[t] = block_start(b, p0, b.at(p0));
+    } else {
+      const MemRow row{base + static_cast<size_t>(t) * n};
+      carry[t] = block_start(row, p0, row.at(p0));
+    }
   }
   __syncthreads();
   const int pb = p0 + kPer * t;                     // this thread's first position
@@ -89,17 +116,25 @@ __global__ void __launch_bounds__(kThreads) mask_bmax_kernel(const int32_t* __re
   MaskT m[kPer] = {0, 0, 0, 0};
   int longest = 0;
   for (int k = 0; k < s; ++k) {
-    const int32_t* row = base + static_cast<size_t>(k) * n;
-    int32_t id[kPer];
-    if (vec) {
-      const int4 v = *reinterpret_cast<const int4*>(row + pb);
-      id[0] = v.x; id[1] = v.y; id[2] = v.z; id[3] = v.w;
-    } else {
+    int32_t id[kPer], prev, next;
+    if constexpr (kFromTable) {
+      const Binning b = bins[k];
 #pragma unroll
-      for (int e = 0; e < kPer; ++e) id[e] = (pb + e < n) ? row[pb + e] : 0;
+      for (int e = 0; e < kPer; ++e) id[e] = (pb + e < n) ? b.at(pb + e) : 0;
+      prev = (pb > 0 && pb < n) ? b.at(pb - 1) : 0;
+      next = (pb + kPer < n) ? b.at(pb + kPer) : 0;
+    } else {
+      const int32_t* row = base + static_cast<size_t>(k) * n;
+      if (vec) {
+        const int4 v = *reinterpret_cast<const int4*>(row + pb);
+        id[0] = v.x; id[1] = v.y; id[2] = v.z; id[3] = v.w;
+      } else {
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) id[e] = (pb + e < n) ? row[pb + e] : 0;
+      }
+      prev = (pb > 0 && pb < n) ? row[pb - 1] : 0;
+      next = (pb + kPer < n) ? row[pb + kPer] : 0;
     }
-    const int32_t prev = (pb > 0 && pb < n) ? row[pb - 1] : 0;
-    const int32_t next = (pb + kPer < n) ? row[pb + kPer] : 0;
     bool st[kPer], en[kPer];
     int mylast = -1;
 #pragma unroll
@@ -147,7 +182,9 @@ __global__ void __launch_bounds__(kThreads) mask_bmax_kernel(const int32_t* __re
 }
 
 // One warp per (head, query tile); lanes walk the hashes.
-__global__ void __launch_bounds__(kThreads) spans_kernel(const int32_t* __restrict__ ids, int H, int s, int n,
+template <bool kFromTable>
+__global__ void __launch_bounds__(kThreads) spans_kernel(const int32_t* __restrict__ ids,
+                                                         const double* __restrict__ table, int H, int s, int n,
                                                          int causal, int32_t* __restrict__ spans) {
   const int T = (n + PLSH_TILE - 1) / PLSH_TILE;
   const int warp = (blockIdx.x * kThreads + threadIdx.x) >> 5;
@@ -158,9 +195,15 @@ __global__ void __launch_bounds__(kThreads) spans_kernel(const int32_t* __restri
   const int i1 = min(n, i0 + PLSH_TILE) - 1;
   int lo = i0, hi = i1;
   for (int k = lane; k < s; k += 32) {
-    const int32_t* row = ids + (static_cast<size_t>(h) * s + k) * n;
-    lo = min(lo, block_start(row, i0, row[i0]));
-    if (!causal) hi = max(hi, block_end(row, i1, row[i1], n));
+    if constexpr (kFromTable) {
+      const Binning b = Binning::from_table(table + (static_cast<size_t>(h) * s + k) * 2);
+      lo = min(lo, block_start(b, i0, b.at(i0)));
+      if (!causal) hi = max(hi, block_end(b, i1, b.at(i1), n));
+    } else {
+      const MemRow row{ids + (static_cast<size_t>(h) * s + k) * n};
+      lo = min(lo, block_start(row, i0, row.at(i0)));
+      if (!causal) hi = max(hi, block_end(row, i1, row.at(i1), n));
+    }
   }
   lo = __reduce_min_sync(0xffffffffu, lo);
   hi = __reduce_max_sync(0xffffffffu, hi);
@@ -170,26 +213,37 @@ __global__ void __launch_bounds__(kThreads) spans_kernel(const int32_t* __restri
   }
 }
 
-}  // namespace
-
-int launch_window(const int32_t* ids, int H, int s, int n, int causal, int32_t* bmax,
-                  int32_t* spans, void* bmask, uint32_t* err, cudaStream_t st) {
-  (void)err;
+template <bool kFromTable>
+int launch_window_impl(const int32_t* ids, const double* table, int H, int s, int n, int causal, int32_t* bmax,
+                       int32_t* spans, void* bmask, uint32_t* err, cudaStream_t st) {
   cudaError_t e = cudaMemsetAsync(bmax, 0, sizeof(int32_t) * H, st);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(bmax)");
   dim3 g1(ceil_div(n, 4 * kThreads), H);
   if (s <= 32)
-    mask_bmax_kernel<uint32_t><<<g1, kThreads, 0, st>>>(ids, s, n, static_cast<uint32_t*>(bmask), bmax);
+    mask_bmax_kernel<uint32_t, kFromTable><<<g1, kThreads, 0, st>>>(ids, table, s, n, static_cast<uint32_t*>(bmask),
+                                                                    bmax, err);
   else
-    mask_bmax_kernel<unsigned long long><<<g1, kThreads, 0, st>>>(
-        ids, s, n, static_cast<unsigned long long*>(bmask), bmax);
+    mask_bmax_kernel<unsigned long long, kFromTable><<<g1, kThreads, 0, st>>>(
+        ids, table, s, n, static_cast<unsigned long long*>(bmask), bmax, err);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "mask_bmax_kernel launch");
   const long long warps = static_cast<long long>(H) * ceil_div(n, PLSH_TILE);
   const int g2 = static_cast<int>((warps * 32 + kThreads - 1) / kThreads);
-  spans_kernel<<<g2, kThreads, 0, st>>>(ids, H, s, n, causal, spans);
+  spans_kernel<kFromTable><<<g2, kThreads, 0, st>>>(ids, table, H, s, n, causal, spans);
   e = cudaGetLastError();
   return e == cudaSuccess ? PLSH_OK : cuda_fail(e, "spans_kernel launch");
+}
+
+}  // namespace
+
+int launch_window(const int32_t* ids, int H, int s, int n, int causal, int32_t* bmax,
+                  int32_t* spans, void* bmask, uint32_t* err, cudaStream_t st) {
+  return launch_window_impl<false>(ids, nullptr, H, s, n, causal, bmax, spans, bmask, err, st);
+}
+
+int launch_window_from_table(const double* table, int H, int s, int n, int causal, int32_t* bmax,
+                             int32_t* spans, void* bmask, uint32_t* err, cudaStream_t st) {
+  return launch_window_impl<true>(nullptr, table, H, s, n, causal, bmax, spans, bmask, err, st);
 }
 
 }  // namespace plsh

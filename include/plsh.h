@@ -138,6 +138,25 @@ PLSH_API int plsh_window(const int32_t* ids_dev, int H, int s, int n, int causal
                 int32_t* tile_span_dev, void* bmask_dev, uint32_t* err_dev, void* stream);
 
 /*
+ * plsh_window_from_table (K1 + K2 fused) -- plsh_window's outputs straight
+ * from the (delta, u) table, without the [H][s][n] bin ids.
+ *
+ * Cites: Methodology 1 (mechanism: bin(i) = floor((i + u)/delta); structure:
+ * contiguous blocks) and Methodology 2 (block-size control). Every id the
+ * window reduction needs is evaluated where it is needed, with the same
+ * IEEE float64 steps as plsh_sample_bins, so bmax_dev, tile_span_dev and
+ * bmask_dev equal those of plsh_sample_bins followed by plsh_window, bit for
+ * bit, and err_dev receives the same PLSH_DEVERR_TABLE / PLSH_DEVERR_RANGE
+ * bits. Call plsh_sample_bins as well when the ids themselves are needed
+ * (plsh_attention_varlen_fwd, plsh_attention_bwd).
+ *
+ *   table_dev  [H][s][2] float64 (delta, u), as given to plsh_sample_bins.
+ *   Other arguments as plsh_window.
+ */
+PLSH_API int plsh_window_from_table(const double* table_dev, int H, int s, int n, int causal, int32_t* bmax_dev,
+                                    int32_t* tile_span_dev, void* bmask_dev, uint32_t* err_dev, void* stream);
+
+/*
  * plsh_attention_fwd (K3) -- the fused banded Positional-LSH attention.
  *
  * Cites: Methodology 2 (M~ = (1/s) sum_k M(h_k)), Methodology 3 (ALiBi
