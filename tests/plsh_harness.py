@@ -6,7 +6,6 @@ the seeded inputs from workloads.py.
 """
 from __future__ import annotations
 
-import math
 from typing import Optional, Sequence
 
 import numpy as np
