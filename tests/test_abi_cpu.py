@@ -165,3 +165,15 @@ def test_backward_rejects_bad_arguments_before_any_launch(plsh):
     assert lib.plsh_attention_bwd(*args(causal=2)) == 1
     assert lib.plsh_attention_bwd(*args(dtype=9)) == 2
     assert lib.plsh_attention_bwd(*args(Q=ctypes.c_void_p((1 << 20) + 4))) == 1 and "aligned" in plsh.plsh_last_error()
+
+
+def test_window_from_table_rejects_bad_arguments_before_any_launch(plsh):
+    lib = plsh._lib
+    null = None
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the checks fail first
+    assert lib.plsh_window_from_table(null, 1, 4, 100, 0, fake, fake, fake, fake, null) == 1
+    assert "null" in plsh.plsh_last_error()
+    assert lib.plsh_window_from_table(fake, 1, 4, 100, 2, fake, fake, fake, fake, null) == 1
+    assert lib.plsh_window_from_table(fake, 1, 0, 100, 0, fake, fake, fake, fake, null) == 1
+    assert lib.plsh_window_from_table(fake, 1, 65, 100, 0, fake, fake, fake, fake, null) == 1
+    assert lib.plsh_window_from_table(fake, 0, 4, 100, 0, fake, fake, fake, fake, null) == 1
