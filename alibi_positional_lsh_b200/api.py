@@ -83,7 +83,10 @@ class PlshForward:
         self._ids_ok = False
 
     def ensure_ids(self, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
-        """The bin ids [H][s][n] of the current table (K1, run on `stream` the first time they are needed)."""
+        """The bin ids [H][s][n] of the current table (K1, run on `stream` the first time they are needed).
+
+        K1 reads the device copy of the table that prepare() enqueued on its own stream: with the default
+        (current) stream on both sides the order is implicit; with different streams, order them."""
         if not self._ids_ok:
             st = torch.cuda.current_stream() if stream is None else stream
             plsh_sample_bins(self.table_dev, self.H, self.s, self.n, self._ids, self.err, st)
