@@ -141,3 +141,36 @@ def test_backward_headline_sampled():
         want_v.append(dv)
     _assert_grads((np.stack(got_q), np.stack(got_k), np.stack(got_v)),
                   (np.stack(want_q), np.stack(want_k), np.stack(want_v)), w.torch_dtype, "backward headline")
+
+
+def test_backward_single_head_fp32_workload():
+    """fp32, d = 64, non-causal, n = 1024, s = 8: the full oracle."""
+    w = W["single_head_n1024"]
+    (q, k, v, dO), plan, got = _run(w.B, w.H, w.H_kv, w.n, w.d, w.torch_dtype, w.causal, w.s, w.sigmas(), w.seed)
+    want = oracle.backward(PH.f64(q), PH.f64(k), PH.f64(v), PH.f64(dO), plan.table_host.numpy(), w.causal)
+    _assert_grads(got, want, w.torch_dtype, "backward single_head_n1024")
+
+
+def test_backward_mha8_sampled_non_causal():
+    """bf16, 8 heads, n = 8192, non-causal (both sides of every key): dQ on sampled rows of every head,
+    dK and dV on sampled keys of heads 0 and 5."""
+    w = W["mha8_n8192"]
+    (q, k, v, dO), plan, (dQ, dK, dV) = _run(w.B, w.H, w.H_kv, w.n, w.d, w.torch_dtype, w.causal, w.s,
+                                             w.sigmas(), w.seed)
+    ids = oracle.bin_ids(plan.table_host.numpy(), w.n)
+    Q, K, V, G = PH.f64(q), PH.f64(k), PH.f64(v), PH.f64(dO)
+    rows = sorted(set(workloads.sample_rows(w.n, 8, w.seed + 4)) | {0, 63, 64, w.n - 1})
+    keys = sorted(set(workloads.sample_rows(w.n, 4, w.seed + 5)) | {0, w.n - 1})
+    got, want = ([], [], []), ([], [], [])
+    for h in range(w.H):
+        dq, _, _ = oracle.approx_attention_grad_sampled(Q[0, h], K[0, h], V[0, h], G[0, h], ids[h], w.causal, rows, [])
+        got[0].append(dQ[0, h, rows])
+        want[0].append(dq)
+    for h in (0, 5):
+        _, dk, dv = oracle.approx_attention_grad_sampled(Q[0, h], K[0, h], V[0, h], G[0, h], ids[h], w.causal, [], keys)
+        got[1].append(dK[0, h, keys])
+        want[1].append(dk)
+        got[2].append(dV[0, h, keys])
+        want[2].append(dv)
+    _assert_grads(tuple(np.stack(x) for x in got), tuple(np.stack(x) for x in want), w.torch_dtype,
+                  "backward mha8_n8192")
