@@ -126,3 +126,13 @@ def test_decode_repeated_calls_agree_and_leave_counters_zero():
         counters = plan.decode_scratch[plsh_decode_scratch_bytes(1, H, m, d) // 4 - n_rows:]
         assert int(counters.view(torch.int32).abs().max()) == 0
     assert plan.device_errors() == []
+
+
+def test_decode_mha8_non_causal_both_sides():
+    """8 heads, n = 8192, non-causal: each row's walk runs below and above its position."""
+    w = W["mha8_n8192"]
+    rows = [0, 4095, 4096, w.n - 1]
+    q, k, v, plan, O, R = _run(w.B, w.H, w.H_kv, w.n, w.d, w.torch_dtype, w.causal, w.s, w.sigmas(), w.seed, rows)
+    want_O, want_R = PH.oracle_rows(q, k, v, plan.table_host.numpy(), w.causal, rows)
+    to, tr = PH.tolerance(w.torch_dtype, v)
+    PH.assert_close(O, R, want_O, want_R, to, tr, "decode mha8")
