@@ -8,7 +8,8 @@
 // Blocks are contiguous (Methodology 1, structure), so walking away from i
 // the OR only grows and c_ij only falls: the walk stops at the first chunk
 // of keys whose counts are all zero. Only the keys sharing a block with i in
-// some hash are read, so the kernel is bound by reading their K and V rows.
+// some hash are read: their K and V rows are the bytes the call must move, and
+// the chain of dependent loads along the walk sets its latency.
 //
 // Each query row's walk is spread over G CTAs of 256 threads (G chosen so the
 // grid covers the SMs about twice, at most 8). Keys are taken in chunks of 256
