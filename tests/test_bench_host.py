@@ -47,3 +47,26 @@ def test_bwd_chunk_pairs_match_block_ranges(causal):
             dq += (hq - lo) // bench.BWD_TILE + 1
             dkdv += (hi - lk) // bench.BWD_TILE + 1
     assert bench.bwd_chunk_pairs(ids, causal, 1) == (dq, dkdv)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_issued_and_visited_key_tiles(causal):
+    """The headline roofline counts issued tensor work as 128-key tiles: per query tile, the span of keys
+    with weight rounded up to whole tiles (issued_tiles), and the 128-aligned tiles the kernel walks around
+    the diagonal (kernel_tiles). Both recounted from c_ij."""
+    n, T = 1000, 8
+    ids = _table_ids(n, [3.0, 60.0, 400.0], 5, 6)
+    spans = np.stack([oracle.tile_spans(ids[h], causal) for h in range(ids.shape[0])])
+    issued = visited = 0
+    for h in range(ids.shape[0]):
+        C = oracle.match_counts(ids[h])
+        if causal:
+            C = np.tril(C)
+        for t in range(T):
+            rows = np.arange(t * 128, min(n, t * 128 + 128))
+            nz = np.nonzero(C[rows].sum(axis=0))[0]
+            lo, hi = int(nz.min()), int(nz.max())
+            issued += -(-(hi - lo + 1) // 128)
+            visited += sum(1 for j0 in range(0, n, 128) if j0 + 127 >= lo and j0 <= hi)
+    assert bench.issued_tiles(spans, causal) == issued
+    assert bench.kernel_tiles(spans, causal) == visited
