@@ -12,8 +12,11 @@
 //
 // Persistent CTAs (one per SM) walk a static list of items, heads with the
 // widest windows first. Warp roles (352 threads):
-//   warps 0-7    softmax: warp w owns rows 32 (w % 4) .. + 31 (TMEM lane
-//                quarter w % 4) and keys 64 (w / 4) .. + 63 of every tile
+//   warps 0-7    softmax: warp w owns rows 32 (w % 4) + 16 (w / 4) .. + 15 of
+//                every tile (16 lanes of its TMEM lane quarter w % 4); inside
+//                the warp, threads t and t + 16 share row t % 16 and split each
+//                pair of 16-key chunks (the 16x32bx2 TMEM access shape), so a
+//                row's maximum and sum combine with one shuffle
 //   warp 8       TMA producer: Q per item (two buffers), K and V per key tile
 //                (two stages each)
 //   warp 9       TMEM owner and single-thread tcgen05.mma issuer
@@ -23,8 +26,7 @@
 // and odd index): S(g+1) = Q K^T is issued before O += P(g) V, so the tensor
 // core computes the next tile's scores while the softmax works on the
 // current one; the softmax turns S into bf16 P written back over S, and the
-// PV MMA reads P from TMEM. The two warps sharing a row exchange their half
-// maxima per tile and their half sums per item through shared memory.
+// PV MMA reads P from TMEM.
 //
 // Weights. P_ij = c_ij 2^(S_ij log2(e)/sqrt(d) - m): the count multiplies the
 // exponential as an exact small-integer float, so no logarithm is taken.
@@ -33,19 +35,22 @@
 // depends on the row only (a carry) and a part that depends on the key only,
 // the same for a whole warp: below the diagonal R = Y | suf[c] with Y the OR
 // from the tile's end to the row; above it R = Z | pre[c] with Z the OR from
-// the row to the tile's start. On the diagonal tile each warp owns 32 rows:
-// keys in its own 32-key block are scanned from the row outwards (before S
-// is ready), which yields the carries for the rest of the tile, whose keys
-// take range ORs that end (or start) at the warp's block. Key tiles are
+// the row to the tile's start. On the diagonal tile the rows of each 32-row
+// block (one TMEM lane quarter) scan the keys of the block's own 32 keys from
+// the row outwards (before S is ready), which yields the carries for the rest
+// of the tile, whose keys take range ORs that end (or start) at that block. Key tiles are
 // visited diagonal first, then downward, then upward, so the carries pass
 // from tile to tile.
 // The reference m is a running upper bound: the largest S log2(e)/sqrt(d)
-// over the tile's keys that can carry weight raises it when it exceeds m by
-// more than 8, and O and the row sum are then rescaled; so P <= s 2^8, and
-// the row's own key (c = s) keeps the sum away from zero. Per tile a softmax
-// thread reads its row of S from TMEM twice, in chunks (the maximum, then
-// P), and writes P of keys [16ch, 16ch + 16) as bf16 pairs to columns
-// [8ch, 8ch + 8) of the S region, over columns it has already read.
+// over the tile's live keys raises it when it exceeds m by more than 8, and O
+// and the row sum are then rescaled; so P <= s 2^8, and the row's own key
+// (c = s) keeps the sum away from zero. A pair of chunks whose key nearest to
+// the warp's rows has count 0 for all of them has count 0 throughout (the OR of
+// the masks only grows moving away from a row): its S is neither read nor
+// exponentiated and its P is written as zeros. Per tile a softmax thread reads
+// its live S twice (the maximum, then P, chunk by chunk) and writes P of keys
+// [16ch, 16ch + 16) as bf16 pairs to columns [8ch, 8ch + 8) of the S region,
+// over columns already read.
 //
 // The per-sample comparator (K4) runs the same machinery with each item walked
 // once per hash k over that hash's own window, the boundary masks reduced to
@@ -101,8 +106,9 @@ struct alignas(16) MaskStage {
   // dq[q][c] = OR bm[c + 1 .. 32q] for c < 32q, OR bm[32q + 32 .. c] for c >= 32q + 32
   MaskT dq[4][kTile];
   // the tile as the softmax needs it: valid (0 = end of the CTA's work), kind (0 diagonal,
-  // 1 below, 2 above), first / last tile of its item, item index x, first key j0
-  int valid, kind, first, last, x, j0, pad1, pad2;
+  // 1 below, 2 above), first / last tile of its item,
+  // item index x, first key j0, and the comparator's hash of the sub-item
+  int valid, kind, first, last, x, j0, sub, pad;
 };
 
 template <typename MaskT>
@@ -111,8 +117,6 @@ struct __align__(1024) TcSmem {
   uint8_t k[kStages][kTileBytes];
   uint8_t v[kStages][kTileBytes];
   MaskStage<MaskT> m[kMaskStages];
-  float pmax[2][2][kTile];         // [tile parity][key half][row] half maxima of S
-  float psum[2][2][kTile];         // [item parity][key half][row] half sums of P
   uint32_t cw[8][kSoftmaxWarps * 32];  // diagonal tile: own-block counts, one column per softmax thread
   int16_t order[kMaxSortedHeads];  // heads by decreasing window width
   int32_t width[kMaxSortedHeads];
@@ -121,7 +125,6 @@ struct __align__(1024) TcSmem {
   uint64_t v_full[kStages], v_empty[kStages];
   uint64_t m_full[kMaskStages], m_empty[kMaskStages];
   uint64_t s_full[2], p_full[2], pv_done[2];
-  uint64_t xmax[2], xsum[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -291,45 +294,56 @@ __device__ __forceinline__ void regs_after_wait(uint32_t (&r)[N]) {
   for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
 }
 
+// The largest of m and 32 raw fp32 values (four independent chains of three-input maxima).
 __device__ __forceinline__ float max32(const uint32_t (&v)[32], float m) {
-  float mx[8];
+  float mx[4];
 #pragma unroll
-  for (int u = 0; u < 8; ++u) mx[u] = __uint_as_float(v[u]);
-#pragma unroll
-  for (int c = 8; c < 32; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(v[c]));
-  return fmaxf(m, fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                        fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))));
+  for (int u = 0; u < 4; ++u) {
+    const uint32_t* w = v + 8 * u;
+    float x = max3(__uint_as_float(w[0]), __uint_as_float(w[1]), __uint_as_float(w[2]));
+    x = max3(x, __uint_as_float(w[3]), __uint_as_float(w[4]));
+    x = max3(x, __uint_as_float(w[5]), __uint_as_float(w[6]));
+    mx[u] = fmaxf(x, __uint_as_float(w[7]));
+  }
+  return max3(m, max3(mx[0], mx[1], mx[2]), mx[3]);
 }
 
-// float(v) for 0 <= v < 2^23, exactly: the float with the bits of 2^23 + v, minus 2^23.
-__device__ __forceinline__ float small_count(uint32_t v) { return __int_as_float(0x4B000000u | v) - 8388608.0f; }
+// Constants of the softmax, each as a packed pair: the scale log2(e)/sqrt(d), -m, and -2^23 (which
+// turns the float with the bits of 2^23 + c back into c).
+struct SoftmaxK {
+  uint64_t sc2, negm2, neg2p23;
+};
 
-// s - popcount(carry | km) as a float, exactly, given cs = 2^23 + s.
+// P = c 2^(S sc - m) for 16 keys (S as raw fp32 bits), with c = popcount(keep & ~km[k]) the number
+// of hashes with no block boundary between the row and key k (keep: the hashes without a boundary
+// in the row's own part of the gap); packed as 8 bf16 pairs. Returns the sum of P.
 template <typename MaskT>
-__device__ __forceinline__ float count_weight(MaskT carry, MaskT km, float cs) {
-  return cs - __int_as_float(0x4B000000u | static_cast<uint32_t>(popc_m(static_cast<MaskT>(carry | km))));
-}
-
-// P = w 2^(S sc - m) for 16 keys (S as raw fp32 bits) with w = s - popcount(carry | km[k]),
-// packed as 8 bf16 pairs. Returns the sum of P.
-template <typename MaskT>
-__device__ __forceinline__ float p16_carry(const uint32_t (&sv)[16], const MaskT* km, MaskT carry, float sc,
-                                           float neg_m, float cs, uint32_t (&pk)[8]) {
-  float ls[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+__device__ __forceinline__ float p16_carry(const uint32_t (&sv)[16], const MaskT* km, MaskT keep, const SoftmaxK& k2,
+                                           uint32_t (&pk)[8]) {
+  uint64_t ls2[2] = {0ull, 0ull};
 #pragma unroll
   for (int g4 = 0; g4 < 4; ++g4) {
     MaskT bb[4];
     load4(km + 4 * g4, bb);
-    float p[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      p[e] = ex2_approx(fmaf(__uint_as_float(sv[4 * g4 + e]), sc, neg_m)) * count_weight(carry, bb[e], cs);
-      ls[e] += p[e];
+    for (int e2 = 0; e2 < 2; ++e2) {
+      const int kk = 4 * g4 + 2 * e2;
+      float x0, x1;
+      f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[kk]), __uint_as_float(sv[kk + 1])), k2.sc2, k2.negm2), x0, x1);
+      const uint32_t c0 = 0x4B000000u | static_cast<uint32_t>(popc_m(static_cast<MaskT>(keep & ~bb[2 * e2])));
+      const uint32_t c1 = 0x4B000000u | static_cast<uint32_t>(popc_m(static_cast<MaskT>(keep & ~bb[2 * e2 + 1])));
+      const uint64_t w2 = f2_add(f2_pack(__uint_as_float(c0), __uint_as_float(c1)), k2.neg2p23);
+      const uint64_t p2 = f2_mul(f2_pack(ex2_approx(x0), ex2_approx(x1)), w2);
+      ls2[e2] = f2_add(ls2[e2], p2);
+      float p0, p1;
+      f2_unpack(p2, p0, p1);
+      pk[2 * g4 + e2] = pack_bf16x2(p0, p1);
     }
-    pk[2 * g4] = pack_bf16x2(p[0], p[1]);
-    pk[2 * g4 + 1] = pack_bf16x2(p[2], p[3]);
   }
-  return (ls[0] + ls[1]) + (ls[2] + ls[3]);
+  float a0, a1, b0, b1;
+  f2_unpack(ls2[0], a0, a1);
+  f2_unpack(ls2[1], b0, b1);
+  return (a0 + a1) + (b0 + b1);
 }
 
 // Exact ALiBi: P = 2^(S sc - m - lam |i - j|) for 16 keys, with t0 = lam (i - j) at the first key
@@ -356,21 +370,31 @@ __device__ __forceinline__ float p16_alibi(const uint32_t (&sv)[16], float t0, f
 }
 
 // The same with the counts given as bytes: the count of key k in byte k % 4 of c4[k / 4].
-__device__ __forceinline__ float p16_counts(const uint32_t (&sv)[16], const uint32_t (&c4)[4], float sc,
-                                            float neg_m, uint32_t (&pk)[8]) {
-  float ls[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+__device__ __forceinline__ float p16_counts(const uint32_t (&sv)[16], const uint32_t (&c4)[4], const SoftmaxK& k2,
+                                            uint32_t (&pk)[8]) {
+  uint64_t ls2[2] = {0ull, 0ull};
 #pragma unroll
   for (int g4 = 0; g4 < 4; ++g4) {
-    float p[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      p[e] = ex2_approx(fmaf(__uint_as_float(sv[4 * g4 + e]), sc, neg_m)) * small_count((c4[g4] >> (8 * e)) & 0xffu);
-      ls[e] += p[e];
+    for (int e2 = 0; e2 < 2; ++e2) {
+      const int kk = 4 * g4 + 2 * e2;
+      float x0, x1;
+      f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[kk]), __uint_as_float(sv[kk + 1])), k2.sc2, k2.negm2), x0, x1);
+      // bytes 2 e2 and 2 e2 + 1 of c4[g4] under the exponent bits of 2^23
+      const uint32_t c0 = __byte_perm(c4[g4], 0x4B000000u, 0x7540u | (2u * e2));
+      const uint32_t c1 = __byte_perm(c4[g4], 0x4B000000u, 0x7540u | (2u * e2 + 1u));
+      const uint64_t w2 = f2_add(f2_pack(__uint_as_float(c0), __uint_as_float(c1)), k2.neg2p23);
+      const uint64_t p2 = f2_mul(f2_pack(ex2_approx(x0), ex2_approx(x1)), w2);
+      ls2[e2] = f2_add(ls2[e2], p2);
+      float p0, p1;
+      f2_unpack(p2, p0, p1);
+      pk[2 * g4 + e2] = pack_bf16x2(p0, p1);
     }
-    pk[2 * g4] = pack_bf16x2(p[0], p[1]);
-    pk[2 * g4 + 1] = pack_bf16x2(p[2], p[3]);
   }
-  return (ls[0] + ls[1]) + (ls[2] + ls[3]);
+  float a0, a1, b0, b1;
+  f2_unpack(ls2[0], a0, a1);
+  f2_unpack(ls2[1], b0, b1);
+  return (a0 + a1) + (b0 + b1);
 }
 
 // Diagonal tile, warp q (rows [32q, 32q + 32), row r): counts of the warp's own 32 keys, as bytes
@@ -484,8 +508,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       mbar_init(&sm.s_full[i], 1);
       mbar_init(&sm.p_full[i], kSoftmaxWarps);
       mbar_init(&sm.pv_done[i], 1);
-      mbar_init(&sm.xmax[i], kSoftmaxWarps);
-      mbar_init(&sm.xsum[i], kSoftmaxWarps);
     }
     for (int i = 0; i < kMaskStages; ++i) {
       mbar_init(&sm.m_full[i], 1);
@@ -590,9 +612,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         const uint32_t o_tmem = tmem + kColO + 128u * static_cast<uint32_t>(ti.k & 1);
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk) {
-          // keys 16kk..16kk+15: P of key half kk/4 at columns 64 (kk/4) + 8 (kk%4); the keys are two
-          // 8-row groups of the MN-major V tile, whose two d halves sit kChunkBytes apart
-          mma_ts(o_tmem, p_tmem + 64u * (kk >> 2) + 8u * (kk & 3),
+          // keys 16kk..16kk+15: P at columns 8kk; the keys are two 8-row groups of the MN-major V
+          // tile, whose two d halves sit kChunkBytes apart
+          mma_ts(o_tmem, p_tmem + 8u * kk,
                  (st ? v_desc[1] : v_desc[0]) + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
                  (!ti.first() || kk > 0) ? 1u : 0u);
         }
@@ -759,6 +781,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         ms.last = ti.last() ? 1 : 0;
         ms.x = ti.x;
         ms.j0 = ti.j0();
+        ms.sub = ti.sub;
         if (ti.first() && ti.bad_window) atomicOr(err, PLSH_DEVERR_WINDOW);
       }
       __syncwarp();
@@ -782,20 +805,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     }
     }  // masks (PLSH) or descriptors only (exact ALiBi)
   } else {
-    // ------------------------------------------------------------ softmax: quarter warp & 3, key half warp >> 2
+    // ------------------------------------------------------------ softmax
+    // Warp w owns rows 32 (w % 4) + 16 (w / 4) .. + 15 of every tile (16 lanes of its TMEM
+    // quarter). Inside the warp, threads t and t + 16 share row t % 16: of each pair of 16-key
+    // chunks (keys 32m .. 32m + 31) thread t takes the even chunk and thread t + 16 the odd one
+    // (the 16x32bx2 TMEM access shape), so a row's maximum and sum combine with one shuffle.
     const int quarter = warp & 3;
-    const int hf = warp >> 2;           // this warp's key half: keys [64 hf, 64 hf + 64) of every tile
-    const int r = quarter * 32 + lane;  // row within the tile == TMEM lane
-    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const int hq = warp >> 2;   // which 16 rows of the quarter
+    const int kh = lane >> 4;   // which chunk of each pair
+    const int r = quarter * 32 + hq * 16 + (lane & 15);  // row within the tile == TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32 + hq * 16) << 16;
     const float sc = 1.4426950408889634f / sqrtf(static_cast<float>(kD));
     // weights count hashes: all s of them, or (comparator) the one hash of the sub-item
     const int sw = kVarlen ? 1 : s;
-    const float cs = 8388608.0f + static_cast<float>(sw);  // 2^23 + sw
     float m2 = -INFINITY, l = 0.0f;
     MaskT Y = 0, Z = 0;
     float lam = 0.0f;  // exact ALiBi: log2(e) / sigma of the item's head
     int a_i0 = 0;      // exact ALiBi: the item's first row
-    int items = 0;  // items finished by this warp
+    int items = 0;     // items finished by this warp
     for (int g = 0;; ++g) {
       const int st = g % kMaskStages;
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.m_full[st], static_cast<uint32_t>(g / kMaskStages) & 1u,
@@ -822,31 +849,49 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       tc_fence_after();
       const uint32_t s_base = tmem + lane_off + kColS + 128u * static_cast<uint32_t>(g & 1);
 
-      // ---- pass 1: this half's maximum of S over the 16-key chunks that can carry weight (when
-      // causal, the diagonal tile's chunks past the warp's own block cannot); exchange with the
-      // other half of the row
-      const int n_live = (kCausal && kind == 0) ? 2 * quarter + 2 : kTile / 16;
+      // ---- the chunk pairs that carry weight for some row of the warp. Moving away from the row
+      // the OR of the boundary masks only grows (blocks are contiguous), so a pair whose key
+      // nearest to the rows has count 0 for every row of the warp has count 0 throughout: its S
+      // is neither read nor exponentiated, and its P is written as zeros. (When causal, the
+      // diagonal tile's pairs past the warp's own block are dead as well.)
+      const int n_pairs = (kCausal && kind == 0) ? quarter + 1 : kTile / 32;
+      const MaskT Zc = static_cast<MaskT>(Z | ms.bm[0]);
+      // the hashes without a boundary in the row's part of the gap, below and above the rows, and
+      // the per-key part: below Y | suf[c], above Z | bm[0] | pre[c], diagonal lo | dq[c] below
+      // the warp's block and hi | dq[c] above it (the comparator's sub-item counts its own hash)
+      const MaskT hashes = kVarlen ? static_cast<MaskT>(static_cast<MaskT>(1) << ms.sub) : FULL;
+      const MaskT keep_lo = static_cast<MaskT>(hashes & ~(kind == 1 ? Y : lo));
+      const MaskT keep_hi = static_cast<MaskT>(hashes & ~(kind == 2 ? Zc : hi));
+      const MaskT* km_tile = kind == 1 ? ms.suf : (kind == 2 ? ms.pre : ms.dq[quarter]);
+      uint32_t live = 0;  // bit m: pair m
+#pragma unroll
+      for (int m = 0; m < kTile / 32; ++m) {
+        bool lv = m < n_pairs;
+        if (!kAlibi && lv && !(kind == 0 && m == quarter)) {
+          const bool below = kind == 1 || (kind == 0 && m < quarter);
+          const MaskT kn = km_tile[below ? 32 * m + 31 : 32 * m];  // the key nearest to the rows
+          lv = static_cast<MaskT>((below ? keep_lo : keep_hi) & ~kn) != 0;
+        }
+        if (__any_sync(0xffffffffu, lv)) live |= 1u << m;
+      }
+
+      // ---- pass 1: the row's maximum of S over the live 64-key halves (thread t reads columns
+      // [64h, 64h + 32), thread t + 16 [64h + 32, 64h + 64)), combined over the row's two threads
       float mraw = -INFINITY;
       {
-        const int c0 = 4 * hf;
         uint32_t sa[32], sb[32];
-        if (c0 < n_live) tmem_ld32(s_base + 16u * c0, sa);
-        if (c0 + 2 < n_live) tmem_ld32(s_base + 16u * (c0 + 2), sb);
+        if (live & 3u) tmem_ld16x2_32<32>(s_base, sa);
+        if (live & 12u) tmem_ld16x2_32<32>(s_base + 64u, sb);
         tmem_wait_ld();
         regs_after_wait(sa);
         regs_after_wait(sb);
-        if (c0 < n_live) mraw = max32(sa, mraw);
-        if (c0 + 2 < n_live) mraw = max32(sb, mraw);
+        if (live & 3u) mraw = max32(sa, mraw);
+        if (live & 12u) mraw = max32(sb, mraw);
       }
-      sm.pmax[g & 1][hf][r] = mraw;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.xmax[g & 1]);
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.xmax[g & 1], static_cast<uint32_t>(g >> 1) & 1u, abort_flag, err)))
-        break;
-      mraw = fmaxf(mraw, sm.pmax[g & 1][hf ^ 1][r]);
+      mraw = fmaxf(mraw, __shfl_xor_sync(0xffffffffu, mraw, 16));
       const float mt = mraw * sc;
 
-      // ---- reference update (the same in both halves); this half of O is rescaled in place once
+      // ---- reference update (the same in the row's two threads); O is rescaled in place once
       // PV(g-1) has completed
       float alpha = 1.0f;
       bool need_rescale = false;
@@ -863,54 +908,55 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
                                                abort_flag, err)))
           break;
         tc_fence_after();
-        const uint32_t o_half = tmem + lane_off + kColO + 128u * static_cast<uint32_t>(items & 1) + 64u * hf;
+        // thread t: columns [16 q4, 16 q4 + 16), thread t + 16 the same 64 columns further
+        const uint32_t o_row = tmem + lane_off + kColO + 128u * static_cast<uint32_t>(items & 1);
 #pragma unroll 1
         for (int q4 = 0; q4 < 4; ++q4) {
           uint32_t raw[16];
-          tmem_ld16(o_half + 16u * q4, raw);
+          tmem_ld16x2_16<64>(o_row + 16u * q4, raw);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 16; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * alpha);
-          tmem_st16(o_half + 16u * q4, raw);
+          tmem_st16x2_16<64>(o_row + 16u * q4, raw);
         }
       }
 
-      // ---- pass 2: P = c 2^(S sc - m) for this half's 4 chunks; P of chunk 4 hf + c goes to
-      // columns 64 hf + 8c, over S columns of this half already read
-      const MaskT Zc = static_cast<MaskT>(Z | ms.bm[0]);
+      // ---- pass 2: P = c 2^(S sc - m), one chunk pair at a time; P of chunk ch goes to columns
+      // 8 ch, over S columns already read (S of chunk ch sits at columns 16 ch)
+      SoftmaxK k2;
+      k2.sc2 = f2_pack(sc, sc);
+      k2.negm2 = f2_pack(neg_m, neg_m);
+      k2.neg2p23 = f2_pack(-8388608.0f, -8388608.0f);
       float lsum = 0.0f;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        const int ch = 4 * hf + c;
+      for (int m = 0; m < kTile / 32; ++m) {
         uint32_t pk[8];
-        if (ch >= n_live) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) pk[e] = 0u;
-        } else {
+        if (live & (1u << m)) {
           uint32_t sv[16];
-          tmem_ld16(s_base + 16u * ch, sv);
+          tmem_ld16x2_16<16>(s_base + 32u * m, sv);  // this thread's chunk 2m + kh
           tmem_wait_ld();
           regs_after_wait(sv);
+          const int ch = 2 * m + kh;
           if constexpr (kAlibi) {
             // i - j for the chunk's first key; keys past the row (when causal) and past n are dropped
             const int jc = ms.j0 + 16 * ch;
             const int d0 = a_i0 + r - jc;
             lsum += p16_alibi(sv, lam * static_cast<float>(d0), lam, min(kCausal ? d0 : 16, n - 1 - jc), sc, neg_m, pk);
-          } else if (kind == 0 && (ch >> 1) == quarter) {
-            // the warp's own block on the diagonal: counts from the scan
+          } else if (kind == 0 && m == quarter) {
+            // the warp's own block on the diagonal: counts from the scan (words 4 kh .. 4 kh + 3)
             uint32_t c4[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) c4[u] = sm.cw[4 * (ch & 1) + u][threadIdx.x];
-            lsum += p16_counts(sv, c4, sc, neg_m, pk);
+            for (int u = 0; u < 4; ++u) c4[u] = sm.cw[4 * kh + u][threadIdx.x];
+            lsum += p16_counts(sv, c4, k2, pk);
           } else {
-            // below: Y | suf[c]; above: Z | bm[0] | pre[c]; diagonal: lo | dq[c] below the warp's
-            // block, hi | dq[c] above it
-            const MaskT* km = kind == 1 ? ms.suf : (kind == 2 ? ms.pre : ms.dq[quarter]);
-            const MaskT carry = kind == 1 ? Y : (kind == 2 ? Zc : ((ch >> 1) < quarter ? lo : hi));
-            lsum += p16_carry<MaskT>(sv, km + 16 * ch, carry, sc, neg_m, cs, pk);
+            const bool below = kind == 1 || (kind == 0 && m < quarter);
+            lsum += p16_carry<MaskT>(sv, km_tile + 16 * ch, below ? keep_lo : keep_hi, k2, pk);
           }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) pk[e] = 0u;
         }
-        tmem_st8(s_base + 64u * hf + 8u * c, pk);
+        tmem_st16x2_8<8>(s_base + 16u * m, pk);
       }
       if (kAlibi) {
       } else if (kind == 1) {
@@ -929,30 +975,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.p_full[g & 1]);
 
-      // ---- the item's epilogue: this half of O / l, stored four rows at a time by each lane quad
+      // ---- the item's epilogue: O / l once its last PV has completed, stored four rows at a
+      // time by each lane quad (thread t: columns 0..63 of its row, thread t + 16: 64..127)
       if (last) {
         const int kb = items & 1;
-        sm.psum[kb][hf][r] = l;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.xsum[kb]);
-        const bool ok_sum = mbar_wait(&sm.xsum[kb], static_cast<uint32_t>(items >> 1) & 1u, abort_flag, err);
-        const bool ok_pv = ok_sum && mbar_wait(&sm.pv_done[g & 1], static_cast<uint32_t>(g >> 1) & 1u, abort_flag, err);
-        if (!__all_sync(0xffffffffu, ok_pv)) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.pv_done[g & 1], static_cast<uint32_t>(g >> 1) & 1u, abort_flag, err)))
+          break;
         tc_fence_after();
-        const float ltot = l + sm.psum[kb][hf ^ 1][r];
+        const float ltot = l + __shfl_xor_sync(0xffffffffu, l, 16);
         const int BT = prm.B * prm.T;
         const int hh = (H <= kMaxSortedHeads) ? static_cast<int>(sm.order[tx / BT]) : tx / BT;
         const int rem = tx % BT;
         const int bb = rem / prm.T, i0 = (rem % prm.T) * kTile;
         const float inv = 1.0f / ltot;
         const int p4 = lane & 3;
-        const int quad_row = quarter * 32 + (lane & ~3);  // first of the quad's four rows
-        const uint32_t o_half = tmem + lane_off + kColO + 128u * static_cast<uint32_t>(kb) + 64u * hf;
-        __nv_bfloat16* obase = O + (static_cast<size_t>(bb) * H + hh) * static_cast<size_t>(n) * kD + 64 * hf;
+        const int quad_row = quarter * 32 + hq * 16 + ((lane & 15) & ~3);  // first of the quad's four rows
+        const uint32_t o_row = tmem + lane_off + kColO + 128u * static_cast<uint32_t>(kb);
+        __nv_bfloat16* obase = O + (static_cast<size_t>(bb) * H + hh) * static_cast<size_t>(n) * kD + 64 * kh;
 #pragma unroll 1
         for (int blk = 0; blk < 2; ++blk) {
           uint32_t raw[32];
-          tmem_ld32(o_half + 32u * blk, raw);
+          tmem_ld16x2_32<64>(o_row + 32u * blk, raw);
           tmem_wait_ld();
           regs_after_wait(raw);
           uint32_t a[4][4];  // [16-byte chunk][word] of this row's 32 columns
@@ -988,7 +1031,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         }
         tc_fence_before();
         const int i = i0 + r;
-        if (hf == 0 && i < n)
+        if (kh == 0 && i < n)
           row_sum[(static_cast<size_t>(bb) * H + hh) * n + i] =
               (log2f(ltot) + m2) * 0.6931471805599453f - (kAlibi ? 0.0f : logf(static_cast<float>(s)));
         ++items;
