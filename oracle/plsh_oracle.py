@@ -13,7 +13,7 @@ Attention with Linear Biases"):
   [zh M1..M3], [ja M1..M3]: the same sections of the zh and ja pages, which
   agree with the nl page statement for statement.
 
-Readings taken where the pages are silent (each is repeated in the design doc):
+Readings taken where the pages are silent:
   * The hash is the Random Binning Features construction of Rahimi & Recht
     for the Laplace kernel, applied to integer positions [nl M1]: pitch
     delta ~ Gamma(shape 2, scale sigma) (the Gamma law the proof leans on,
@@ -108,7 +108,7 @@ def draw_table(seed: int, sigma: Sequence[float], s: int) -> np.ndarray:
     U1, U2, U3 are SplitMix64 outputs ((h << 16) | k) * 3 + {0, 1, 2}; the
     logarithm is the C library's (math.log), element by element.
     Pinned by: KS tests against the Gamma(2, sigma) and uniform laws, and the
-    first two moments, in tests/test_oracle_table.py.
+    first two moments (tests/oracle_pins.py: check_table_laws, check_table_moments).
     """
     if s < 1 or s > (1 << COUNTER_HEAD_SHIFT):
         raise ValueError("s out of range")
@@ -198,7 +198,8 @@ def boundary_bits(ids_hs: np.ndarray) -> np.ndarray:
 
     Bit k is set where hash k opens a new block. Because blocks are contiguous
     ([nl M1] structure), c_ij = s - popcount(OR_{min(i,j) < p <= max(i,j)} Bm(p)).
-    Pinned by: that identity against match_counts, in tests/test_oracle_masks.py.
+    Pinned by: that identity against match_counts (tests/oracle_pins.py:
+    check_boundary_identity) and hand-worked bits (check_bins_worked).
     """
     s, n = ids_hs.shape
     bits = np.zeros(n, dtype=np.uint64)
@@ -347,7 +348,13 @@ def forward(Q: np.ndarray, K: np.ndarray, V: np.ndarray, table: np.ndarray, caus
 
 def forward_exact(Q: np.ndarray, K: np.ndarray, V: np.ndarray, sigma: Sequence[float],
                   causal: bool, rows: Optional[Sequence[int]] = None) -> np.ndarray:
-    """Multi-head exact ALiBi T*, same layout as forward()."""
+    """Multi-head exact ALiBi T*, same layout as forward() ([nl M1], [nl R]).
+
+    Query head h reads KV head h // (H / H_kv) and uses its own sigma_h.
+    Pinned by: torch SDPA's grouped-query attention with the additive bias
+    -|i-j|/sigma_h, and sampled rows against all rows (tests/oracle_pins.py:
+    check_forward_exact_gqa).
+    """
     B, H, n, d = Q.shape
     group = H // K.shape[1]
     nr = n if rows is None else len(rows)

@@ -400,6 +400,30 @@ def check_rows_and_gqa(orc, n=160, d=8):
         np.testing.assert_allclose(O[0, 2], O1, rtol=1e-13, atol=1e-13)
 
 
+def check_forward_exact_gqa(orc, n=140, d=8):
+    """Multi-head exact ALiBi T* with grouped KV heads equals torch SDPA's own grouped-query
+    attention (enable_gqa) with the additive bias -|i-j|/sigma_h per head ([nl M1]: ALiBi's bias
+    matrix); sampled rows equal the full computation's rows."""
+    r = np.random.default_rng(10)
+    B, H, Hkv = 2, 4, 2
+    Q = r.standard_normal((B, H, n, d))
+    K = r.standard_normal((B, Hkv, n, d))
+    V = r.standard_normal((B, Hkv, n, d))
+    sigma = [1.5, 4.0, 12.0, 40.0]
+    rows = [0, 3, 64, 139]
+    dist = np.abs(np.arange(n)[:, None] - np.arange(n)[None, :]).astype(float)
+    bias = np.stack([-dist / sg for sg in sigma])
+    for causal in (False, True):
+        O = orc.forward_exact(Q, K, V, sigma, causal)
+        mask = np.where(np.tril(np.ones((n, n))) > 0, bias, -np.inf) if causal else bias
+        want = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(Q), torch.from_numpy(K), torch.from_numpy(V),
+            attn_mask=torch.from_numpy(mask)[None], enable_gqa=True).numpy()
+        np.testing.assert_allclose(O, want, rtol=1e-10, atol=1e-12)
+        Orow = orc.forward_exact(Q, K, V, sigma, causal, rows)
+        np.testing.assert_allclose(Orow, O[:, :, rows], rtol=1e-13, atol=1e-13)
+
+
 # ---------------------------------------------------------------------------
 # Gradients
 # ---------------------------------------------------------------------------

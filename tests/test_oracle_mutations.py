@@ -192,6 +192,30 @@ _ORIG_GRAD = O.approx_attention_grad
 _ORIG_SAMPLED = O.approx_attention_grad_sampled
 
 
+def _forward_exact_wrong_gqa(Q, K, V, sigma, causal, rows=None):
+    B, H, n, d = Q.shape
+    Hkv = K.shape[1]
+    nr = n if rows is None else len(rows)
+    out = np.empty((B, H, nr, d))
+    for b in range(B):
+        for h in range(H):
+            out[b, h], _ = O.exact_attention(Q[b, h], K[b, h % Hkv], V[b, h % Hkv], float(sigma[h]), causal, rows)
+    return out
+
+
+def _forward_exact_sigma_of_kv_head(Q, K, V, sigma, causal, rows=None):
+    # the length scale of the KV head instead of the query head's own
+    B, H, n, d = Q.shape
+    group = H // K.shape[1]
+    nr = n if rows is None else len(rows)
+    out = np.empty((B, H, nr, d))
+    for b in range(B):
+        for h in range(H):
+            out[b, h], _ = O.exact_attention(Q[b, h], K[b, h // group], V[b, h // group],
+                                             float(sigma[(h // group) * group]), causal, rows)
+    return out
+
+
 def _sampled_reach_ignores_causal(q, k, v, do, ids_hs, causal, rows, keys, chunk=256):
     # collects dK, dV from the non-causal rows' P (rows above the key are skipped, but P is not causal)
     dq, _, _ = _ORIG_SAMPLED(q, k, v, do, ids_hs, causal, rows, keys, chunk)
@@ -211,6 +235,8 @@ MUTATIONS = [
     ("approx_attention", _approx_no_sqrt_d, [P.check_one_bin_dense]),
     ("alibi_matrix", _alibi_times_sigma, [P.check_tiny_attention, P.check_exact_alibi_sdpa]),
     ("forward", _forward_wrong_gqa, [P.check_rows_and_gqa]),
+    ("forward_exact", _forward_exact_wrong_gqa, [P.check_forward_exact_gqa]),
+    ("forward_exact", _forward_exact_sigma_of_kv_head, [P.check_forward_exact_gqa]),
     ("tile_spans", _spans_ignore_causal, [P.check_bins_worked]),
     ("bmax", _bmax_interior_only, [P.check_bins_worked]),
     ("varlen_spans", _varlen_union_window, [P.check_bins_worked, P.check_varlen_spans_from_blocks]),

@@ -89,6 +89,10 @@ def test_sampled_rows_and_gqa():
     P.check_rows_and_gqa(oracle)
 
 
+def test_exact_alibi_multi_head_gqa():
+    P.check_forward_exact_gqa(oracle)
+
+
 def test_gradients_match_autograd_of_log_count_bias():
     P.check_grad_autograd(oracle)
 
