@@ -2,10 +2,10 @@
 // then the launch. Every check that can be made on the host is made here,
 // before anything is enqueued.
 #include <cmath>
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
-#include <mutex>
 
 #include "plsh_internal.h"
 
@@ -48,6 +48,34 @@ using plsh::fail;
 extern "C" const char* plsh_last_error(void) { return plsh::g_last_error; }
 
 extern "C" int plsh_version(void) { return 100; }
+
+// ---------------------------------------------------------------- bounded waits (failure detection)
+
+namespace plsh {
+namespace {
+std::atomic<uint64_t> g_wait_limit_ns{0};  // 0: the kernel's default
+std::atomic<int> g_withhold_mma{0};
+}  // namespace
+
+uint64_t wait_limit_ns() {
+  const uint64_t v = g_wait_limit_ns.load(std::memory_order_relaxed);
+  return v ? v : plsh::kDefaultWaitLimitNs;
+}
+bool withhold_mma() { return g_withhold_mma.load(std::memory_order_relaxed) != 0; }
+}  // namespace plsh
+
+extern "C" int plsh_set_wait_limit_ns(uint64_t limit_ns) {
+  if (limit_ns > PLSH_MAX_WAIT_LIMIT_NS)
+    return fail(PLSH_ERR_RANGE, "plsh_set_wait_limit_ns: %llu ns exceeds the maximum %llu ns",
+                static_cast<unsigned long long>(limit_ns), static_cast<unsigned long long>(PLSH_MAX_WAIT_LIMIT_NS));
+  plsh::g_wait_limit_ns.store(limit_ns, std::memory_order_relaxed);
+  return PLSH_OK;
+}
+
+extern "C" int plsh_test_withhold_mma(int on) {
+  plsh::g_withhold_mma.store(on ? 1 : 0, std::memory_order_relaxed);
+  return PLSH_OK;
+}
 
 extern "C" int plsh_sample_bins(const double* table_dev, int H, int s, int n, int32_t* ids_dev,
                                 uint32_t* err_dev, void* stream) {
@@ -172,25 +200,14 @@ namespace {
 // kernel before the attention kernel reads it, so nothing in it needs to start at zero.
 static __device__ __align__(256) int32_t g_varlen_static_scratch[PLSH_VARLEN_STATIC_SCRATCH_BYTES / sizeof(int32_t)];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_static_mutex;
-void* g_static_ptr[kMaxDevices] = {};
-
-// The buffer's device address on the current device, looked up once per device (with that
-// device current) and cached.
-int static_scratch_ptr(const char* fn, void** out) {
-  int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  if (dev < 0 || dev >= kMaxDevices) return fail(PLSH_ERR_RANGE, "%s: device ordinal %d not supported", fn, dev);
-  std::lock_guard<std::mutex> lock(g_static_mutex);
-  if (!g_static_ptr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_varlen_static_scratch);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(g_varlen_static_scratch)");
-    g_static_ptr[dev] = p;
-  }
-  *out = g_static_ptr[dev];
+// The buffer's device address in the current context. Looked up on every call rather than
+// cached: the lookup allocates nothing, and a cached address would outlive a reset or re-created
+// context, after which the module (and the buffer) may sit elsewhere.
+int static_scratch_ptr(void** out) {
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_varlen_static_scratch);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(g_varlen_static_scratch)");
+  *out = p;
   return PLSH_OK;
 }
 
@@ -214,7 +231,7 @@ extern "C" int plsh_attention_varlen_fwd_static(const void* Q, const void* K, co
                 "static buffer; use plsh_attention_varlen_fwd with caller scratch",
                 fn, need, static_cast<size_t>(PLSH_VARLEN_STATIC_SCRATCH_BYTES));
   void* scratch = nullptr;
-  if (int rc = plsh::static_scratch_ptr(fn, &scratch)) return rc;
+  if (int rc = plsh::static_scratch_ptr(&scratch)) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int32_t* spans = static_cast<int32_t*>(scratch);
   if (int rc = plsh::launch_varlen_spans(ids_dev, H, s, n, causal, spans, st)) return rc;

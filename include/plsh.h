@@ -22,8 +22,7 @@
  *   - "_dev" pointers are device memory owned by the caller; "_host"
  *     pointers are host memory owned by the caller. The library allocates
  *     no device memory and keeps no state between calls except the
- *     thread-local error string, a cached driver entry point and, for
- *     plsh_attention_varlen_fwd_static, the cached address of its buffer.
+ *     thread-local error string and a cached driver entry point.
  *   - Device work is enqueued on `stream` (a cudaStream_t passed as void*,
  *     NULL = legacy default stream) and is asynchronous: no entry point
  *     synchronises the device.
@@ -79,6 +78,31 @@ PLSH_API const char* plsh_last_error(void);
 PLSH_API int plsh_version(void);
 
 /*
+ * Failure detection of the fused attention kernel. The pages have no
+ * counterpart: these govern how the kernel gives up, not what it computes.
+ *
+ * Every wait of the tensor-core attention kernel (plsh_attention_fwd,
+ * plsh_attention_varlen_fwd[_static], plsh_alibi_banded_fwd with bf16,
+ * d = 128) on one of its roles is bounded in wall-clock time. A wait that runs
+ * out sets PLSH_DEVERR_TIMEOUT in err_dev; every role then leaves its loop,
+ * copies and tensor-core operations already in flight are drained (with a
+ * separate limit of 0.1 s), Tensor Memory is freed and the kernel returns, so
+ * the context stays usable. The outputs of such a launch are unspecified.
+ *
+ * plsh_set_wait_limit_ns -- the limit for launches made after the call, in
+ *   every host thread. 0 restores the default (2 s); above
+ *   PLSH_MAX_WAIT_LIMIT_NS (60 s) returns PLSH_ERR_RANGE and changes nothing.
+ *
+ * plsh_test_withhold_mma -- test hook: while `on` is nonzero, the kernel's
+ *   tensor-core issuer issues nothing, so every wait for a tile of scores runs
+ *   out after the wait limit. For testing the failure path only (pair it with
+ *   a short limit); off by default.
+ */
+#define PLSH_MAX_WAIT_LIMIT_NS 60000000000ull
+PLSH_API int plsh_set_wait_limit_ns(uint64_t limit_ns);
+PLSH_API int plsh_test_withhold_mma(int on);
+
+/*
  * plsh_draw_table -- the (delta, u) table of s random binnings per head, on
  * the host.
  *
@@ -99,6 +123,22 @@ PLSH_API int plsh_version(void);
  * Pure host code; needs no GPU.
  */
 PLSH_API int plsh_draw_table(uint64_t seed, int H, int s, const double* sigma_host, double* table_host);
+
+/*
+ * plsh_draw_table_heads -- rows h0 .. h0 + H - 1 of the table plsh_draw_table
+ * would draw for a larger head count: row h comes from the counters of head
+ * h0 + h, so the slices that the ranks of a head partition draw concatenate,
+ * bit for bit, to the whole table. (The pages shard nothing; this only lets a
+ * problem be split over devices by heads.)
+ *
+ *   h0          first global head, >= 0, with h0 + H <= PLSH_MAX_HEADS.
+ *   H, s, sigma_host, table_host   as plsh_draw_table, for the H heads of the
+ *               slice (sigma_host[h] belongs to global head h0 + h).
+ * Pure host code; needs no GPU.
+ */
+#define PLSH_MAX_HEADS 65536
+PLSH_API int plsh_draw_table_heads(uint64_t seed, int h0, int H, int s, const double* sigma_host,
+                                   double* table_host);
 
 /*
  * plsh_sample_bins (K1) -- bin ids of every (head, hash, position).
@@ -173,7 +213,11 @@ PLSH_API int plsh_window_from_table(const double* table_dev, int H, int s, int n
  *   dtype          PLSH_BF16 (bf16 in and out, fp32 accumulation, tcgen05
  *                  tensor cores when d == 128) or PLSH_F32 (fp32 in and out,
  *                  fp32 CUDA-core arithmetic).
- *   d              64 or 128.
+ *   d              64 or 128. bf16 with d == 64 is served by the CUDA-core
+ *                  kernel on purpose: the bf16 inputs are widened to fp32 and
+ *                  the result is rounded to bf16 once, so it meets the bf16
+ *                  tolerance with room to spare, but it runs at CUDA-core
+ *                  speed (the tensor-core kernel is built for d == 128).
  *   sigma_dev      [H] doubles, the ALiBi length scales the table was drawn
  *                  for; checked finite and > 0 (PLSH_DEVERR_SIGMA). May be NULL.
  *   s              hashes per head, as given to plsh_window.
@@ -260,9 +304,11 @@ PLSH_API int plsh_attention_varlen_fwd(const void* Q, const void* K, const void*
  *   and scratch_bytes.
  *   Limit: 8 * H * s * ceil(n/128) <= PLSH_VARLEN_STATIC_SCRATCH_BYTES, else
  *   PLSH_ERR_RANGE with nothing launched (H=16, s=20 fits up to n = 209,664).
- *   The first call on a device looks the buffer's address up
- *   (cudaGetSymbolAddress, with that device current) and caches it; make that
- *   first call before any stream capture. Calls that overlap on one device
+ *   Every call looks the buffer's address up in the current context
+ *   (cudaGetSymbolAddress, which allocates nothing), so a reset or re-created
+ *   context never leaves a stale address behind; the first call in a context
+ *   also loads the library's module there, so make it before any stream
+ *   capture. Calls that overlap on one device
  *   (on different streams, or from different host threads without ordering)
  *   share the buffer and race: order them, or use plsh_attention_varlen_fwd.
  */

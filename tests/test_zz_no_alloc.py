@@ -57,3 +57,68 @@ def test_static_buffer_refuses_oversize_before_launch():
     assert ei.value.code == 3
     assert "static buffer" in str(ei.value)
     torch.cuda.synchronize()
+
+
+def _static_call(plan, q, k, v, B, H, H_kv, n, d, s, causal, O, R):
+    from alibi_positional_lsh_b200 import plsh_attention_varlen_fwd_static
+    plsh_attention_varlen_fwd_static(q, k, v, plan.dtype_code, B, H, H_kv, n, d, plan.sigma_dev, s,
+                                     plan.table_dev, plan.ids, plan.bmask, int(causal), O, R, plan.err)
+
+
+def test_static_buffer_call_allocates_nothing():
+    """After a first call (which loads the module in this context), a call changes neither the
+    bytes torch has allocated nor the device's free bytes."""
+    from alibi_positional_lsh_b200 import PlshForward
+    B, H, H_kv, n, d, s, causal = 1, 2, 1, 900, 128, 20, True
+    w = workloads.Workload("case", B, H, H_kv, n, d, "bf16", causal, s, 77)
+    q, k, v = (t.cuda() for t in workloads.make_qkv(w))
+    plan = PlshForward(B, H, H_kv, n, d, s, causal, [3.0, 40.0], 5, torch.bfloat16, "cuda:0")
+    plan.prepare()
+    plan.ensure_ids()
+    O = torch.empty_like(q)
+    R = torch.empty((B, H, n), dtype=torch.float32, device="cuda:0")
+    _static_call(plan, q, k, v, B, H, H_kv, n, d, s, causal, O, R)
+    torch.cuda.synchronize()
+    alloc0, free0 = torch.cuda.memory_allocated(), torch.cuda.mem_get_info()[0]
+    for _ in range(3):
+        _static_call(plan, q, k, v, B, H, H_kv, n, d, s, causal, O, R)
+    torch.cuda.synchronize()
+    assert torch.cuda.memory_allocated() == alloc0
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert plan.device_errors() == []
+
+
+def test_static_buffer_exact_limit_accepted_one_tile_more_refused():
+    """8 H s ceil(n/128) equal to the buffer size runs and matches the caller-scratch entry point;
+    one query tile more is refused with PLSH_ERR_RANGE before any launch."""
+    from alibi_positional_lsh_b200 import (PLSH_BF16, PLSH_VARLEN_STATIC_SCRATCH_BYTES, PlshError, PlshForward,
+                                           plsh_attention_varlen_fwd_static, plsh_varlen_scratch_bytes)
+    B, H, H_kv, d, s, causal = 1, 8, 8, 128, 64, True
+    n = (PLSH_VARLEN_STATIC_SCRATCH_BYTES // (8 * H * s)) * 128
+    assert plsh_varlen_scratch_bytes(H, s, n) == PLSH_VARLEN_STATIC_SCRATCH_BYTES
+    g = torch.Generator(device="cuda:0").manual_seed(3)
+    q = torch.randn((B, H, n, d), generator=g, device="cuda:0").to(torch.bfloat16)
+    k = torch.randn((B, H_kv, n, d), generator=g, device="cuda:0").to(torch.bfloat16)
+    v = torch.randn((B, H_kv, n, d), generator=g, device="cuda:0").to(torch.bfloat16)
+    # short length scales: every hash's blocks are a few positions long, so the comparator's
+    # 64 passes per query tile stay near the diagonal
+    plan = PlshForward(B, H, H_kv, n, d, s, causal, [0.7 + 0.3 * h for h in range(H)], 11, torch.bfloat16, "cuda:0")
+    plan.prepare()
+    O_ref, R_ref = (t.clone() for t in plan.attend_varlen(q, k, v))
+    O = torch.full_like(O_ref, float("nan"))
+    R = torch.full_like(R_ref, float("nan"))
+    _static_call(plan, q, k, v, B, H, H_kv, n, d, s, causal, O, R)
+    torch.cuda.synchronize()
+    assert torch.equal(O, O_ref)
+    assert torch.equal(R, R_ref)
+    assert plan.device_errors() == []
+    # one more query tile: refused on the host, nothing launched (stand-in buffers are never touched)
+    n2 = n + 1
+    assert plsh_varlen_scratch_bytes(H, s, n2) > PLSH_VARLEN_STATIC_SCRATCH_BYTES
+    t = torch.zeros((256,), dtype=torch.bfloat16, device="cuda:0")
+    i = torch.zeros((256,), dtype=torch.int32, device="cuda:0")
+    f = torch.zeros((256,), dtype=torch.float32, device="cuda:0")
+    with pytest.raises(PlshError) as ei:
+        plsh_attention_varlen_fwd_static(t, t, t, PLSH_BF16, B, H, H_kv, n2, d, None, s, None, i, i, 1, t, f, i)
+    assert ei.value.code == 3
+    torch.cuda.synchronize()
