@@ -44,8 +44,14 @@ def _load() -> ctypes.CDLL:
     lib.plsh_last_error.argtypes = []
     lib.plsh_version.restype = i32
     lib.plsh_version.argtypes = []
+    lib.plsh_set_wait_limit_ns.restype = i32
+    lib.plsh_set_wait_limit_ns.argtypes = [u64]
+    lib.plsh_test_withhold_mma.restype = i32
+    lib.plsh_test_withhold_mma.argtypes = [i32]
     lib.plsh_draw_table.restype = i32
     lib.plsh_draw_table.argtypes = [u64, i32, i32, dp, dp]
+    lib.plsh_draw_table_heads.restype = i32
+    lib.plsh_draw_table_heads.argtypes = [u64, i32, i32, i32, dp, dp]
     lib.plsh_sample_bins.restype = i32
     lib.plsh_sample_bins.argtypes = [vp, i32, i32, i32, vp, vp, vp]
     lib.plsh_window.restype = i32
@@ -112,6 +118,14 @@ def plsh_version() -> int:
     return _lib.plsh_version()
 
 
+def plsh_set_wait_limit_ns(limit_ns: int) -> None:
+    _check(_lib.plsh_set_wait_limit_ns(ctypes.c_uint64(int(limit_ns))))
+
+
+def plsh_test_withhold_mma(on: bool) -> None:
+    _check(_lib.plsh_test_withhold_mma(1 if on else 0))
+
+
 def plsh_draw_table(seed: int, H: int, s: int, sigma_host: np.ndarray, table_host: np.ndarray) -> None:
     """Host call: fills table_host float64 [H][s][2] with (delta, u)."""
     sig = np.ascontiguousarray(sigma_host, dtype=np.float64)
@@ -121,6 +135,17 @@ def plsh_draw_table(seed: int, H: int, s: int, sigma_host: np.ndarray, table_hos
         raise ValueError("table_host must be a contiguous float64 array [H][s][2]")
     _check(_lib.plsh_draw_table(ctypes.c_uint64(seed & (2 ** 64 - 1)), H, s,
                                 sig.ctypes.data_as(ctypes.c_void_p), table_host.ctypes.data_as(ctypes.c_void_p)))
+
+
+def plsh_draw_table_heads(seed: int, h0: int, H: int, s: int, sigma_host: np.ndarray, table_host: np.ndarray) -> None:
+    """Host call: rows of global heads h0 .. h0 + H - 1 of the table, float64 [H][s][2]."""
+    sig = np.ascontiguousarray(sigma_host, dtype=np.float64)
+    if sig.shape != (H,):
+        raise ValueError("sigma_host must have shape [H]")
+    if table_host.dtype != np.float64 or table_host.shape != (H, s, 2) or not table_host.flags.c_contiguous:
+        raise ValueError("table_host must be a contiguous float64 array [H][s][2]")
+    _check(_lib.plsh_draw_table_heads(ctypes.c_uint64(seed & (2 ** 64 - 1)), h0, H, s,
+                                      sig.ctypes.data_as(ctypes.c_void_p), table_host.ctypes.data_as(ctypes.c_void_p)))
 
 
 def plsh_sample_bins(table_dev, H: int, s: int, n: int, ids_dev, err_dev, stream=None) -> None:
@@ -220,4 +245,4 @@ def decode_device_error(word: int) -> list:
     return [name for bit, name in DEVERR_BITS.items() if word & bit]
 
 
-from .api import HostPipeline, PlshForward, fixed_blocks_table, forward  # noqa: E402,F401
+from .api import HostPipeline, PlshForward, fixed_blocks_table, forward, head_partition  # noqa: E402,F401

@@ -142,6 +142,10 @@ struct Params {
   // window of a query tile reaches W_h = ceil(sigma_h ln(1/eps)) keys past its rows
   const double* sigma;
   double log_inv_eps;
+  // wall-clock limit of every barrier wait; for failure-detection tests, the MMA issuer can be
+  // told to issue nothing, so that every wait for a score tile runs out
+  uint64_t wait_ns;
+  int withhold_mma;
 };
 
 // Keys past which exp(-|i - j| / sigma) < eps, clamped to [0, n].
@@ -539,7 +543,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         const int zkv = ti.b * prm.H_kv + ti.h / (H / prm.H_kv);
         if (ti.first()) {
           const int qb = ti.k & 1;
-          if (ti.k >= 2 && !mbar_wait(&sm.q_empty[qb], ((ti.k >> 1) & 1) ^ 1, abort_flag, err)) break;
+          if (ti.k >= 2 && !mbar_wait(&sm.q_empty[qb], ((ti.k >> 1) & 1) ^ 1, abort_flag, err, prm.wait_ns)) break;
           mbar_arrive_expect_tx(&sm.q_full[qb], kTileBytes);
           tma_load_3d(sm.q[qb], &tmap_q, 0, ti.i0, ti.b * H + ti.h, &sm.q_full[qb]);
           tma_load_3d(sm.q[qb] + kChunkBytes, &tmap_q, 64, ti.i0, ti.b * H + ti.h, &sm.q_full[qb]);
@@ -548,12 +552,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         const int st = ti.g % kStages;
         const uint32_t ph = static_cast<uint32_t>(ti.g / kStages) & 1u;
         const int j0 = ti.j0();
-        if (ti.g >= kStages && !mbar_wait(&sm.k_empty[st], ph ^ 1u, abort_flag, err)) break;
+        if (ti.g >= kStages && !mbar_wait(&sm.k_empty[st], ph ^ 1u, abort_flag, err, prm.wait_ns)) break;
         mbar_arrive_expect_tx(&sm.k_full[st], kTileBytes);
         tma_load_3d(sm.k[st], &tmap_k, 0, j0, zkv, &sm.k_full[st]);
         tma_load_3d(sm.k[st] + kChunkBytes, &tmap_k, 64, j0, zkv, &sm.k_full[st]);
         issued_g = ti.g + 1;
-        if (ti.g >= kStages && !mbar_wait(&sm.v_empty[st], ph ^ 1u, abort_flag, err)) break;
+        if (ti.g >= kStages && !mbar_wait(&sm.v_empty[st], ph ^ 1u, abort_flag, err, prm.wait_ns)) break;
         mbar_arrive_expect_tx(&sm.v_full[st], kTileBytes);
         tma_load_3d(sm.v[st], &tmap_v, 0, j0, zkv, &sm.v_full[st]);
         tma_load_3d(sm.v[st] + kChunkBytes, &tmap_v, 64, j0, zkv, &sm.v_full[st]);
@@ -586,9 +590,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       }
       auto issue_s = [&](const TileIter<kVarlen, kAlibi>& ti) -> bool {
         const int qb = ti.k & 1;
-        if (ti.first() && !mbar_wait(&sm.q_full[qb], (ti.k >> 1) & 1, abort_flag, err)) return false;
+        if (ti.first() && !mbar_wait(&sm.q_full[qb], (ti.k >> 1) & 1, abort_flag, err, prm.wait_ns)) return false;
         const int st = ti.g % kStages;
-        if (!mbar_wait(&sm.k_full[st], static_cast<uint32_t>(ti.g / kStages) & 1u, abort_flag, err)) return false;
+        if (!mbar_wait(&sm.k_full[st], static_cast<uint32_t>(ti.g / kStages) & 1u, abort_flag, err, prm.wait_ns)) return false;
         tc_fence_after();
         const uint32_t d_tmem = tmem + kColS + 128u * static_cast<uint32_t>(ti.g & 1);
 #pragma unroll
@@ -605,8 +609,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       };
       auto issue_pv = [&](const TileIter<kVarlen, kAlibi>& ti) -> bool {
         const int st = ti.g % kStages;
-        if (!mbar_wait(&sm.p_full[ti.g & 1], static_cast<uint32_t>(ti.g >> 1) & 1u, abort_flag, err)) return false;
-        if (!mbar_wait(&sm.v_full[st], static_cast<uint32_t>(ti.g / kStages) & 1u, abort_flag, err)) return false;
+        if (!mbar_wait(&sm.p_full[ti.g & 1], static_cast<uint32_t>(ti.g >> 1) & 1u, abort_flag, err, prm.wait_ns)) return false;
+        if (!mbar_wait(&sm.v_full[st], static_cast<uint32_t>(ti.g / kStages) & 1u, abort_flag, err, prm.wait_ns)) return false;
         tc_fence_after();
         const uint32_t p_tmem = tmem + kColS + 128u * static_cast<uint32_t>(ti.g & 1);
         const uint32_t o_tmem = tmem + kColO + 128u * static_cast<uint32_t>(ti.k & 1);
@@ -625,6 +629,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       TileIter<kVarlen, kAlibi> cur, nxt;
       cur.start(&prm, sm.order);
       nxt.start(&prm, sm.order);
+      if (prm.withhold_mma) cur.valid = nxt.valid = false;  // failure-detection tests only
       bool ok = !cur.valid || issue_s(cur);
       if (nxt.valid) nxt.next();
       while (ok && cur.valid) {
@@ -648,7 +653,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       while (ti.valid) {
         const int st = ti.g % kMaskStages;
         if (ti.g >= kMaskStages) {
-          ok = mbar_wait(&sm.m_empty[st], (static_cast<uint32_t>(ti.g / kMaskStages) & 1u) ^ 1u, abort_flag, err);
+          ok = mbar_wait(&sm.m_empty[st], (static_cast<uint32_t>(ti.g / kMaskStages) & 1u) ^ 1u, abort_flag, err, prm.wait_ns);
           if (!__all_sync(0xffffffffu, ok)) {
             ok = false;
             break;
@@ -671,7 +676,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       if (ok && !*abort_flag) {
         const int st = g_end % kMaskStages;
         ok = g_end < kMaskStages ||
-             mbar_wait(&sm.m_empty[st], (static_cast<uint32_t>(g_end / kMaskStages) & 1u) ^ 1u, abort_flag, err);
+             mbar_wait(&sm.m_empty[st], (static_cast<uint32_t>(g_end / kMaskStages) & 1u) ^ 1u, abort_flag, err, prm.wait_ns);
         if (__all_sync(0xffffffffu, ok) && lane == 0) {
           sm.m[st].valid = 0;
           mbar_arrive(&sm.m_full[st]);
@@ -704,7 +709,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       MaskT nv[4] = {FULL, FULL, FULL, FULL}, n128 = FULL;
       if (nx.valid) load_masks(nx, nv, n128);  // lands while this tile is processed
       if (ti.g >= kMaskStages) {
-        ok = mbar_wait(&sm.m_empty[st], (static_cast<uint32_t>(ti.g / kMaskStages) & 1u) ^ 1u, abort_flag, err);
+        ok = mbar_wait(&sm.m_empty[st], (static_cast<uint32_t>(ti.g / kMaskStages) & 1u) ^ 1u, abort_flag, err, prm.wait_ns);
         if (!__all_sync(0xffffffffu, ok)) {
           ok = false;
           break;
@@ -797,7 +802,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     if (ok && !*abort_flag) {
       const int st = g_end % kMaskStages;
       ok = g_end < kMaskStages ||
-           mbar_wait(&sm.m_empty[st], (static_cast<uint32_t>(g_end / kMaskStages) & 1u) ^ 1u, abort_flag, err);
+           mbar_wait(&sm.m_empty[st], (static_cast<uint32_t>(g_end / kMaskStages) & 1u) ^ 1u, abort_flag, err, prm.wait_ns);
       if (__all_sync(0xffffffffu, ok) && lane == 0) {
         sm.m[st].valid = 0;
         mbar_arrive(&sm.m_full[st]);
@@ -826,7 +831,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     for (int g = 0;; ++g) {
       const int st = g % kMaskStages;
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.m_full[st], static_cast<uint32_t>(g / kMaskStages) & 1u,
-                                             abort_flag, err)))
+                                             abort_flag, err, prm.wait_ns)))
         break;
       const MaskStage<MaskT>& ms = sm.m[st];
       if (!ms.valid) break;
@@ -844,7 +849,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       // weights that need only the masks: the diagonal's own block and its carries
       MaskT lo = 0, hi = 0;
       if (!kAlibi && kind == 0) diag_scan<MaskT, kCausal>(ms, quarter, r, sw, &sm.cw[0][threadIdx.x], kSoftmaxWarps * 32, lo, hi);
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[g & 1], static_cast<uint32_t>(g >> 1) & 1u, abort_flag, err)))
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[g & 1], static_cast<uint32_t>(g >> 1) & 1u, abort_flag, err, prm.wait_ns)))
         break;
       tc_fence_after();
       const uint32_t s_base = tmem + lane_off + kColS + 128u * static_cast<uint32_t>(g & 1);
@@ -905,7 +910,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       const float neg_m = -m2;
       if (__any_sync(0xffffffffu, need_rescale)) {
         if (!__all_sync(0xffffffffu, mbar_wait(&sm.pv_done[(g - 1) & 1], static_cast<uint32_t>((g - 1) >> 1) & 1u,
-                                               abort_flag, err)))
+                                               abort_flag, err, prm.wait_ns)))
           break;
         tc_fence_after();
         // thread t: columns [16 q4, 16 q4 + 16), thread t + 16 the same 64 columns further
@@ -979,7 +984,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       // time by each lane quad (thread t: columns 0..63 of its row, thread t + 16: 64..127)
       if (last) {
         const int kb = items & 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(&sm.pv_done[g & 1], static_cast<uint32_t>(g >> 1) & 1u, abort_flag, err)))
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.pv_done[g & 1], static_cast<uint32_t>(g >> 1) & 1u, abort_flag, err, prm.wait_ns)))
           break;
         tc_fence_after();
         const float ltot = l + __shfl_xor_sync(0xffffffffu, l, 16);
@@ -1106,6 +1111,8 @@ int launch_tc_typed(const AttnArgs& a, cudaStream_t st) {
   prm.spans = a.spans;
   prm.sigma = a.sigma;
   prm.log_inv_eps = a.log_inv_eps;
+  prm.wait_ns = wait_limit_ns();
+  prm.withhold_mma = withhold_mma() ? 1 : 0;
   auto kern = attn_tc_kernel<MaskT, kCausal, kVarlen, kAlibi>;
   const size_t smem = sizeof(TcSmem<MaskT>) + 1024;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));

@@ -16,6 +16,12 @@ int cuda_fail(cudaError_t e, const char* what);
 
 inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
+// Process-wide settings of the fused attention kernel's bounded waits (plsh_set_wait_limit_ns,
+// plsh_test_withhold_mma), read at each launch.
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
+uint64_t wait_limit_ns();
+bool withhold_mma();
+
 // Kernel launchers (each returns PLSH_OK or an error code; arguments are
 // already validated by the entry point).
 int launch_sample_bins(const double* table, int H, int s, int n, int32_t* ids, uint32_t* err,

@@ -73,22 +73,23 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wall-clock limit of every barrier wait. A wait that runs out sets
-// PLSH_DEVERR_TIMEOUT in the error word and raises the CTA's abort flag so
-// every role leaves its loop; the kernel then drains and returns.
+// Default wall-clock limit of every barrier wait (the caller can set another
+// per launch). A wait that runs out sets PLSH_DEVERR_TIMEOUT in the error word
+// and raises the CTA's abort flag so every role leaves its loop; the kernel
+// then drains and returns.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-// Waits for the phase of parity `parity` to complete. Returns false if the
-// limit ran out or another role aborted.
+// Waits for the phase of parity `parity` to complete. Returns false if
+// `limit_ns` ran out or another role aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          uint32_t* err) {
+                                          uint32_t* err, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 63u) == 0) {
       if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         atomicOr(err, PLSH_DEVERR_TIMEOUT);
         return false;

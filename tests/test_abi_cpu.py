@@ -177,3 +177,14 @@ def test_window_from_table_rejects_bad_arguments_before_any_launch(plsh):
     assert lib.plsh_window_from_table(fake, 1, 0, 100, 0, fake, fake, fake, fake, null) == 1
     assert lib.plsh_window_from_table(fake, 1, 65, 100, 0, fake, fake, fake, fake, null) == 1
     assert lib.plsh_window_from_table(fake, 0, 4, 100, 0, fake, fake, fake, fake, null) == 1
+
+
+def test_wait_limit_setting_checks_its_range(plsh):
+    from alibi_positional_lsh_b200 import PlshError, plsh_set_wait_limit_ns, plsh_test_withhold_mma
+    plsh_set_wait_limit_ns(5_000_000)
+    plsh_set_wait_limit_ns(0)          # back to the default
+    with pytest.raises(PlshError) as ei:
+        plsh_set_wait_limit_ns(61_000_000_000)
+    assert ei.value.code == 3
+    plsh_test_withhold_mma(True)
+    plsh_test_withhold_mma(False)
