@@ -22,8 +22,8 @@ import torch
 
 from . import (PLSH_BF16, PLSH_F32, PLSH_TILE, PlshError, decode_device_error, plsh_alibi_banded_fwd,
                plsh_attention_bwd, plsh_attention_fwd, plsh_attention_varlen_fwd, plsh_decode_fwd,
-               plsh_decode_scratch_bytes, plsh_draw_table, plsh_sample_bins, plsh_window_from_table,
-               plsh_varlen_scratch_bytes)
+               plsh_decode_scratch_bytes, plsh_draw_table_heads, plsh_sample_bins,
+               plsh_window_from_table, plsh_varlen_scratch_bytes)
 
 
 class PlshForward:
@@ -31,12 +31,16 @@ class PlshForward:
 
     def __init__(self, B: int, H: int, H_kv: int, n: int, d: int, s: int, causal: bool,
                  sigma: Sequence[float], seed: int, dtype: torch.dtype = torch.bfloat16,
-                 device: str = "cuda"):
+                 device: str = "cuda", head_offset: int = 0):
+        """head_offset: the plan's heads are global heads head_offset .. head_offset + H - 1 of a
+        larger problem (a slice of a head partition, see head_partition): its table rows are drawn
+        from those heads' counters, so the slices of all ranks make up the whole problem's table."""
         if dtype not in (torch.bfloat16, torch.float32):
             raise ValueError("dtype must be torch.bfloat16 or torch.float32")
         self.B, self.H, self.H_kv, self.n, self.d, self.s = B, H, H_kv, n, d, s
         self.causal = bool(causal)
         self.seed = int(seed)
+        self.head_offset = int(head_offset)
         self.dtype = dtype
         self.dtype_code = PLSH_BF16 if dtype == torch.bfloat16 else PLSH_F32
         self.device = torch.device(device)
@@ -67,7 +71,7 @@ class PlshForward:
         if self._table_copied is not None:
             self._table_copied.synchronize()   # the pinned buffer may still be in flight
         if table is None:
-            plsh_draw_table(self.seed, self.H, self.s, self.sigma_host, self.table_host.numpy())
+            plsh_draw_table_heads(self.seed, self.head_offset, self.H, self.s, self.sigma_host, self.table_host.numpy())
         else:
             t = np.ascontiguousarray(table, dtype=np.float64)
             if t.shape != (self.H, self.s, 2):
@@ -286,6 +290,24 @@ class HostPipeline:
         st = torch.cuda.current_stream() if stream is None else stream
         for t in range(max(0, self.t - 2), self.t):
             st.wait_event(self.copied_out[t % 2])
+
+
+def head_partition(H: int, H_kv: int, world: int, rank: int) -> Tuple[int, int]:
+    """Query heads [h0, h1) of `rank` when one problem is split over `world` devices by heads.
+
+    Whole GQA groups stay together: the KV heads are dealt out as evenly as possible (the first
+    H_kv % world ranks take one more), and each rank takes the query heads that read its KV
+    heads. Every (batch, head) is independent given the table, so the ranks exchange nothing;
+    with head_offset=h0 each rank's PlshForward draws exactly its rows of the whole table.
+    A rank left without KV heads (world > H_kv) gets an empty range.
+    """
+    if H_kv < 1 or H % H_kv or world < 1 or not 0 <= rank < world:
+        raise ValueError("need H_kv >= 1 dividing H and 0 <= rank < world")
+    group = H // H_kv
+    base, extra = divmod(H_kv, world)
+    g0 = rank * base + min(rank, extra)
+    g1 = g0 + base + (1 if rank < extra else 0)
+    return g0 * group, g1 * group
 
 
 def fixed_blocks_table(H: int, block: float) -> np.ndarray:

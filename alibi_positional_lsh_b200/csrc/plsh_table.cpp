@@ -38,22 +38,26 @@ inline double unit_closed_open(uint64_t z) { return static_cast<double>(z >> 11)
 
 }  // namespace
 
-extern "C" int plsh_draw_table(uint64_t seed, int H, int s, const double* sigma_host,
-                               double* table_host) {
+// Rows of global heads h0 .. h0 + H - 1 of the table; row h is drawn from the counters of head
+// h0 + h, so the slices of a head partition concatenate to the whole table.
+static int draw_heads(const char* fn, uint64_t seed, int h0, int H, int s, const double* sigma_host,
+                      double* table_host) {
   if (H < 1 || s < 1 || s > PLSH_MAX_S)
-    return plsh::fail(PLSH_ERR_INVALID_ARG, "plsh_draw_table: need H >= 1 and 1 <= s <= %d (H=%d s=%d)",
-                      PLSH_MAX_S, H, s);
-  if (!sigma_host || !table_host)
-    return plsh::fail(PLSH_ERR_INVALID_ARG, "plsh_draw_table: null pointer");
+    return plsh::fail(PLSH_ERR_INVALID_ARG, "%s: need H >= 1 and 1 <= s <= %d (H=%d s=%d)", fn, PLSH_MAX_S, H, s);
+  if (h0 < 0 || static_cast<int64_t>(h0) + H > PLSH_MAX_HEADS)
+    return plsh::fail(PLSH_ERR_INVALID_ARG, "%s: need 0 <= h0 and h0 + H <= %d (h0=%d H=%d)", fn, PLSH_MAX_HEADS,
+                      h0, H);
+  if (!sigma_host || !table_host) return plsh::fail(PLSH_ERR_INVALID_ARG, "%s: null pointer", fn);
   for (int h = 0; h < H; ++h) {
     const double sg = sigma_host[h];
     if (!(std::isfinite(sg) && sg > 0.0))
-      return plsh::fail(PLSH_ERR_INVALID_ARG, "plsh_draw_table: sigma[%d] = %g is not finite and > 0", h, sg);
+      return plsh::fail(PLSH_ERR_INVALID_ARG, "%s: sigma[%d] = %g is not finite and > 0", fn, h, sg);
   }
   for (int h = 0; h < H; ++h) {
     const double neg_sigma = -sigma_host[h];
+    const uint64_t hg = static_cast<uint64_t>(h0) + static_cast<uint64_t>(h);
     for (int k = 0; k < s; ++k) {
-      const uint64_t base = ((static_cast<uint64_t>(h) << kHeadShift) | static_cast<uint64_t>(k)) * 3u;
+      const uint64_t base = ((hg << kHeadShift) | static_cast<uint64_t>(k)) * 3u;
       const double u1 = unit_open(splitmix64_output(seed, base));
       const double u2 = unit_open(splitmix64_output(seed, base + 1));
       const double u3 = unit_closed_open(splitmix64_output(seed, base + 2));
@@ -64,4 +68,13 @@ extern "C" int plsh_draw_table(uint64_t seed, int H, int s, const double* sigma_
     }
   }
   return PLSH_OK;
+}
+
+extern "C" int plsh_draw_table(uint64_t seed, int H, int s, const double* sigma_host, double* table_host) {
+  return draw_heads("plsh_draw_table", seed, 0, H, s, sigma_host, table_host);
+}
+
+extern "C" int plsh_draw_table_heads(uint64_t seed, int h0, int H, int s, const double* sigma_host,
+                                     double* table_host) {
+  return draw_heads("plsh_draw_table_heads", seed, h0, H, s, sigma_host, table_host);
 }
