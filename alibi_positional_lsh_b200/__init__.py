@@ -77,6 +77,9 @@ def _load() -> ctypes.CDLL:
     lib.plsh_attention_bwd.restype = i32
     lib.plsh_attention_bwd.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, i32, vp, vp,
                                        vp, vp, vp, vp]
+    lib.plsh_attention_bwd_tc.restype = i32
+    lib.plsh_attention_bwd_tc.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, i32,
+                                          vp, vp, vp, vp, vp, vp]
     lib.plsh_decode_fwd.restype = i32
     lib.plsh_decode_fwd.argtypes = [vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, i32, vp,
                                     ctypes.c_size_t, vp, vp, vp, vp]
@@ -239,6 +242,16 @@ def plsh_attention_bwd(Q, K, V, O, dO, row_sum, dtype: int, B: int, H: int, H_kv
                                    _dev_ptr(ids_dev, "ids_dev"), int(causal), _dev_ptr(delta_dev, "delta_dev"),
                                    _dev_ptr(dQ, "dQ"), _dev_ptr(dK, "dK"), _dev_ptr(dV, "dV"),
                                    _dev_ptr(err_dev, "err_dev"), _stream_ptr(stream)))
+
+
+def plsh_attention_bwd_tc(Q, K, V, O, dO, row_sum, B: int, H: int, H_kv: int, n: int, d: int, s: int, bmask_dev,
+                          tile_span_dev, key_span_dev, causal: int, delta_dev, dQ, dK, dV, err_dev, stream=None) -> None:
+    _check(_lib.plsh_attention_bwd_tc(_dev_ptr(Q, "Q"), _dev_ptr(K, "K"), _dev_ptr(V, "V"), _dev_ptr(O, "O"),
+                                      _dev_ptr(dO, "dO"), _dev_ptr(row_sum, "row_sum"), B, H, H_kv, n, d, s,
+                                      _dev_ptr(bmask_dev, "bmask_dev"), _dev_ptr(tile_span_dev, "tile_span_dev"),
+                                      _dev_ptr(key_span_dev, "key_span_dev"), int(causal),
+                                      _dev_ptr(delta_dev, "delta_dev"), _dev_ptr(dQ, "dQ"), _dev_ptr(dK, "dK"),
+                                      _dev_ptr(dV, "dV"), _dev_ptr(err_dev, "err_dev"), _stream_ptr(stream)))
 
 
 def decode_device_error(word: int) -> list:

@@ -21,7 +21,7 @@ import numpy as np
 import torch
 
 from . import (PLSH_BF16, PLSH_F32, PLSH_TILE, PlshError, decode_device_error, plsh_alibi_banded_fwd,
-               plsh_attention_bwd, plsh_attention_fwd, plsh_attention_varlen_fwd, plsh_decode_fwd,
+               plsh_attention_bwd, plsh_attention_bwd_tc, plsh_attention_fwd, plsh_attention_varlen_fwd, plsh_decode_fwd,
                plsh_decode_scratch_bytes, plsh_draw_table_heads, plsh_sample_bins,
                plsh_window_from_table, plsh_varlen_scratch_bytes)
 
@@ -63,6 +63,8 @@ class PlshForward:
         self.row_sum = torch.empty((B, H, n), dtype=torch.float32, device=dev)
         self.scratch = None  # per-hash windows of the comparator, allocated on first use
         self.grads = None    # (delta, dQ, dK, dV) of backward(), allocated on first use
+        self._kspans = None  # (non-causal windows, their b_max and masks) for the tensor-core backward
+        self._kspans_ok = False
         self.decode_scratch = None  # partial results of decode(), grown on demand
 
     # a1 + a2 + a3
@@ -85,6 +87,7 @@ class PlshForward:
         plsh_window_from_table(self.table_dev, self.H, self.s, self.n, int(self.causal), self.bmax, self.spans,
                                self.bmask, self.err, st)
         self._ids_ok = False
+        self._kspans_ok = False
 
     def ensure_ids(self, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
         """The bin ids [H][s][n] of the current table (K1, run on `stream` the first time they are needed).
@@ -148,9 +151,30 @@ class PlshForward:
                               int(self.causal), self.O, self.row_sum, self.err, st)
         return self.O, self.row_sum
 
+    def key_spans(self, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+        """[H][T][2] non-causal windows of the current table: by the symmetry of the counts, the query rows
+        that reach each 128-key tile (the windows themselves when the plan is not causal)."""
+        if not self.causal:
+            return self.spans
+        if not self._kspans_ok:
+            if self._kspans is None:
+                dev = self.O.device
+                T = self.spans.shape[1]
+                self._kspans = (torch.empty((self.H, T, 2), dtype=torch.int32, device=dev),
+                                torch.empty((self.H,), dtype=torch.int32, device=dev), torch.empty_like(self.bmask))
+            st = torch.cuda.current_stream() if stream is None else stream
+            spans, bmax, bmask = self._kspans
+            plsh_window_from_table(self.table_dev, self.H, self.s, self.n, 0, bmax, spans, bmask, self.err, st)
+            self._kspans_ok = True
+        return self._kspans[0]
+
     def backward(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dO: torch.Tensor,
-                 stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
-        """dQ, dK, dV of <dO, T~> for the inputs of the last attend() (its O and row_sum, the same table)."""
+                 stream: Optional[torch.cuda.Stream] = None,
+                 path: str = "auto") -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+        """dQ, dK, dV of <dO, T~> for the inputs of the last attend() (its O and row_sum, the same table).
+
+        path: "tc" the tcgen05 kernels (bf16, d = 128), "simt" the fp32 CUDA-core kernels, "auto" the
+        former where it applies."""
         B, H, H_kv, n, d = self.B, self.H, self.H_kv, self.n, self.d
         if q.shape != (B, H, n, d) or dO.shape != (B, H, n, d) or k.shape != (B, H_kv, n, d) \
                 or v.shape != (B, H_kv, n, d):
@@ -165,9 +189,15 @@ class PlshForward:
                           torch.empty((B, H_kv, n, d), dtype=self.dtype, device=dev))
         delta, dQ, dK, dV = self.grads
         st = torch.cuda.current_stream() if stream is None else stream
-        plsh_attention_bwd(q, k, v, self.O, dO, self.row_sum, self.dtype_code, B, H, H_kv, n, d, self.s,
-                           self.ensure_ids(st),
-                           int(self.causal), delta, dQ, dK, dV, self.err, st)
+        tc_ok = self.dtype == torch.bfloat16 and d == 128
+        if path not in ("auto", "tc", "simt") or (path == "tc" and not tc_ok):
+            raise ValueError("path must be 'auto', 'simt' or (bf16 with d = 128) 'tc'")
+        if path == "tc" or (path == "auto" and tc_ok):
+            plsh_attention_bwd_tc(q, k, v, self.O, dO, self.row_sum, B, H, H_kv, n, d, self.s, self.bmask, self.spans,
+                                  self.key_spans(st), int(self.causal), delta, dQ, dK, dV, self.err, st)
+        else:
+            plsh_attention_bwd(q, k, v, self.O, dO, self.row_sum, self.dtype_code, B, H, H_kv, n, d, self.s,
+                               self.ensure_ids(st), int(self.causal), delta, dQ, dK, dV, self.err, st)
         return dQ, dK, dV
 
     def decode(self, q_rows: torch.Tensor, pos: torch.Tensor, k: torch.Tensor, v: torch.Tensor,

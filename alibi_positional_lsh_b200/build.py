@@ -30,6 +30,7 @@ SOURCES = [
     "plsh_varlen.cu",
     "plsh_decode.cu",
     "plsh_bwd.cu",
+    "plsh_bwd_tc.cu",
 ]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

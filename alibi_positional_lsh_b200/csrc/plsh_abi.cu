@@ -319,3 +319,28 @@ extern "C" int plsh_attention_bwd(const void* Q, const void* K, const void* V, c
   plsh::BwdArgs a{Q, K, V, O, dO, row_sum, ids_dev, dtype, B, H, H_kv, n, d, s, causal, delta_dev, dQ, dK, dV};
   return plsh::launch_bwd(a, static_cast<cudaStream_t>(stream));
 }
+
+extern "C" int plsh_attention_bwd_tc(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                                     const float* row_sum, int B, int H, int H_kv, int n, int d, int s,
+                                     const void* bmask_dev, const int32_t* tile_span_dev,
+                                     const int32_t* key_span_dev, int causal, float* delta_dev, void* dQ, void* dK,
+                                     void* dV, uint32_t* err_dev, void* stream) {
+  const char* fn = "plsh_attention_bwd_tc";
+  if (int rc = plsh::check_sizes(fn, H, s, n)) return rc;
+  if (B < 1 || B > 65535) return fail(PLSH_ERR_INVALID_ARG, "%s: need 1 <= B <= 65535 (B=%d)", fn, B);
+  if (H_kv < 1 || H % H_kv != 0)
+    return fail(PLSH_ERR_INVALID_ARG, "%s: H_kv must divide H (H=%d H_kv=%d)", fn, H, H_kv);
+  if (causal != 0 && causal != 1) return fail(PLSH_ERR_INVALID_ARG, "%s: causal must be 0 or 1", fn);
+  if (d != 128) return fail(PLSH_ERR_UNSUPPORTED, "%s: head dim %d (the tensor-core backward needs 128)", fn, d);
+  if (!Q || !K || !V || !O || !dO || !row_sum || !bmask_dev || !tile_span_dev || !key_span_dev || !delta_dev || !dQ ||
+      !dK || !dV || !err_dev)
+    return fail(PLSH_ERR_INVALID_ARG, "%s: null pointer", fn);
+  if (!plsh::aligned16(Q) || !plsh::aligned16(K) || !plsh::aligned16(V) || !plsh::aligned16(O) ||
+      !plsh::aligned16(dO) || !plsh::aligned16(dQ) || !plsh::aligned16(dK) || !plsh::aligned16(dV))
+    return fail(PLSH_ERR_INVALID_ARG, "%s: Q, K, V, O, dO, dQ, dK and dV must be 16-byte aligned", fn);
+  if (static_cast<size_t>(B) * H * n > (size_t{1} << 31))
+    return fail(PLSH_ERR_RANGE, "%s: B*H*n exceeds 2^31", fn);
+  plsh::BwdTcArgs a{Q, K, V, O, dO, row_sum, bmask_dev, tile_span_dev, key_span_dev, B, H, H_kv, n, d, s, causal,
+                    delta_dev, dQ, dK, dV, err_dev};
+  return plsh::launch_bwd_tc(a, static_cast<cudaStream_t>(stream));
+}

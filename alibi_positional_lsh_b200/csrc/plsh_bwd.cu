@@ -456,6 +456,24 @@ int launch_bwd_typed(const BwdArgs& a, cudaStream_t st) {
 
 }  // namespace
 
+int launch_bwd_delta(const void* O, const void* dO, int dtype, int d, size_t rows, float* delta, cudaStream_t st) {
+  const unsigned blocks = static_cast<unsigned>((rows + kThreads / 32 - 1) / (kThreads / 32));
+  if (dtype == PLSH_F32) {
+    if (d == 64)
+      bwd_delta_kernel<float, 64><<<blocks, kThreads, 0, st>>>(static_cast<const float*>(O), static_cast<const float*>(dO), delta, rows);
+    else
+      bwd_delta_kernel<float, 128><<<blocks, kThreads, 0, st>>>(static_cast<const float*>(O), static_cast<const float*>(dO), delta, rows);
+  } else {
+    using bf = __nv_bfloat16;
+    if (d == 64)
+      bwd_delta_kernel<bf, 64><<<blocks, kThreads, 0, st>>>(static_cast<const bf*>(O), static_cast<const bf*>(dO), delta, rows);
+    else
+      bwd_delta_kernel<bf, 128><<<blocks, kThreads, 0, st>>>(static_cast<const bf*>(O), static_cast<const bf*>(dO), delta, rows);
+  }
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? PLSH_OK : cuda_fail(e, "bwd_delta_kernel launch");
+}
+
 int launch_bwd(const BwdArgs& a, cudaStream_t st) {
   if (a.dtype == PLSH_F32) return a.d == 64 ? launch_bwd_typed<float, 64>(a, st) : launch_bwd_typed<float, 128>(a, st);
   return a.d == 64 ? launch_bwd_typed<__nv_bfloat16, 64>(a, st) : launch_bwd_typed<__nv_bfloat16, 128>(a, st);

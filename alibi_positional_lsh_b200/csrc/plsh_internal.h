@@ -67,6 +67,20 @@ struct BwdArgs {
   void* dQ; void* dK; void* dV;
 };
 int launch_bwd(const BwdArgs& a, cudaStream_t st);
+// D_i = dO_i . O_i for `rows` rows of d elements (the backward's row dots).
+int launch_bwd_delta(const void* O, const void* dO, int dtype, int d, size_t rows, float* delta, cudaStream_t st);
+// Tensor-core backward (bf16, d = 128): masks and windows instead of ids. tile_spans are the forward's
+// windows (plsh_window with the same causal flag), key_spans the non-causal ones (the query rows that
+// reach each key tile, by the symmetry of c_ij).
+struct BwdTcArgs {
+  const void* Q; const void* K; const void* V; const void* O; const void* dO;
+  const float* row_sum; const void* bmask; const int32_t* tile_spans; const int32_t* key_spans;
+  int B, H, H_kv, n, d, s, causal;
+  float* delta;
+  void* dQ; void* dK; void* dV;
+  uint32_t* err;
+};
+int launch_bwd_tc(const BwdTcArgs& a, cudaStream_t st);
 int launch_varlen_spans(const int32_t* ids, int H, int s, int n, int causal, int32_t* spans, cudaStream_t st);
 int launch_attention_simt(const AttnArgs& a, cudaStream_t st);
 int launch_attention_tc(const AttnArgs& a, cudaStream_t st);

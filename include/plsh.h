@@ -421,6 +421,41 @@ PLSH_API int plsh_attention_bwd(const void* Q, const void* K, const void* V, con
                                 const int32_t* ids_dev, int causal, float* delta_dev, void* dQ, void* dK,
                                 void* dV, uint32_t* err_dev, void* stream);
 
+/*
+ * plsh_attention_bwd_tc -- the same gradients on the tcgen05 tensor cores,
+ * for bf16 inputs with d = 128 (else PLSH_ERR_UNSUPPORTED; use
+ * plsh_attention_bwd).
+ *
+ * Cites: as plsh_attention_bwd. The counts c_ij come from the boundary masks
+ * as in plsh_attention_fwd (Methodology 1, structure: contiguous blocks).
+ * S, dP and the gradient products run as bf16 MMAs with fp32 accumulation;
+ * P and dS are rounded to bf16 for the products, so the gradients meet a
+ * bf16 tolerance (they are not the fp32 path's results bit for bit).
+ *
+ *   Q, K, V, O, dO, row_sum, B, H, H_kv, n, s, causal   as plsh_attention_bwd
+ *                  (bf16 tensors).
+ *   bmask_dev      [H][n] boundary masks from plsh_window (or
+ *                  plsh_window_from_table) for this table.
+ *   tile_span_dev  [H][ceil(n/128)][2] windows from plsh_window with the same
+ *                  causal flag (the key range each 128-row query tile reaches).
+ *   key_span_dev   [H][ceil(n/128)][2] windows from plsh_window with
+ *                  causal = 0: by the symmetry of c_ij, the query rows that
+ *                  reach each 128-key tile (equal to tile_span_dev when
+ *                  causal = 0).
+ *   delta_dev      [B][H][n] float32 scratch (written: D_i).
+ *   dQ             [B][H][n][128] out; dK, dV [B][H_kv][n][128] out, each row
+ *                  written once.
+ *   err_dev        device error word: PLSH_DEVERR_WINDOW for a window that
+ *                  does not cover its tile, PLSH_DEVERR_TIMEOUT as for
+ *                  plsh_attention_fwd (same wait limit).
+ * Every pointer to a tensor must be 16-byte aligned.
+ */
+PLSH_API int plsh_attention_bwd_tc(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                                   const float* row_sum, int B, int H, int H_kv, int n, int d, int s,
+                                   const void* bmask_dev, const int32_t* tile_span_dev,
+                                   const int32_t* key_span_dev, int causal, float* delta_dev, void* dQ, void* dK,
+                                   void* dV, uint32_t* err_dev, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -174,3 +174,42 @@ def test_backward_mha8_sampled_non_causal():
         want[2].append(dv)
     _assert_grads(tuple(np.stack(x) for x in got), tuple(np.stack(x) for x in want), w.torch_dtype,
                   "backward mha8_n8192")
+
+
+# ---------------------------------------------------------------- the tcgen05 kernels (bf16, d = 128)
+
+TC_MORE = [
+    (1, 2, 1, 600, 128, torch.bfloat16, False, 20, "tiny"),
+    (1, 2, 1, 600, 128, torch.bfloat16, True, 20, "huge"),
+    (1, 2, 2, 129, 128, torch.bfloat16, False, 64, "mixed"),
+    (2, 4, 1, 1000, 128, torch.bfloat16, False, 40, "mixed"),
+    (1, 4, 2, 2000, 128, torch.bfloat16, True, 12, "mixed"),
+]
+
+
+@pytest.mark.parametrize("B,H,H_kv,n,d,dtype,causal,s,kind", TC_MORE,
+                         ids=[f"B{c[0]}H{c[1]}kv{c[2]}n{c[3]}{'c' if c[6] else 'nc'}s{c[7]}{c[8]}" for c in TC_MORE])
+def test_backward_tensor_cores_full_oracle(B, H, H_kv, n, d, dtype, causal, s, kind):
+    """bf16 with d = 128 takes the tcgen05 kernels (plsh_attention_bwd_tc): tiny and huge length
+    scales, 64-bit masks, grouped heads both ways, ragged n."""
+    (q, k, v, dO), plan, got = _run(B, H, H_kv, n, d, dtype, causal, s, _sigmas(kind, H), 900 + n + s)
+    want = oracle.backward(PH.f64(q), PH.f64(k), PH.f64(v), PH.f64(dO), plan.table_host.numpy(), causal)
+    _assert_grads(got, want, dtype, "backward tensor cores")
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_backward_tensor_cores_agree_with_cuda_core_path(causal):
+    """The tcgen05 kernels and the fp32 CUDA-core kernels on the same inputs: within the bf16 bar of
+    each other (both are within it of the oracle)."""
+    from alibi_positional_lsh_b200 import PlshForward
+    B, H, H_kv, n, d, s = 1, 4, 2, 3000, 128, 20
+    w = workloads.Workload("case", B, H, H_kv, n, d, "bf16", causal, s, 71)
+    q, k, v = (t.cuda() for t in workloads.make_qkv(w))
+    dO = _grad_out((B, H, n, d), torch.bfloat16, 72).cuda()
+    plan = PlshForward(B, H, H_kv, n, d, s, causal, _sigmas("mixed", H), 73, torch.bfloat16, "cuda:0")
+    plan(q, k, v)
+    tc = [t.double().clone() for t in plan.backward(q, k, v, dO, path="tc")]
+    simt = [t.double().clone() for t in plan.backward(q, k, v, dO, path="simt")]
+    assert plan.device_errors() == []
+    for name, a, b in zip(("dQ", "dK", "dV"), tc, simt):
+        assert float((a - b).abs().max()) <= 2e-2 * max(float(b.abs().max()), 1e-3), name
