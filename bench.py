@@ -300,40 +300,75 @@ def bwd_chunk_pairs(ids: np.ndarray, causal: bool, group: int) -> tuple:
     return dq, dkdv
 
 
-def bwd_timing(plan, q, k, v, stream, w, sm_count: int, sm_max_mhz: float):
-    """plsh_attention_bwd on the step's inputs with a seeded dO: device time per call and its issued fp32
-    FLOPs (per 64 x 64 pair: S, dP and dQ in the dQ kernel, S, dP, dV and dK in the dK/dV kernel, 2d each)
-    against the CUDA-core fp32 FMA peak derived from the SM count and the maximum SM clock."""
+def bwd_tc_tiles(spans: np.ndarray, key_spans: np.ndarray, causal: bool) -> tuple:
+    """(key tiles the tensor-core dQ kernel visits, query tiles the dK/dV kernel walks) for one batch
+    element. spans: the forward's windows [H][T][2]; key_spans: the non-causal ones (the query rows
+    that reach each key tile). The dK/dV kernel walks, per head and key tile, the key tile's own
+    tile, the tiles before it (non-causal only) and the tiles after it up to the window's end."""
+    dq = kernel_tiles(spans, causal)
+    H, T, _ = key_spans.shape
+    j0 = (np.arange(T) * TILE)[None, :]
+    lo = np.minimum(key_spans[..., 0].astype(np.int64), j0)
+    hi = key_spans[..., 1].astype(np.int64)
+    below = 0 if causal else (j0 - lo + TILE - 1) // TILE
+    dkdv = int(np.sum(1 + below + (hi - j0) // TILE))
+    return dq, dkdv
+
+
+def bwd_timing(plan, q, k, v, stream, w, sm_count: int, sm_max_mhz: float, bf16_peak: float):
+    """plsh_attention_bwd on the step's inputs with a seeded dO: device time per call of the tcgen05
+    kernels (bf16, d = 128) and of the fp32 CUDA-core kernels. The tensor-core roofline counts 3 MMAs
+    of 128 x 128 x 128 per dQ tile (S, dP, dQ += dS K) and 4 per dK/dV tile (S^T, dP^T, dV, dK)
+    against the dense bf16 peak; the CUDA-core figure counts its 64 x 64 pairs (S, dP and dQ; S, dP,
+    dV and dK; 2d each) against the fp32 FMA peak derived from the SM count and maximum clock."""
     g = torch.Generator(device=q.device).manual_seed(w.seed + 99)
     dO = torch.randn(q.shape, generator=g, device=q.device, dtype=torch.float32).to(q.dtype)
     plan.attend(q, k, v, stream)             # O and row_sum of these inputs
-    for _ in range(2):
-        plan.backward(q, k, v, dO, stream)
-    ts = []
-    for _ in range(5):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        plan.backward(q, k, v, dO, stream)
-        b.record(stream)
-        torch.cuda.synchronize()
-        ts.append(a.elapsed_time(b))
-    errs = plan.device_errors()
-    if errs:
-        raise RuntimeError(f"device errors in backward: {errs}")
+    tc_ok = w.dtype == "bf16" and w.d == 128
+
+    def timed(path):
+        for _ in range(2):
+            plan.backward(q, k, v, dO, stream, path=path)
+        ts = []
+        for _ in range(5):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            plan.backward(q, k, v, dO, stream, path=path)
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        errs = plan.device_errors()
+        if errs:
+            raise RuntimeError(f"device errors in backward ({path}): {errs}")
+        return float(np.median(ts))
+
+    ms_simt = timed("simt")
     ids = plan.ids.cpu().numpy()
     dq_pairs, dkdv_pairs = bwd_chunk_pairs(ids, w.causal, w.H // w.H_kv)
     per_pair = 2.0 * w.d * BWD_TILE * BWD_TILE
     flops = (3 * dq_pairs + 4 * dkdv_pairs) * per_pair * w.B
-    ms = float(np.median(ts))
     peak = sm_count * FP32_LANES_PER_SM * 2 * sm_max_mhz * 1e6 / 1e12
-    achieved = flops / (ms * 1e-3) / 1e12
-    return {"path": "backward (plsh_attention_bwd): dQ, dK, dV of T~, fp32 CUDA-core arithmetic",
-            "kernels": ["bwd_delta_kernel", "bwd_dkdv_kernel", "bwd_dq_kernel"], "ms_per_call": ms,
+    achieved = flops / (ms_simt * 1e-3) / 1e12
+    simt = {"path": "plsh_attention_bwd: fp32 CUDA-core arithmetic",
+            "kernels": ["bwd_delta_kernel", "bwd_dkdv_kernel", "bwd_dq_kernel"], "ms_per_call": ms_simt,
             "issued_fp32_flops": flops, "achieved_TFLOPs": achieved,
             "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak,
                          "peak_source": f"derived: {sm_count} SMs x {FP32_LANES_PER_SM} fp32 lanes x 2 x "
                                         f"{sm_max_mhz:.0f} MHz"}}
+    if not tc_ok:
+        return dict(simt, path="backward (" + simt["path"] + ")")
+    ms = timed("tc")
+    dq_tiles, dkdv_tiles = bwd_tc_tiles(plan.spans.cpu().numpy(), plan.key_spans().cpu().numpy(), w.causal)
+    mma = 2.0 * TILE * TILE * w.d
+    tflops = (3 * dq_tiles + 4 * dkdv_tiles) * mma * w.B
+    ach = tflops / (ms * 1e-3) / 1e12
+    return {"path": "backward (plsh_attention_bwd_tc): dQ, dK, dV of T~ on the tcgen05 tensor cores",
+            "kernels": ["bwd_delta_kernel", "bwd_dq_tc_kernel", "bwd_dkdv_tc_kernel"], "ms_per_call": ms,
+            "dq_tiles_per_batch": dq_tiles, "dkdv_tiles_per_batch": dkdv_tiles, "issued_tensor_flops": tflops,
+            "roofline": {"bound": "tensor", "achieved": ach, "peak": bf16_peak, "unit": "TFLOP/s",
+                         "frac": ach / bf16_peak},
+            "cuda_core_path": simt, "speedup_over_cuda_core_path": ms_simt / ms}
 
 
 def decode_timing(plan, q, k, v, stream, w):
@@ -376,6 +411,58 @@ def decode_timing(plan, q, k, v, stream, w):
             "achieved_GBps": kv_bytes / (us * 1e-6) / 1e9}
 
 
+def decode_batched_timing(w, stream, peak_gbs: float, batch: int = 64):
+    """plsh_decode_fwd for a batch of `batch` sequences of the workload's shape (one query row per
+    (b, h) at the newest position n-1, B*H rows, each against its own cache): device time per call
+    and the K/V rows of the weighted keys, which no two rows share, against the HBM peak."""
+    from alibi_positional_lsh_b200 import PlshForward
+    wb = w.with_(B=batch)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    g = torch.Generator(device=dev).manual_seed(w.seed + 7)
+    dt = wb.torch_dtype
+    k = torch.randn((batch, w.H_kv, w.n, w.d), generator=g, device=dev, dtype=torch.float32).to(dt)
+    v = torch.randn((batch, w.H_kv, w.n, w.d), generator=g, device=dev, dtype=torch.float32).to(dt)
+    q1 = torch.randn((batch, w.H, 1, w.d), generator=g, device=dev, dtype=torch.float32).to(dt)
+    plan = PlshForward(batch, w.H, w.H_kv, w.n, w.d, w.s, w.causal, w.sigmas(), w.seed, dt, str(dev))
+    plan.prepare(stream)
+    i = w.n - 1
+    pos = torch.tensor([i], dtype=torch.int32, device=dev)
+    for _ in range(3):
+        plan.decode(q1, pos, k, v, stream)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        plan.decode(q1, pos, k, v)
+    reps = 20
+    ts = []
+    for _ in range(5):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b) / reps)
+    del graph
+    errs = plan.device_errors()
+    if errs:
+        raise RuntimeError(f"device errors in batched decode: {errs}")
+    bm = plan.bmask.cpu().numpy()
+    bm = bm.view(np.uint32) if w.s <= 32 else bm.view(np.uint64)
+    keys = decode_keys(bm, w.s, i, w.causal) * batch
+    elt = 2 if w.dtype == "bf16" else 4
+    kv_bytes = keys * 2 * w.d * elt
+    us = float(np.median(ts)) * 1e3
+    gbs = kv_bytes / (us * 1e-6) / 1e9
+    del k, v, q1, plan
+    torch.cuda.empty_cache()
+    return {"path": f"batched decode (plsh_decode_fwd), {batch} sequences x {w.H} heads = {batch * w.H} rows at "
+                    "position n-1, each against its own cache", "rows": batch * w.H, "us_per_call": us,
+            "timing": "CUDA graph of one call, replayed 20 times back to back; median of 5",
+            "weighted_keys": keys, "kv_bytes": kv_bytes, "achieved_GBps": gbs, "hbm_peak_GBps": peak_gbs,
+            "frac_of_hbm": gbs / peak_gbs}
+
+
 def run_ours(args, rank, world, local):
     from alibi_positional_lsh_b200 import PlshForward
     import alibi_positional_lsh_b200 as plsh_mod  # noqa: F401
@@ -383,6 +470,8 @@ def run_ours(args, rank, world, local):
     w = workloads.WORKLOADS[args.workload]
     if args.batch:
         w = w.with_(B=args.batch)
+    if args.s:
+        w = w.with_(s=args.s)
     dev = f"cuda:{local}"
     torch.cuda.set_device(local)
     wr = rank_workload(w, rank)                      # independent problem per rank
@@ -537,11 +626,14 @@ def run_ours(args, rank, world, local):
                            "this_path_speedup": float(np.median(ts)) / attn_avg})
 
     decode = decode_timing(plan, q, k, v, stream, w) if (world == 1 and not alibi) else None
+    decode_batched = None
+    if world == 1 and not alibi and w.dtype == "bf16" and w.n <= 32768:   # 64 caches of up to 8.6 GB
+        decode_batched = decode_batched_timing(w, stream, load_peaks()[0]["hbm_gbs"])
     bwd = None
     if world == 1 and not alibi and not args.no_backward:
         props = torch.cuda.get_device_properties(local)
         bwd = bwd_timing(plan, q, k, v, stream, w, props.multi_processor_count,
-                         float(clocks.get("sm_max_mhz") or 1965))
+                         float(clocks.get("sm_max_mhz") or 1965), load_peaks()[0]["bf16_tflops"])
 
     tokens = w.B * w.n * world
     value = job_value(w.B * w.n, world, ms_step)
@@ -614,6 +706,8 @@ def run_ours(args, rank, world, local):
         line["comparison"] = others
     if decode:
         line["decode"] = decode
+    if decode_batched:
+        line["decode_batched"] = decode_batched
     if bwd:
         line["backward"] = bwd
     if rank == 0 and not args.no_cpu_baseline:
@@ -627,6 +721,8 @@ def run_ours(args, rank, world, local):
 def run_reference(args, rank, world):
     """The CPU oracle as the reference arm: rank 0 only, a bounded sample per step."""
     w = workloads.WORKLOADS[args.workload]
+    if args.s:
+        w = w.with_(s=args.s)
     if rank != 0:
         return None
     sampler = OracleSampler(w)
@@ -677,6 +773,7 @@ def main(argv=None):
                          "exact banded ALiBi")
     ap.add_argument("--eps", type=float, default=1e-4,
                     help="band cut-off of exact banded ALiBi (keys lighter than eps are left out)")
+    ap.add_argument("--s", type=int, default=None, help="hashes per head instead of the workload's own")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller cases for profiling)")
     args = ap.parse_args(argv)

@@ -70,3 +70,24 @@ def test_issued_and_visited_key_tiles(causal):
             visited += sum(1 for j0 in range(0, n, 128) if j0 + 127 >= lo and j0 <= hi)
     assert bench.issued_tiles(spans, causal) == issued
     assert bench.kernel_tiles(spans, causal) == visited
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_tensor_core_backward_tiles(causal):
+    """The tensor-core backward's work counts, recounted from c_ij: the dQ kernel visits the forward's
+    tiles; the dK/dV kernel walks, per head and 128-key tile, every 128-row query tile holding a row that
+    shares a block with one of the keys (only rows at or after the tile's first key when causal)."""
+    n, T = 1000, 8
+    ids = _table_ids(n, [3.0, 60.0, 400.0], 5, 7)
+    spans = np.stack([oracle.tile_spans(ids[h], causal) for h in range(ids.shape[0])])
+    kspans = np.stack([oracle.tile_spans(ids[h], False) for h in range(ids.shape[0])])
+    walked = 0
+    for h in range(ids.shape[0]):
+        C = oracle.match_counts(ids[h])
+        for t in range(T):
+            keys = np.arange(t * 128, min(n, t * 128 + 128))
+            rows = np.nonzero(C[:, keys].sum(axis=1))[0]
+            if causal:
+                rows = rows[rows >= t * 128]
+            walked += len({int(r) // 128 for r in rows} | {t})
+    assert bench.bwd_tc_tiles(spans, kspans, causal) == (bench.kernel_tiles(spans, causal), walked)
