@@ -193,12 +193,28 @@ def job_value(tokens_per_rank: int, world: int, ms_step_max: float) -> float:
     return tokens_per_rank * world / (ms_step_max * 1e-3)
 
 
+L2_BYTES = 126 * 2 ** 20          # B200 L2
+FLUSH_BYTES = 256 * 2 ** 20       # written between timed steps when the inputs fit in L2
+
+
+def qkv_bytes(w: workloads.Workload) -> int:
+    return (w.B * w.H * w.n * w.d + 2 * w.B * w.H_kv * w.n * w.d) * (2 if w.dtype == "bf16" else 4)
+
+
+def needs_l2_flush(w: workloads.Workload) -> bool:
+    """Inputs that fit in L2 would stay cached from one timed step to the next: flush between steps."""
+    return qkv_bytes(w) <= L2_BYTES
+
+
 def config_of(w: workloads.Workload, world: int) -> dict:
-    qkv = (w.B * w.H * w.n * w.d + 2 * w.B * w.H_kv * w.n * w.d) * (2 if w.dtype == "bf16" else 4)
+    qkv = qkv_bytes(w)
+    l2 = (f"flushed: Q+K+V = {qkv / 1e6:.0f} MB fits in the 126 MB L2, so a {FLUSH_BYTES >> 20} MB buffer is "
+          "written between timed steps, outside the per-step events" if needs_l2_flush(w) else
+          f"no flush: Q+K+V = {qkv / 1e6:.0f} MB per step, larger than the 126 MB L2")
     return {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.H_kv, "n": w.n, "d": w.d, "s": w.s,
             "causal": w.causal, "global_batch": w.B * world, "seq_len": w.n,
             "parallelism": f"independent problem per GPU x{world}",
-            "l2": f"no flush: Q+K+V = {qkv / 1e6:.0f} MB per step, larger than the 126 MB L2"}
+            "l2": l2}
 
 
 def barrier(world: int):
@@ -316,8 +332,8 @@ def bwd_tc_tiles(spans: np.ndarray, key_spans: np.ndarray, causal: bool) -> tupl
 
 
 def bwd_timing(plan, q, k, v, stream, w, sm_count: int, sm_max_mhz: float, bf16_peak: float):
-    """plsh_attention_bwd on the step's inputs with a seeded dO: device time per call of the tcgen05
-    kernels (bf16, d = 128) and of the fp32 CUDA-core kernels. The tensor-core roofline counts 3 MMAs
+    """plsh_attention_bwd on the step's inputs with a seeded dO: device time per call (L2 flushed before
+    each) of the tcgen05 kernels (bf16, d = 128) and of the fp32 CUDA-core kernels. The tensor-core roofline counts 3 MMAs
     of 128 x 128 x 128 per dQ tile (S, dP, dQ += dS K) and 4 per dK/dV tile (S^T, dP^T, dV, dK)
     against the dense bf16 peak; the CUDA-core figure counts its 64 x 64 pairs (S, dP and dQ; S, dP,
     dV and dK; 2d each) against the fp32 FMA peak derived from the SM count and maximum clock."""
@@ -326,11 +342,14 @@ def bwd_timing(plan, q, k, v, stream, w, sm_count: int, sm_max_mhz: float, bf16_
     plan.attend(q, k, v, stream)             # O and row_sum of these inputs
     tc_ok = w.dtype == "bf16" and w.d == 128
 
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=q.device)
+
     def timed(path):
         for _ in range(2):
             plan.backward(q, k, v, dO, stream, path=path)
         ts = []
         for _ in range(5):
+            flush.fill_(2)                   # L2 cold at the start of every timed call
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
             plan.backward(q, k, v, dO, stream, path=path)
@@ -371,6 +390,38 @@ def bwd_timing(plan, q, k, v, stream, w, sm_count: int, sm_max_mhz: float, bf16_
             "cuda_core_path": simt, "speedup_over_cuda_core_path": ms_simt / ms}
 
 
+def graph_call_us(call, stream, reps: int) -> dict:
+    """Device time of one call, from CUDA graphs replayed back to back (one call timed alone on an
+    idle GPU would include the host's launch latency). `warm_us`: the call's graph replayed `reps`
+    times, so what one call reads may still sit in L2 for the next. `cold_us`: a graph of an L2 flush
+    (a write of FLUSH_BYTES) followed by the call, minus a graph of the flush alone. Medians of 5."""
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=torch.device("cuda", torch.cuda.current_device()))
+    graphs = {}
+    for name in ("warm", "flush_call", "flush"):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            if name != "warm":
+                flush.fill_(1)
+            if name != "flush":
+                call()
+        graphs[name] = g
+    out = {}
+    for name, g in graphs.items():
+        g.replay()
+        ts = []
+        for _ in range(5):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(reps):
+                g.replay()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b) * 1e3 / reps)
+        out[name] = float(np.median(ts))
+    del graphs, flush
+    return {"warm_us": out["warm"], "cold_us": out["flush_call"] - out["flush"], "flush_us": out["flush"]}
+
+
 def decode_timing(plan, q, k, v, stream, w):
     """plsh_decode_fwd on the newest position (one query row per (b, h) at i = n-1) against the whole
     cache: device time per call and the K/V bytes it must read (the weighted keys' rows)."""
@@ -380,22 +431,7 @@ def decode_timing(plan, q, k, v, stream, w):
     for _ in range(3):
         plan.decode(q1, pos, k, v, stream)
     torch.cuda.synchronize()
-    # one call's device time: a CUDA graph of the call, replayed back to back (a single call timed on an
-    # idle GPU would include the host's launch latency)
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        plan.decode(q1, pos, k, v)
-    reps = 50
-    ts = []
-    for _ in range(5):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(reps):
-            graph.replay()
-        b.record(stream)
-        torch.cuda.synchronize()
-        ts.append(a.elapsed_time(b) / reps)
-    del graph
+    t = graph_call_us(lambda: plan.decode(q1, pos, k, v), stream, 50)
     errs = plan.device_errors()
     if errs:
         raise RuntimeError(f"device errors in decode: {errs}")
@@ -404,10 +440,12 @@ def decode_timing(plan, q, k, v, stream, w):
     keys = decode_keys(bm, w.s, i, w.causal) * w.B
     elt = 2 if w.dtype == "bf16" else 4
     kv_bytes = keys * 2 * w.d * elt
-    us = float(np.median(ts)) * 1e3
+    us = t["cold_us"]
     return {"path": "decode (plsh_decode_fwd), one query row per (b, h) at position n-1, whole cache",
             "kernels": ["decode_partial_kernel"], "us_per_call": us,
-            "timing": "CUDA graph of one call, replayed 50 times back to back; median of 5", "weighted_keys": keys, "kv_bytes": kv_bytes,
+            "timing": "L2 flushed before each call: CUDA graph of (flush, call) minus graph of the flush, "
+                      "50 replays, median of 5",
+            "us_per_call_l2_warm": t["warm_us"], "weighted_keys": keys, "kv_bytes": kv_bytes,
             "achieved_GBps": kv_bytes / (us * 1e-6) / 1e9}
 
 
@@ -430,20 +468,7 @@ def decode_batched_timing(w, stream, peak_gbs: float, batch: int = 64):
     for _ in range(3):
         plan.decode(q1, pos, k, v, stream)
     torch.cuda.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        plan.decode(q1, pos, k, v)
-    reps = 20
-    ts = []
-    for _ in range(5):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(reps):
-            graph.replay()
-        b.record(stream)
-        torch.cuda.synchronize()
-        ts.append(a.elapsed_time(b) / reps)
-    del graph
+    t = graph_call_us(lambda: plan.decode(q1, pos, k, v), stream, 20)
     errs = plan.device_errors()
     if errs:
         raise RuntimeError(f"device errors in batched decode: {errs}")
@@ -452,13 +477,15 @@ def decode_batched_timing(w, stream, peak_gbs: float, batch: int = 64):
     keys = decode_keys(bm, w.s, i, w.causal) * batch
     elt = 2 if w.dtype == "bf16" else 4
     kv_bytes = keys * 2 * w.d * elt
-    us = float(np.median(ts)) * 1e3
+    us = t["cold_us"]
     gbs = kv_bytes / (us * 1e-6) / 1e9
     del k, v, q1, plan
     torch.cuda.empty_cache()
     return {"path": f"batched decode (plsh_decode_fwd), {batch} sequences x {w.H} heads = {batch * w.H} rows at "
                     "position n-1, each against its own cache", "rows": batch * w.H, "us_per_call": us,
-            "timing": "CUDA graph of one call, replayed 20 times back to back; median of 5",
+            "timing": "L2 flushed before each call: CUDA graph of (flush, call) minus graph of the flush, "
+                      "20 replays, median of 5",
+            "us_per_call_l2_warm": t["warm_us"],
             "weighted_keys": keys, "kv_bytes": kv_bytes, "achieved_GBps": gbs, "hbm_peak_GBps": peak_gbs,
             "frac_of_hbm": gbs / peak_gbs}
 
@@ -515,20 +542,27 @@ def run_ours(args, rank, world, local):
     tiles_min = issued_tiles(spans, w.causal)
     tiles_run = kernel_tiles(spans, w.causal)
 
-    # timed region: K steps, device-timed, inputs (Q+K+V > L2) already resident
+    # timed region: K steps, device-timed, inputs already resident; inputs that fit in L2 are
+    # evicted between steps by a write larger than L2, which each step's own events leave out
     K = args.steps
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev) if needs_l2_flush(w) else None
     ev_k = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    ev_s = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         barrier(world)
         torch.cuda.synchronize()
         start.record(stream)
         for i in range(K):
+            if flush is not None:
+                flush.fill_(i & 255)
+            ev_s[i][0].record(stream)
             step(ev_k[i])
+            ev_s[i][1].record(stream)
         end.record(stream)
         torch.cuda.synchronize()
         barrier(world)
-    ms_total = start.elapsed_time(end)
+    ms_total = (sum(a.elapsed_time(b) for a, b in ev_s) if flush is not None else start.elapsed_time(end))
     attn_ms = [a.elapsed_time(b) for a, b in ev_k]
     ms_total = dist_max(ms_total, world)
     ms_step = ms_total / K
