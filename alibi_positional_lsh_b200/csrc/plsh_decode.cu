@@ -12,7 +12,8 @@
 // the chain of dependent loads along the walk sets its latency.
 //
 // Each query row's walk is spread over G CTAs of 256 threads (G chosen so the
-// grid covers the SMs about twice, at most 8). Keys are taken in chunks of 256
+// grid covers the SMs about twelve times, at most 8; four CTAs fit on an SM,
+// at 64 registers a thread). Keys are taken in chunks of 256
 // on each side of i (i and below, then above when not causal); CTA g of a row
 // takes chunks g, g + G, g + 2G, ... Its carry -- the OR of the masks between
 // i and its chunk -- is OR-reduced from the masks of the chunks in between,
@@ -58,14 +59,17 @@ __device__ __forceinline__ float dot_row(const float* q, const float* row) {
 template <int D>
 __device__ __forceinline__ float dot_row(const float* q, const __nv_bfloat16* row) {
   float acc = 0.0f;
+#pragma unroll 1
+  for (int h0 = 0; h0 < D; h0 += 64) {  // 64 dims (eight 16-byte loads) at a time
 #pragma unroll
-  for (int e = 0; e < D; e += 8) {
-    const uint4 u = *reinterpret_cast<const uint4*>(row + e);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    for (int e = h0; e < h0 + 64; e += 8) {
+      const uint4 u = *reinterpret_cast<const uint4*>(row + e);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float lo = __uint_as_float(w[k] << 16), hi = __uint_as_float(w[k] & 0xFFFF0000u);
-      acc = fmaf(q[e + 2 * k], lo, fmaf(q[e + 2 * k + 1], hi, acc));
+      for (int k = 0; k < 4; ++k) {
+        const float lo = __uint_as_float(w[k] << 16), hi = __uint_as_float(w[k] & 0xFFFF0000u);
+        acc = fmaf(q[e + 2 * k], lo, fmaf(q[e + 2 * k + 1], hi, acc));
+      }
     }
   }
   return acc;
@@ -148,7 +152,7 @@ __device__ __forceinline__ MaskT walk_or(const MaskT* bm, int i, int n, int side
 // One of G CTAs of query row t of (b, h): the chunks g, g + G, g + 2G, ... of each side's walk. Its
 // partial result -- running maximum, sum and unnormalised output row -- goes to part.
 template <typename T, int D, typename MaskT>
-__global__ void __launch_bounds__(kThreads) decode_partial_kernel(
+__global__ void __launch_bounds__(kThreads, 4) decode_partial_kernel(
     const T* __restrict__ Q, const int32_t* __restrict__ pos, int m, const T* __restrict__ K,
     const T* __restrict__ V, int H, int H_kv, int n, int s, int causal, const MaskT* __restrict__ bmask, int G,
     float* __restrict__ part, unsigned* __restrict__ done, T* __restrict__ O, float* __restrict__ row_sum,
@@ -200,12 +204,12 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, o);
     lw += psum;
-    // O += p_j V_j over the warp's keys, lanes over dims; 16 keys at a time, their loads issued together
+    // O += p_j V_j over the warp's keys, lanes over dims; 8 keys at a time, their loads issued together
 #pragma unroll 1
-    for (int k0 = 0; k0 < 32; k0 += 16) {
-      float pk[16], vv[16][DPL];
+    for (int k0 = 0; k0 < 32; k0 += 8) {
+      float pk[8], vv[8][DPL];
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
+      for (int u = 0; u < 8; ++u) {
         pk[u] = __shfl_sync(0xffffffffu, p, k0 + u);
         const int jk = __shfl_sync(0xffffffffu, j, k0 + u);
         if (pk[u] != 0.0f) {
@@ -216,7 +220,7 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(
         }
       }
 #pragma unroll
-      for (int u = 0; u < 16; ++u)
+      for (int u = 0; u < 8; ++u)
 #pragma unroll
         for (int e = 0; e < DPL; ++e) ow[e] = fmaf(pk[u], vv[u][e], ow[e]);
     }
@@ -342,12 +346,13 @@ int launch_decode_mask(const DecodeArgs& a, int G, cudaStream_t st) {
 }  // namespace
 
 int launch_decode(const DecodeArgs& a, cudaStream_t st) {
-  // CTAs per row: enough for about two CTAs per SM over all rows, at most kDecodeMaxSplit
+  // CTAs per row: enough for about twelve CTAs per SM over all rows (a row's walk can be long, and
+  // a few long rows would otherwise set the time of the whole grid), at most kDecodeMaxSplit
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     sms = 148;
   const long long rows = static_cast<long long>(a.B) * a.H * a.m;
-  const int G = static_cast<int>(std::min<long long>(kDecodeMaxSplit, std::max<long long>(1, (2LL * sms + rows - 1) / rows)));
+  const int G = static_cast<int>(std::min<long long>(kDecodeMaxSplit, std::max<long long>(1, (12LL * sms + rows - 1) / rows)));
   if (a.dtype == PLSH_F32)
     return a.d == 64 ? launch_decode_mask<float, 64>(a, G, st) : launch_decode_mask<float, 128>(a, G, st);
   return a.d == 64 ? launch_decode_mask<__nv_bfloat16, 64>(a, G, st) : launch_decode_mask<__nv_bfloat16, 128>(a, G, st);

@@ -205,17 +205,16 @@ __device__ __forceinline__ void regs_after_wait(uint32_t (&r)[N]) {
   for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
 }
 
-// Diagonal tile, 32-row block q (rows [32q, 32q + 32), row r): counts of the block's own 32 keys,
+// Diagonal tile, one 32-row block (rows [32q, 32q + 32) of the tile, row r): counts of the block's own 32 keys,
 // as bytes (key 32q + 4j + e in byte e of word j), written to this thread's column cw[j * ld] of
 // shared memory, and the carries for the other keys. Keys c < r: R = OR bm[c + 1 .. r], scanned
 // from the row down (count 0 unless kBelow); the row's own key: count s; keys c > r:
 // R = OR bm[r + 1 .. c], scanned from the row up (count 0 unless kAbove). On return
 // lo = OR bm[32q + 1 .. r] and hi = OR bm[r + 1 .. 32q + 31] (0 unless kAbove).
+// bq[c] = mask of the block's key c (c = 0..32), rr = the row within the block (0..31).
 template <typename MaskT, bool kBelow, bool kAbove>
-__device__ __forceinline__ void diag_scan(const MaskStage<MaskT>& ms, int q, int r, int s, uint32_t* cw, int ld,
-                                          MaskT& lo, MaskT& hi) {
-  const MaskT* bq = ms.bm + 32 * q;
-  const int rr = r - 32 * q;  // the row within the block, 0..31
+__device__ __forceinline__ void diag_scan_block(const MaskT* bq, int rr, int s, uint32_t* cw, int ld, MaskT& lo,
+                                                MaskT& hi) {
   MaskT R = 0;
 #pragma unroll 1
   for (int j = 7; j >= 0; --j) {
@@ -246,6 +245,12 @@ __device__ __forceinline__ void diag_scan(const MaskStage<MaskT>& ms, int q, int
     }
   }
   hi = R2;
+}
+// The same for row r of the published stage's 32-row block q (bm[c] = mask of key j0 + c, c = 0..128).
+template <typename MaskT, bool kBelow, bool kAbove>
+__device__ __forceinline__ void diag_scan(const MaskStage<MaskT>& ms, int q, int r, int s, uint32_t* cw, int ld,
+                                          MaskT& lo, MaskT& hi) {
+  diag_scan_block<MaskT, kBelow, kAbove>(ms.bm + 32 * q, r - 32 * q, s, cw, ld, lo, hi);
 }
 
 // The masks of a key tile as the mask warp publishes them: xv[e] is the mask of key 4 lane + e,
@@ -348,6 +353,21 @@ inline int make_map(CUtensorMap* map, const void* base, int rows, int planes) {
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PLSH_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return PLSH_OK;
+}
+
+// [planes][rows][128] bf16, boxes of 32 x 32 x 1 without swizzle (an output tile of 32 rows and
+// 32 columns staged row-major, 64 bytes a row); elements past `rows` are not written.
+inline int make_map_o(CUtensorMap* map, void* base, int rows, int planes) {
+  auto enc = get_encode_fn();
+  if (!enc) return fail(PLSH_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(planes)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(kD) * 2, static_cast<cuuint64_t>(rows) * kD * 2};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(PLSH_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
   return PLSH_OK;
 }
