@@ -271,8 +271,7 @@ extern "C" int plsh_alibi_banded_fwd(const void* Q, const void* K, const void* V
 
 extern "C" size_t plsh_decode_scratch_bytes(int B, int H, int m, int d) {
   if (B < 1 || H < 1 || m < 1 || d < 1) return 0;
-  const size_t rows = static_cast<size_t>(B) * H * m;
-  return sizeof(float) * rows * plsh::kDecodeMaxSplit * (static_cast<size_t>(d) + 2) + sizeof(unsigned) * rows;
+  return plsh::decode_scratch_bytes(static_cast<long long>(B) * H * m, d);
 }
 
 extern "C" int plsh_decode_fwd(const void* Q, const int32_t* pos_dev, int m, const void* K, const void* V, int dtype,

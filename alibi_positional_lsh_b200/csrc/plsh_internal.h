@@ -46,8 +46,9 @@ struct AttnArgs {
   double log_inv_eps;
 };
 // Decode: query rows Q [B][H][m][d] at positions pos [m] against K, V [B][H_kv][n][d].
-// part: caller scratch of B*H*m*kDecodeMaxSplit*(d+2) floats for the per-CTA partial results, then one
-// unsigned counter per row (zero before the first call; every completed call leaves them zero).
+// part: caller scratch (decode_scratch_bytes): B*H*m*kDecodeMaxSplit*(d+2) floats for the partial
+// results of a row's work units, the call's work list, then one unsigned counter per row (zero before
+// the first call; every completed call leaves them zero).
 constexpr int kDecodeMaxSplit = 8;
 struct DecodeArgs {
   const void* Q; const int32_t* pos; int m;
@@ -58,6 +59,9 @@ struct DecodeArgs {
   float* part;
 };
 int launch_decode(const DecodeArgs& a, cudaStream_t st);
+// Bytes of decode scratch for `rows` query rows of width d (partial results, per-row walk data,
+// one counter per row at the end).
+size_t decode_scratch_bytes(long long rows, int d);
 // Backward: dQ, dK, dV of T~ (Q, O, dO, dQ [B][H][n][d]; K, V, dK, dV [B][H_kv][n][d]).
 struct BwdArgs {
   const void* Q; const void* K; const void* V; const void* O; const void* dO;

@@ -442,7 +442,7 @@ def decode_timing(plan, q, k, v, stream, w):
     kv_bytes = keys * 2 * w.d * elt
     us = t["cold_us"]
     return {"path": "decode (plsh_decode_fwd), one query row per (b, h) at position n-1, whole cache",
-            "kernels": ["decode_partial_kernel"], "us_per_call": us,
+            "kernels": ["decode_range_kernel", "decode_unit_kernel"], "us_per_call": us,
             "timing": "L2 flushed before each call: CUDA graph of (flush, call) minus graph of the flush, "
                       "50 replays, median of 5",
             "us_per_call_l2_warm": t["warm_us"], "weighted_keys": keys, "kv_bytes": kv_bytes,
@@ -662,7 +662,7 @@ def run_ours(args, rank, world, local):
     decode = decode_timing(plan, q, k, v, stream, w) if (world == 1 and not alibi) else None
     decode_batched = None
     if world == 1 and not alibi and w.dtype == "bf16" and w.n <= 32768:   # 64 caches of up to 8.6 GB
-        decode_batched = decode_batched_timing(w, stream, load_peaks()[0]["hbm_gbs"])
+        decode_batched = decode_batched_timing(w, stream, load_peaks()[0]["hbm_gbs"], args.decode_batch)
     bwd = None
     if world == 1 and not alibi and not args.no_backward:
         props = torch.cuda.get_device_properties(local)
@@ -808,6 +808,8 @@ def main(argv=None):
     ap.add_argument("--eps", type=float, default=1e-4,
                     help="band cut-off of exact banded ALiBi (keys lighter than eps are left out)")
     ap.add_argument("--s", type=int, default=None, help="hashes per head instead of the workload's own")
+    ap.add_argument("--decode-batch", type=int, default=64,
+                    help="sequences of the batched decode timing (64; fewer for a small profiling case)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller cases for profiling)")
     args = ap.parse_args(argv)

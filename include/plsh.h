@@ -364,12 +364,13 @@ PLSH_API int plsh_alibi_banded_fwd(const void* Q, const void* K, const void* V, 
  *   dtype, d, s, causal, bmask_dev, err_dev   as plsh_attention_fwd; the
  *              masks are plsh_window's for this n (with causal, only the
  *              entries at positions <= max(pos) are read).
- *   scratch_dev    device scratch: the partial results of the CTAs that
- *                  share a row's walk (up to 8 per row), then one counter
- *                  per row. Zero the whole buffer once before its first use
- *                  (for example with cudaMemsetAsync). Every call that runs
- *                  to completion leaves the counters at zero again; after a
- *                  call that did not (a CUDA error), zero it again.
+ *   scratch_dev    device scratch: the partial results of the work units
+ *                  that share a row's walk (up to 8 per row), the row's
+ *                  walk data, then one counter per row. Zero the whole
+ *                  buffer once before its first use (for example with
+ *                  cudaMemsetAsync). Every call that runs to completion
+ *                  leaves the counters at zero again; after a call that did
+ *                  not (a CUDA error, or PLSH_DEVERR_TIMEOUT), zero it again.
  *                  scratch_bytes is its size, at least
  *                  plsh_decode_scratch_bytes(B, H, m, d), else
  *                  PLSH_ERR_INVALID_ARG.
@@ -383,7 +384,10 @@ PLSH_API int plsh_decode_fwd(const void* Q, const int32_t* pos_dev, int m, const
 
 /*
  * plsh_decode_scratch_bytes -- bytes of scratch plsh_decode_fwd needs:
- * 4 * B * H * m * (8 * (d + 2) + 1). Returns 0 for a non-positive size.
+ * B * H * m * (32 * (d + 2) + 260) + 16: the partial results of up to 8
+ * work units per row, the call's work list (up to 8 units of 32 bytes per
+ * row, and its counter), then one 4-byte counter per row (the buffer's last
+ * B * H * m words). Returns 0 for a non-positive size.
  */
 PLSH_API size_t plsh_decode_scratch_bytes(int B, int H, int m, int d);
 

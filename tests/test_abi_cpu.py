@@ -143,7 +143,7 @@ def test_decode_rejects_bad_arguments_before_any_launch(plsh):
     args = lambda m=4, pos=fake, d=128, H_kv=1, causal=1, nbytes=1 << 30: (
         fake, pos, m, fake, fake, 0, 1, 2, H_kv, 256, d, 20, fake, causal, fake, ctypes.c_size_t(nbytes), fake, fake,
         fake, null)
-    assert lib.plsh_decode_scratch_bytes(1, 2, 4, 128) == 4 * 2 * 4 * (8 * 130 + 1)
+    assert lib.plsh_decode_scratch_bytes(1, 2, 4, 128) == 2 * 4 * (32 * 130 + 260) + 16
     assert lib.plsh_decode_fwd(*args(nbytes=100)) == 1 and "scratch" in plsh.plsh_last_error()
     assert lib.plsh_decode_fwd(*args(m=0)) == 1 and "m >= 1" in plsh.plsh_last_error()
     assert lib.plsh_decode_fwd(*args(pos=null)) == 1 and "null" in plsh.plsh_last_error()
