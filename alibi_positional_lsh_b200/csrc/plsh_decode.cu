@@ -27,7 +27,8 @@
 //
 // Every wait on a copy is bounded in time (PLSH_DEVERR_TIMEOUT); a CTA that
 // gives up waits (again bounded) for the copies it issued and returns, and its
-// row's output is left unwritten.
+// rows' outputs are left unwritten. A test hook (plsh_test_withhold_mma) makes
+// the producer issue nothing, so that the compute warps' waits run out.
 #include <algorithm>
 #include <cmath>
 
@@ -315,7 +316,7 @@ __global__ void __launch_bounds__(kUnitThreads) decode_unit_kernel(
     const T* __restrict__ Q, const T* __restrict__ K, const T* __restrict__ V, int m, int H, int H_kv, int n, int s,
     const MaskT* __restrict__ bmask, const UnitDesc* __restrict__ units, const unsigned* __restrict__ unit_count,
     float* __restrict__ part, unsigned* __restrict__ done, T* __restrict__ O, float* __restrict__ row_sum,
-    uint32_t* __restrict__ err, uint64_t wait_ns) {
+    uint32_t* __restrict__ err, uint64_t wait_ns, int withhold) {
   using Smem = UnitSmem<T, D, MaskT>;
   constexpr int SEG = Smem::kSeg;
   constexpr int KPW = SEG / kComputeWarps;  // keys per compute warp per segment
@@ -352,10 +353,11 @@ __global__ void __launch_bounds__(kUnitThreads) decode_unit_kernel(
 
   if (warp == kWarpProducer) {
     // ------------------------------------------------------------ producer
+    // (a failure-detection test can tell it to issue nothing, so that the compute warps' waits run out)
     int issued = 0;
-    bool ok = true;
+    bool ok = withhold == 0;
     UnitDesc nxt;  // the next unit's descriptor, loaded one unit ahead
-    if (has_unit(0)) nxt = units[blockIdx.x];
+    if (ok && has_unit(0)) nxt = units[blockIdx.x];
     for (int ord = 0; ok && has_unit(ord); ++ord) {
       const UnitDesc pd = nxt;
       if (has_unit(ord + 1)) nxt = units[blockIdx.x + static_cast<unsigned>(ord + 1) * G];
@@ -639,7 +641,7 @@ int launch_decode_typed(const DecodeArgs& a, cudaStream_t st) {
   kern<<<static_cast<unsigned>(grid), kUnitThreads, smem, st>>>(
       static_cast<const T*>(a.Q), static_cast<const T*>(a.K), static_cast<const T*>(a.V), a.m, a.H, a.H_kv, a.n, a.s,
       static_cast<const MaskT*>(a.bmask), sc.units, sc.unit_count, a.part, sc.done, static_cast<T*>(a.O),
-      a.row_sum, a.err, wait_limit_ns());
+      a.row_sum, a.err, wait_limit_ns(), withhold_mma() ? 1 : 0);
   e = cudaGetLastError();
   return e == cudaSuccess ? PLSH_OK : cuda_fail(e, "decode_unit_kernel launch");
 }

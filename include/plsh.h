@@ -83,20 +83,23 @@ PLSH_API int plsh_version(void);
  *
  * Every wait of the tensor-core attention kernel (plsh_attention_fwd,
  * plsh_attention_varlen_fwd[_static], plsh_alibi_banded_fwd with bf16,
- * d = 128) on one of its roles is bounded in wall-clock time. A wait that runs
- * out sets PLSH_DEVERR_TIMEOUT in err_dev; every role then leaves its loop,
- * copies and tensor-core operations already in flight are drained (with a
- * separate limit of 0.1 s), Tensor Memory is freed and the kernel returns, so
- * the context stays usable. The outputs of such a launch are unspecified.
+ * d = 128), of the tensor-core backward (plsh_attention_bwd_tc) and of the
+ * decode kernels (plsh_decode_fwd) on one of its roles is bounded in
+ * wall-clock time. A wait that runs out sets PLSH_DEVERR_TIMEOUT in err_dev;
+ * every role then leaves its loop, copies and tensor-core operations already
+ * in flight are drained (with a separate limit of 0.1 s), Tensor Memory is
+ * freed and the kernel returns, so the context stays usable. The outputs of
+ * such a launch are unspecified.
  *
  * plsh_set_wait_limit_ns -- the limit for launches made after the call, in
  *   every host thread. 0 restores the default (2 s); above
  *   PLSH_MAX_WAIT_LIMIT_NS (60 s) returns PLSH_ERR_RANGE and changes nothing.
  *
- * plsh_test_withhold_mma -- test hook: while `on` is nonzero, the kernel's
- *   tensor-core issuer issues nothing, so every wait for a tile of scores runs
- *   out after the wait limit. For testing the failure path only (pair it with
- *   a short limit); off by default.
+ * plsh_test_withhold_mma -- test hook: while `on` is nonzero, the attention
+ *   kernel's tensor-core issuer issues nothing, so every wait for a tile of
+ *   scores runs out after the wait limit, and the decode kernel's producer
+ *   issues no copies, so every wait for a segment runs out. For testing the
+ *   failure path only (pair it with a short limit); off by default.
  */
 #define PLSH_MAX_WAIT_LIMIT_NS 60000000000ull
 PLSH_API int plsh_set_wait_limit_ns(uint64_t limit_ns);

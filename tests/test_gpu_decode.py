@@ -136,3 +136,16 @@ def test_decode_mha8_non_causal_both_sides():
     want_O, want_R = PH.oracle_rows(q, k, v, plan.table_host.numpy(), w.causal, rows)
     to, tr = PH.tolerance(w.torch_dtype, v)
     PH.assert_close(O, R, want_O, want_R, to, tr, "decode mha8")
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 64)])
+def test_decode_long_runs_both_sides(dtype, d):
+    """Blocks much longer than the sequence (sigma = 1e6) and not causal: every row's runs reach both ends
+    of a 20,000-key cache, so the range pass takes several 2,048-key steps, each side gets several work
+    units of many segments, and every unit but the first starts from a carry."""
+    n, H = 20000, 2
+    rows = [0, 137, 9999, 19998, 19999]
+    q, k, v, plan, O, R = _run(1, H, 1, n, d, dtype, False, 20, [1.0e6, 3.0e3], 2024, rows)
+    want_O, want_R = PH.oracle_rows(q, k, v, plan.table_host.numpy(), False, rows)
+    to, tr = PH.tolerance(dtype, v)
+    PH.assert_close(O, R, want_O, want_R, to, tr, "decode long runs")
