@@ -360,7 +360,8 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  constexpr uint32_t kColS = 0, kColDP = 128, kColAcc = 256;
+  // S (then dS) of tile g at columns 0 or 384 by g's parity, dP at 128, the dQ accumulator at 256
+  constexpr uint32_t kColS = 0, kColDP = 128, kColAcc = 256, kColS1 = 384;
 
   if (warp == kWarpTma) {
     // ------------------------------------------------------------ TMA: Q and dO per item, K and V per tile
@@ -409,8 +410,11 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
-    // Per tile: S = Q K^T, dP = dO V^T; once dS is written over S: dQ += dS K. The next tile's S
-    // and dP follow dQ's MMAs in issue order, so they overwrite dS only after dQ has read it.
+    // Per tile g: S(g) = Q K^T into the S buffer of g's parity, dP(g) = dO V^T; once dS(g) is written
+    // over S(g): dQ += dS(g) K. S(g+1) is issued before waiting for dS(g), so it computes while the
+    // elementwise warps work on tile g, and dP(g+1) right after dS(g), before dQ's MMAs, so the
+    // elementwise warps wait for one MMA between tiles. S(g+2) reuses dS(g)'s buffer and follows
+    // dQ(g)'s MMAs in issue order, so it overwrites dS only after dQ has read it.
     if (lane == 0) {
       constexpr uint32_t idesc_nt = idesc_bf16_f32(128, 128, 0);  // B K-major (S, dP)
       constexpr uint32_t idesc_nn = idesc_bf16_f32(128, 128, 1);  // B MN-major (dQ += dS K)
@@ -422,21 +426,25 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
         v_desc[i] = smem_desc_sw128(smem_u32(sm.v[i]), 16, 1024);
         kmn_desc[i] = smem_desc_sw128(smem_u32(sm.k[i]), kChunkBytes, 1024);
       }
-      TileIter<false, false> ti;
-      ti.start(&prm, sm.order);
-      bool ok = true;
-      while (ok && ti.valid) {
-        const int st = ti.g % kStages;
-        const uint32_t ph = static_cast<uint32_t>(ti.g / kStages) & 1u;
-        if (ti.first() && !(ok = mbar_wait(&sm.q_full, static_cast<uint32_t>(ti.k) & 1u, abort_flag, err, wait_ns))) break;
-        if (!(ok = mbar_wait(&sm.k_full[st], ph, abort_flag, err, wait_ns))) break;
-        if (!(ok = mbar_wait(&sm.v_full[st], ph, abort_flag, err, wait_ns))) break;
+      auto s_col = [&](int g) { return (g & 1) ? kColS1 : kColS; };
+      // S(t) = Q K^T (waits for the item's Q and the tile's K)
+      auto issue_s = [&](const TileIter<false, false>& t) -> bool {
+        const int st = t.g % kStages;
+        if (t.first() && !mbar_wait(&sm.q_full, static_cast<uint32_t>(t.k) & 1u, abort_flag, err, wait_ns)) return false;
+        if (!mbar_wait(&sm.k_full[st], static_cast<uint32_t>(t.g / kStages) & 1u, abort_flag, err, wait_ns)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
-          mma_ss(tmem + kColS, q_desc + off, (st ? k_desc[1] : k_desc[0]) + off, idesc_nt, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + s_col(t.g), q_desc + off, (st ? k_desc[1] : k_desc[0]) + off, idesc_nt, kk > 0 ? 1u : 0u);
         }
+        return true;
+      };
+      // dP(t) = dO V^T, then s_full (S(t) and dP(t) complete)
+      auto issue_dp = [&](const TileIter<false, false>& t) -> bool {
+        const int st = t.g % kStages;
+        if (!mbar_wait(&sm.v_full[st], static_cast<uint32_t>(t.g / kStages) & 1u, abort_flag, err, wait_ns)) return false;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
@@ -444,17 +452,40 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
         }
         mma_commit(&sm.s_full);
         mma_commit(&sm.v_empty[st]);
-        if (ti.last()) mma_commit(&sm.q_empty);
-        if (!(ok = mbar_wait(&sm.p_full, static_cast<uint32_t>(ti.g) & 1u, abort_flag, err, wait_ns))) break;
+        if (t.last()) mma_commit(&sm.q_empty);  // the item's Q and dO are no longer read
+        return true;
+      };
+      TileIter<false, false> cur, nxt;
+      cur.start(&prm, sm.order);
+      nxt.start(&prm, sm.order);
+      if (nxt.valid) nxt.next();
+      bool ok = !cur.valid || (issue_s(cur) && issue_dp(cur));
+      while (ok && cur.valid) {
+        const int st = cur.g % kStages;
+        // the next tile's scores, unless they need the next item's Q (loaded once this item's last
+        // scores are done)
+        const bool s_early = nxt.valid && !nxt.first();
+        if (s_early && !(ok = issue_s(nxt))) break;
+        if (!(ok = mbar_wait(&sm.p_full, static_cast<uint32_t>(cur.g) & 1u, abort_flag, err, wait_ns))) break;
         tc_fence_after();
+        auto issue_dq = [&]() {
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ts(tmem + kColAcc, tmem + kColS + 8u * kk,
-                 (st ? kmn_desc[1] : kmn_desc[0]) + static_cast<uint64_t>((kk * 2048) >> 4), idesc_nn,
-                 (!ti.first() || kk > 0) ? 1u : 0u);
-        mma_commit(&sm.g_done);
-        mma_commit(&sm.k_empty[st]);
-        ti.next();
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            mma_ts(tmem + kColAcc, tmem + s_col(cur.g) + 8u * kk,
+                   (st ? kmn_desc[1] : kmn_desc[0]) + static_cast<uint64_t>((kk * 2048) >> 4), idesc_nn,
+                   (!cur.first() || kk > 0) ? 1u : 0u);
+          mma_commit(&sm.g_done);
+          mma_commit(&sm.k_empty[st]);
+        };
+        if (s_early) {  // within an item: the next tile's dP first, which the elementwise warps wait for
+          if (!(ok = issue_dp(nxt))) break;
+          issue_dq();
+        } else {        // the item's last tile: its dQ first, which the item's epilogue waits for
+          issue_dq();
+          if (nxt.valid && !(ok = issue_s(nxt) && issue_dp(nxt))) break;
+        }
+        cur.next();
+        if (nxt.valid) nxt.next();
       }
       mma_commit(&sm.drain);
       mbar_wait_drain(&sm.drain, 0, kDrainNs);
@@ -530,7 +561,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
     const int kh = lane >> 4;
     const int r = quarter * 32 + hq * 16 + (lane & 15);
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32 + hq * 16) << 16;
-    const uint32_t s_base = tmem + lane_off + kColS, dp_base = tmem + lane_off + kColDP;
+    const uint32_t dp_base = tmem + lane_off + kColDP;
     const float sc = kLog2e / sqrtf(static_cast<float>(kD));
     const float log2s = log2f(static_cast<float>(s));
     const uint64_t sc2 = f2_pack(sc, sc);
@@ -580,6 +611,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full, static_cast<uint32_t>(g) & 1u, abort_flag, err, wait_ns)))
         break;
       tc_fence_after();
+      const uint32_t s_base = tmem + lane_off + ((g & 1) ? kColS1 : kColS);  // S(g), then dS(g)
 #pragma unroll 1
       for (int m = 0; m < kTile / 32; ++m) {
         uint32_t pk[8];
@@ -621,7 +653,13 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.p_full);
       if (last) {
-        // the item's dQ once its last MMA has completed: dQ / sqrt(d)
+        // the item's dQ once its last MMA has completed: dQ / sqrt(d). g_done completes once per tile,
+        // and the next tile's dP is issued before this tile's dQ, so when these warps get here the
+        // latest completed phase can be g - 2: wait for phase g - 1, then g (a parity wait alone
+        // would take phase g - 2 for g)
+        if (g >= 1 && !__all_sync(0xffffffffu, mbar_wait(&sm.g_done, static_cast<uint32_t>(g - 1) & 1u, abort_flag,
+                                                         err, wait_ns)))
+          break;
         if (!__all_sync(0xffffffffu, mbar_wait(&sm.g_done, static_cast<uint32_t>(g) & 1u, abort_flag, err, wait_ns)))
           break;
         tc_fence_after();
