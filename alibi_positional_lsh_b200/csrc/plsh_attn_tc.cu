@@ -135,38 +135,6 @@ struct SoftmaxK {
   uint64_t sc2, negm2, neg2p23;
 };
 
-// P = c 2^(S sc - m) for 16 keys (S as raw fp32 bits), with c = popcount(keep & ~km[k]) the number
-// of hashes with no block boundary between the row and key k (keep: the hashes without a boundary
-// in the row's own part of the gap); packed as 8 bf16 pairs. Returns the sum of P.
-template <typename MaskT>
-__device__ __forceinline__ float p16_carry(const uint32_t (&sv)[16], const MaskT* km, MaskT keep, const SoftmaxK& k2,
-                                           uint32_t (&pk)[8]) {
-  uint64_t ls2[2] = {0ull, 0ull};
-#pragma unroll
-  for (int g4 = 0; g4 < 4; ++g4) {
-    MaskT bb[4];
-    load4(km + 4 * g4, bb);
-#pragma unroll
-    for (int e2 = 0; e2 < 2; ++e2) {
-      const int kk = 4 * g4 + 2 * e2;
-      float x0, x1;
-      f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[kk]), __uint_as_float(sv[kk + 1])), k2.sc2, k2.negm2), x0, x1);
-      const uint32_t c0 = 0x4B000000u | static_cast<uint32_t>(popc_m(static_cast<MaskT>(keep & ~bb[2 * e2])));
-      const uint32_t c1 = 0x4B000000u | static_cast<uint32_t>(popc_m(static_cast<MaskT>(keep & ~bb[2 * e2 + 1])));
-      const uint64_t w2 = f2_add(f2_pack(__uint_as_float(c0), __uint_as_float(c1)), k2.neg2p23);
-      const uint64_t p2 = f2_mul(f2_pack(ex2_approx(x0), ex2_approx(x1)), w2);
-      ls2[e2] = f2_add(ls2[e2], p2);
-      float p0, p1;
-      f2_unpack(p2, p0, p1);
-      pk[2 * g4 + e2] = pack_bf16x2(p0, p1);
-    }
-  }
-  float a0, a1, b0, b1;
-  f2_unpack(ls2[0], a0, a1);
-  f2_unpack(ls2[1], b0, b1);
-  return (a0 + a1) + (b0 + b1);
-}
-
 // Exact ALiBi: P = 2^(S sc - m - lam |i - j|) for 16 keys, with t0 = lam (i - j) at the first key
 // (i - j falls by one per key) and keys k > lim dropped (the causal mask, and keys past n, which
 // the tensor map reads as zeros). Returns the sum of P.
@@ -190,9 +158,10 @@ __device__ __forceinline__ float p16_alibi(const uint32_t (&sv)[16], float t0, f
   return (ls[0] + ls[1]) + (ls[2] + ls[3]);
 }
 
-// The same with the counts given as bytes: the count of key k in byte k % 4 of c4[k / 4].
-__device__ __forceinline__ float p16_counts(const uint32_t (&sv)[16], const uint32_t (&c4)[4], const SoftmaxK& k2,
-                                            uint32_t (&pk)[8]) {
+// P = c 2^(S sc - m) for 16 keys (S as raw fp32 bits), with cf[k] the float bits of 2^23 + c_k;
+// packed as 8 bf16 pairs. Returns the sum of P.
+__device__ __forceinline__ float p16_cf(const uint32_t (&sv)[16], const uint32_t (&cf)[16], const SoftmaxK& k2,
+                                        uint32_t (&pk)[8]) {
   uint64_t ls2[2] = {0ull, 0ull};
 #pragma unroll
   for (int g4 = 0; g4 < 4; ++g4) {
@@ -201,10 +170,7 @@ __device__ __forceinline__ float p16_counts(const uint32_t (&sv)[16], const uint
       const int kk = 4 * g4 + 2 * e2;
       float x0, x1;
       f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[kk]), __uint_as_float(sv[kk + 1])), k2.sc2, k2.negm2), x0, x1);
-      // bytes 2 e2 and 2 e2 + 1 of c4[g4] under the exponent bits of 2^23
-      const uint32_t c0 = __byte_perm(c4[g4], 0x4B000000u, 0x7540u | (2u * e2));
-      const uint32_t c1 = __byte_perm(c4[g4], 0x4B000000u, 0x7540u | (2u * e2 + 1u));
-      const uint64_t w2 = f2_add(f2_pack(__uint_as_float(c0), __uint_as_float(c1)), k2.neg2p23);
+      const uint64_t w2 = f2_add(f2_pack(__uint_as_float(cf[kk]), __uint_as_float(cf[kk + 1])), k2.neg2p23);
       const uint64_t p2 = f2_mul(f2_pack(ex2_approx(x0), ex2_approx(x1)), w2);
       ls2[e2] = f2_add(ls2[e2], p2);
       float p0, p1;
@@ -660,15 +626,34 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
             const int jc = ms.j0 + 16 * ch;
             const int d0 = a_i0 + r - jc;
             lsum += p16_alibi(sv, lam * static_cast<float>(d0), lam, min(kCausal ? d0 : 16, n - 1 - jc), sc, neg_m, pk);
-          } else if (kind == 0 && m == quarter) {
-            // the warp's own block on the diagonal: counts from the scan (words 4 kh .. 4 kh + 3)
-            uint32_t c4[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) c4[u] = sm.cw[4 * kh + u][threadIdx.x];
-            lsum += p16_counts(sv, c4, k2, pk);
           } else {
-            const bool below = kind == 1 || (kind == 0 && m < quarter);
-            lsum += p16_carry<MaskT>(sv, km_tile + 16 * ch, below ? keep_lo : keep_hi, k2, pk);
+            // the chunk's counts as the float bits of 2^23 + c, from the diagonal scan's bytes or
+            // from the masks, then one P body for both (a second copy of it in the loop costs more
+            // in instruction fetch than the extra integer work here)
+            uint32_t cf[16];
+            if (kind == 0 && m == quarter) {
+              // the warp's own block on the diagonal: counts from the scan (words 4 kh .. 4 kh + 3)
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const uint32_t c4 = sm.cw[4 * kh + u][threadIdx.x];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) cf[4 * u + e] = __byte_perm(c4, 0x4B000000u, 0x7540u | e);
+              }
+            } else {
+              // c = popcount(keep & ~km[k]): the hashes with no block boundary between the row and key k
+              const bool below = kind == 1 || (kind == 0 && m < quarter);
+              const MaskT keep = below ? keep_lo : keep_hi;
+              const MaskT* km = km_tile + 16 * ch;
+#pragma unroll
+              for (int g4 = 0; g4 < 4; ++g4) {
+                MaskT bb[4];
+                load4(km + 4 * g4, bb);
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  cf[4 * g4 + e] = 0x4B000000u | static_cast<uint32_t>(popc_m(static_cast<MaskT>(keep & ~bb[e])));
+              }
+            }
+            lsum += p16_cf(sv, cf, k2, pk);
           }
         } else {
 #pragma unroll

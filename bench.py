@@ -33,7 +33,8 @@ import workloads  # noqa: E402
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 TILE = 128
-ATTN_KERNEL_SRC = os.path.join(ROOT, "alibi_positional_lsh_b200", "csrc", "plsh_attn_tc.cu")
+ATTN_KERNEL_SRC = [os.path.join(ROOT, "alibi_positional_lsh_b200", "csrc", f) for f in
+                   ("plsh_attn_tc.cu", "plsh_sm100.cuh", "plsh_tile_common.cuh", "plsh_internal.h")]
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "attn_tc_qwen3_0p6b_n32k.md")
 
 
@@ -49,8 +50,12 @@ def load_peaks():
 
 
 def kernel_source_hash() -> str:
-    with open(ATTN_KERNEL_SRC, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """Hash of the attention kernel's source and the headers it is built from."""
+    h = hashlib.sha256()
+    for path in ATTN_KERNEL_SRC:
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def profiled_traffic():
