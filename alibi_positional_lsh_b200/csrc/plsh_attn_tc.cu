@@ -26,7 +26,9 @@
 // and odd index): S(g+1) = Q K^T is issued before O += P(g) V, so the tensor
 // core computes the next tile's scores while the softmax works on the
 // current one; the softmax turns S into bf16 P written back over S, and the
-// PV MMA reads P from TMEM.
+// PV MMA reads P from TMEM. An item's epilogue (O / l to global memory) runs
+// after the next tile's mask-only work (the diagonal scan), so that work
+// overlaps the item's last PV on the tensor core.
 //
 // Weights. P_ij = c_ij 2^(S_ij log2(e)/sqrt(d) - m): the count multiplies the
 // exponential as an exact small-integer float, so no logarithm is taken.
@@ -507,14 +509,83 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     float lam = 0.0f;  // exact ALiBi: log2(e) / sigma of the item's head
     int a_i0 = 0;      // exact ALiBi: the item's first row
     int items = 0;     // items finished by this warp
+    bool pend = false;  // an item's epilogue is pending
+    int pend_tx = 0, pend_g = 0;  // its item index and last tile
     for (int g = 0;; ++g) {
       const int st = g % kMaskStages;
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.m_full[st], static_cast<uint32_t>(g / kMaskStages) & 1u,
                                              abort_flag, err, prm.wait_ns)))
         break;
       const MaskStage<MaskT>& ms = sm.m[st];
-      if (!ms.valid) break;
+      const bool valid = ms.valid != 0;
       const int kind = ms.kind, first = ms.first, last = ms.last, tx = ms.x;
+      // weights that need only the masks: the diagonal's own block and its carries (before the
+      // previous item's epilogue, whose last PV is still running on the tensor core)
+      MaskT lo = 0, hi = 0;
+      if (!kAlibi && valid && kind == 0) diag_scan<MaskT, true, !kCausal>(ms, quarter, r, sw, &sm.cw[0][threadIdx.x], kSoftmaxWarps * 32, lo, hi);
+      // ---- the previous item's epilogue: O / l once its last PV has completed, stored four rows
+      // at a time by each lane quad (thread t: columns 0..63 of its row, thread t + 16: 64..127)
+      if (pend) {
+        pend = false;
+        const int kb = items & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.pv_done[pend_g & 1], static_cast<uint32_t>(pend_g >> 1) & 1u, abort_flag, err, prm.wait_ns)))
+          break;
+        tc_fence_after();
+        const float ltot = l + __shfl_xor_sync(0xffffffffu, l, 16);
+        const int BT = prm.B * prm.T;
+        const int hh = (H <= kMaxSortedHeads) ? static_cast<int>(sm.order[pend_tx / BT]) : pend_tx / BT;
+        const int rem = pend_tx % BT;
+        const int bb = rem / prm.T, i0 = (rem % prm.T) * kTile;
+        const float inv = 1.0f / ltot;
+        const int p4 = lane & 3;
+        const int quad_row = quarter * 32 + hq * 16 + ((lane & 15) & ~3);  // first of the quad's four rows
+        const uint32_t o_row = tmem + lane_off + kColO + 128u * static_cast<uint32_t>(kb);
+        __nv_bfloat16* obase = O + (static_cast<size_t>(bb) * H + hh) * static_cast<size_t>(n) * kD + 64 * kh;
+#pragma unroll 1
+        for (int blk = 0; blk < 2; ++blk) {
+          uint32_t raw[32];
+          tmem_ld16x2_32<64>(o_row + 32u * blk, raw);
+          tmem_wait_ld();
+          regs_after_wait(raw);
+          uint32_t a[4][4];  // [16-byte chunk][word] of this row's 32 columns
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+              a[c][w] = pack_bf16x2(__uint_as_float(raw[8 * c + 2 * w]) * inv,
+                                    __uint_as_float(raw[8 * c + 2 * w + 1]) * inv);
+          // 4x4 transpose of 16-byte chunks inside the quad: lane p then holds chunk p of the quad's rows
+#pragma unroll
+          for (int msk = 2; msk >= 1; msk >>= 1) {
+            const bool lo_lane = (p4 & msk) == 0;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              if (c & msk) continue;
+#pragma unroll
+              for (int w = 0; w < 4; ++w) {
+                const uint32_t send = lo_lane ? a[c | msk][w] : a[c][w];
+                const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, msk);
+                if (lo_lane) a[c | msk][w] = recv;
+                else a[c][w] = recv;
+              }
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int row = i0 + quad_row + e;
+            if (row < n)
+              *reinterpret_cast<uint4*>(obase + static_cast<size_t>(row) * kD + 32 * blk + 8 * p4) =
+                  make_uint4(a[e][0], a[e][1], a[e][2], a[e][3]);
+          }
+        }
+        tc_fence_before();
+        const int i = i0 + r;
+        if (kh == 0 && i < n)
+          row_sum[(static_cast<size_t>(bb) * H + hh) * n + i] =
+              (log2f(ltot) + m2) * 0.6931471805599453f - (kAlibi ? 0.0f : logf(static_cast<float>(s)));
+        ++items;
+      }
+      if (!valid) break;
       if (first) {
         m2 = -INFINITY;
         l = 0.0f;
@@ -525,9 +596,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
           a_i0 = ((tx % BT) % prm.T) * kTile;
         }
       }
-      // weights that need only the masks: the diagonal's own block and its carries
-      MaskT lo = 0, hi = 0;
-      if (!kAlibi && kind == 0) diag_scan<MaskT, true, !kCausal>(ms, quarter, r, sw, &sm.cw[0][threadIdx.x], kSoftmaxWarps * 32, lo, hi);
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[g & 1], static_cast<uint32_t>(g >> 1) & 1u, abort_flag, err, prm.wait_ns)))
         break;
       tc_fence_after();
@@ -678,66 +746,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.p_full[g & 1]);
 
-      // ---- the item's epilogue: O / l once its last PV has completed, stored four rows at a
-      // time by each lane quad (thread t: columns 0..63 of its row, thread t + 16: 64..127)
-      if (last) {
-        const int kb = items & 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(&sm.pv_done[g & 1], static_cast<uint32_t>(g >> 1) & 1u, abort_flag, err, prm.wait_ns)))
-          break;
-        tc_fence_after();
-        const float ltot = l + __shfl_xor_sync(0xffffffffu, l, 16);
-        const int BT = prm.B * prm.T;
-        const int hh = (H <= kMaxSortedHeads) ? static_cast<int>(sm.order[tx / BT]) : tx / BT;
-        const int rem = tx % BT;
-        const int bb = rem / prm.T, i0 = (rem % prm.T) * kTile;
-        const float inv = 1.0f / ltot;
-        const int p4 = lane & 3;
-        const int quad_row = quarter * 32 + hq * 16 + ((lane & 15) & ~3);  // first of the quad's four rows
-        const uint32_t o_row = tmem + lane_off + kColO + 128u * static_cast<uint32_t>(kb);
-        __nv_bfloat16* obase = O + (static_cast<size_t>(bb) * H + hh) * static_cast<size_t>(n) * kD + 64 * kh;
-#pragma unroll 1
-        for (int blk = 0; blk < 2; ++blk) {
-          uint32_t raw[32];
-          tmem_ld16x2_32<64>(o_row + 32u * blk, raw);
-          tmem_wait_ld();
-          regs_after_wait(raw);
-          uint32_t a[4][4];  // [16-byte chunk][word] of this row's 32 columns
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-#pragma unroll
-            for (int w = 0; w < 4; ++w)
-              a[c][w] = pack_bf16x2(__uint_as_float(raw[8 * c + 2 * w]) * inv,
-                                    __uint_as_float(raw[8 * c + 2 * w + 1]) * inv);
-          // 4x4 transpose of 16-byte chunks inside the quad: lane p then holds chunk p of the quad's rows
-#pragma unroll
-          for (int msk = 2; msk >= 1; msk >>= 1) {
-            const bool lo_lane = (p4 & msk) == 0;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              if (c & msk) continue;
-#pragma unroll
-              for (int w = 0; w < 4; ++w) {
-                const uint32_t send = lo_lane ? a[c | msk][w] : a[c][w];
-                const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, msk);
-                if (lo_lane) a[c | msk][w] = recv;
-                else a[c][w] = recv;
-              }
-            }
-          }
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int row = i0 + quad_row + e;
-            if (row < n)
-              *reinterpret_cast<uint4*>(obase + static_cast<size_t>(row) * kD + 32 * blk + 8 * p4) =
-                  make_uint4(a[e][0], a[e][1], a[e][2], a[e][3]);
-          }
-        }
-        tc_fence_before();
-        const int i = i0 + r;
-        if (kh == 0 && i < n)
-          row_sum[(static_cast<size_t>(bb) * H + hh) * n + i] =
-              (log2f(ltot) + m2) * 0.6931471805599453f - (kAlibi ? 0.0f : logf(static_cast<float>(s)));
-        ++items;
+      if (last) {  // the item's epilogue runs at the top of the next iteration
+        pend = true;
+        pend_tx = tx;
+        pend_g = g;
       }
     }
   }

@@ -23,7 +23,9 @@
 //                       dS^T over them, dV += P^T dO and dK += dS^T Q (TS MMAs).
 // Tensor Memory holds S, dP and the accumulators (dQ; dV and dK): the score MMAs of a tile wait
 // for the previous tile's gradient MMAs to read the elementwise results (one thread's MMAs run in
-// order). D_i comes from the existing row-dot kernel before both.
+// order). An item's epilogue (the accumulators to global memory) runs after the next tile's
+// mask-only work (the diagonal scan), which so overlaps the item's last gradient MMAs. D_i comes
+// from the existing row-dot kernel before both.
 #include <cmath>
 
 #include <cuda.h>
@@ -122,39 +124,10 @@ struct KvIter {
   __device__ __forceinline__ bool last() const { return it == total - 1 && sub == group() - 1; }
 };
 
-// ds = c 2^(S sc - bias) (dP - Dv) for 16 keys (S, dP as raw fp32 bits) with c = popcount(keep &
-// ~km[k]), per-row bias and Dv; packed as 8 bf16 pairs.
-template <typename MaskT>
-__device__ __forceinline__ void ds16_carry(const uint32_t (&sv)[16], const uint32_t (&dv)[16], const MaskT* km,
-                                           MaskT keep, uint64_t sc2, uint64_t nbias2, uint64_t nD2,
-                                           uint32_t (&pk)[8]) {
-  const uint64_t n2p23 = f2_pack(-8388608.0f, -8388608.0f);
-#pragma unroll
-  for (int g4 = 0; g4 < 4; ++g4) {
-    MaskT bb[4];
-    load4(km + 4 * g4, bb);
-#pragma unroll
-    for (int e2 = 0; e2 < 2; ++e2) {
-      const int kk = 4 * g4 + 2 * e2;
-      float x0, x1;
-      f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[kk]), __uint_as_float(sv[kk + 1])), sc2, nbias2), x0, x1);
-      const uint32_t c0 = 0x4B000000u | static_cast<uint32_t>(popc_m(static_cast<MaskT>(keep & ~bb[2 * e2])));
-      const uint32_t c1 = 0x4B000000u | static_cast<uint32_t>(popc_m(static_cast<MaskT>(keep & ~bb[2 * e2 + 1])));
-      const uint64_t w2 = f2_add(f2_pack(__uint_as_float(c0), __uint_as_float(c1)), n2p23);
-      const uint64_t p2 = f2_mul(f2_pack(ex2_approx(x0), ex2_approx(x1)), w2);
-      const uint64_t d2 = f2_add(f2_pack(__uint_as_float(dv[kk]), __uint_as_float(dv[kk + 1])), nD2);
-      float s0, s1;
-      f2_unpack(f2_mul(p2, d2), s0, s1);
-      pk[2 * g4 + e2] = pack_bf16x2(s0, s1);
-    }
-  }
-}
-
-// The same with the counts given as bytes (the diagonal's own block): count of key k in byte k % 4
-// of c4[k / 4].
-__device__ __forceinline__ void ds16_counts(const uint32_t (&sv)[16], const uint32_t (&dv)[16],
-                                            const uint32_t (&c4)[4], uint64_t sc2, uint64_t nbias2, uint64_t nD2,
-                                            uint32_t (&pk)[8]) {
+// dS = P (dP - D) for 16 keys with P = c 2^(S sc - bias) (S, dP as raw fp32 bits; cf[k] the float
+// bits of 2^23 + c_k), packed as 8 bf16 pairs.
+__device__ __forceinline__ void ds16_cf(const uint32_t (&sv)[16], const uint32_t (&dv)[16], const uint32_t (&cf)[16],
+                                        uint64_t sc2, uint64_t nbias2, uint64_t nD2, uint32_t (&pk)[8]) {
   const uint64_t n2p23 = f2_pack(-8388608.0f, -8388608.0f);
 #pragma unroll
   for (int g4 = 0; g4 < 4; ++g4) {
@@ -163,9 +136,7 @@ __device__ __forceinline__ void ds16_counts(const uint32_t (&sv)[16], const uint
       const int kk = 4 * g4 + 2 * e2;
       float x0, x1;
       f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[kk]), __uint_as_float(sv[kk + 1])), sc2, nbias2), x0, x1);
-      const uint32_t c0 = __byte_perm(c4[g4], 0x4B000000u, 0x7540u | (2u * e2));
-      const uint32_t c1 = __byte_perm(c4[g4], 0x4B000000u, 0x7540u | (2u * e2 + 1u));
-      const uint64_t w2 = f2_add(f2_pack(__uint_as_float(c0), __uint_as_float(c1)), n2p23);
+      const uint64_t w2 = f2_add(f2_pack(__uint_as_float(cf[kk]), __uint_as_float(cf[kk + 1])), n2p23);
       const uint64_t p2 = f2_mul(f2_pack(ex2_approx(x0), ex2_approx(x1)), w2);
       const uint64_t d2 = f2_add(f2_pack(__uint_as_float(dv[kk]), __uint_as_float(dv[kk + 1])), nD2);
       float s0, s1;
@@ -474,7 +445,6 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
             mma_ts(tmem + kColAcc, tmem + s_col(cur.g) + 8u * kk,
                    (st ? kmn_desc[1] : kmn_desc[0]) + static_cast<uint64_t>((kk * 2048) >> 4), idesc_nn,
                    (!cur.first() || kk > 0) ? 1u : 0u);
-          mma_commit(&sm.g_done);
           mma_commit(&sm.k_empty[st]);
         };
         if (s_early) {  // within an item: the next tile's dP first, which the elementwise warps wait for
@@ -482,6 +452,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
           issue_dq();
         } else {        // the item's last tile: its dQ first, which the item's epilogue waits for
           issue_dq();
+          mma_commit(&sm.g_done);  // once per item: the item's dQ is complete
           if (nxt.valid && !(ok = issue_s(nxt) && issue_dp(nxt))) break;
         }
         cur.next();
@@ -568,14 +539,34 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
     uint64_t nbias2 = 0, nD2 = 0;
     MaskT Y = 0, Z = 0;
     int bb = 0, hh = 0, i0 = 0;
+    bool pend = false;  // an item's epilogue is pending (the item of bb, hh, i0)
+    int items = 0;      // items whose epilogue is done
     for (int g = 0;; ++g) {
       const int st = g % kMaskStages;
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.m_full[st], static_cast<uint32_t>(g / kMaskStages) & 1u,
                                              abort_flag, err, wait_ns)))
         break;
       const MaskStage<MaskT>& ms = sm.m[st];
-      if (!ms.valid) break;
+      const bool valid = ms.valid != 0;
       const int kind = ms.kind, first = ms.first, last = ms.last, tx = ms.x;
+      // the mask-only work first, while the previous item's last dQ MMA runs
+      MaskT lo = 0, hi = 0;
+      if (valid && kind == 0) diag_scan<MaskT, true, !kCausal>(ms, quarter, r, s, &sm.cw[0][threadIdx.x], kElemWarps * 32, lo, hi);
+      if (pend) {
+        pend = false;
+        // the previous item's dQ once its last MMA has completed (g_done completes once per item,
+        // and the next completion needs this item's successor's dS, so one parity wait is exact):
+        // dQ / sqrt(d)
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.g_done, static_cast<uint32_t>(items) & 1u, abort_flag, err, wait_ns)))
+          break;
+        ++items;
+        tc_fence_after();
+        store_rows(tmem + lane_off + kColAcc, 1.0f / sqrtf(static_cast<float>(kD)),
+                   dQ + (static_cast<size_t>(bb) * H + hh) * static_cast<size_t>(n) * kD, i0,
+                   quarter * 32 + hq * 16 + ((lane & 15) & ~3), n, kh, lane);
+        tc_fence_before();
+      }
+      if (!valid) break;
       if (first) {
         // P_ij = c_ij 2^(S_ij log2(e)/sqrt(d) - (L_i log2(e) + log2 s)); rows past n get L = D = 0
         const int BT = prm.B * prm.T;
@@ -590,8 +581,6 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
         nbias2 = f2_pack(nb, nb);
         nD2 = f2_pack(-Dv, -Dv);
       }
-      MaskT lo = 0, hi = 0;
-      if (kind == 0) diag_scan<MaskT, true, !kCausal>(ms, quarter, r, s, &sm.cw[0][threadIdx.x], kElemWarps * 32, lo, hi);
       const int n_pairs = (kCausal && kind == 0) ? quarter + 1 : kTile / 32;
       const MaskT Zc = static_cast<MaskT>(Z | ms.bm[0]);
       const MaskT keep_lo = static_cast<MaskT>(FULL & ~(kind == 1 ? Y : lo));
@@ -623,15 +612,30 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
           regs_after_wait(sv);
           regs_after_wait(dv);
           const int ch = 2 * m + kh;
+          // the chunk's counts as the float bits of 2^23 + c, from the diagonal scan's bytes or from
+          // the masks, then one dS body for both (a smaller loop than two inlined bodies)
+          uint32_t cf[16];
           if (kind == 0 && m == quarter) {
-            uint32_t c4[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) c4[u] = sm.cw[4 * kh + u][threadIdx.x];
-            ds16_counts(sv, dv, c4, sc2, nbias2, nD2, pk);
+            for (int u = 0; u < 4; ++u) {
+              const uint32_t c4 = sm.cw[4 * kh + u][threadIdx.x];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) cf[4 * u + e] = __byte_perm(c4, 0x4B000000u, 0x7540u | e);
+            }
           } else {
             const bool below = kind == 1 || (kind == 0 && m < quarter);
-            ds16_carry<MaskT>(sv, dv, km_tile + 16 * ch, below ? keep_lo : keep_hi, sc2, nbias2, nD2, pk);
+            const MaskT keep = below ? keep_lo : keep_hi;
+            const MaskT* km = km_tile + 16 * ch;
+#pragma unroll
+            for (int g4 = 0; g4 < 4; ++g4) {
+              MaskT kb4[4];
+              load4(km + 4 * g4, kb4);
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                cf[4 * g4 + e] = 0x4B000000u | static_cast<uint32_t>(popc_m(static_cast<MaskT>(keep & ~kb4[e])));
+            }
           }
+          ds16_cf(sv, dv, cf, sc2, nbias2, nD2, pk);
         } else {
 #pragma unroll
           for (int e = 0; e < 8; ++e) pk[e] = 0u;
@@ -652,22 +656,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.p_full);
-      if (last) {
-        // the item's dQ once its last MMA has completed: dQ / sqrt(d). g_done completes once per tile,
-        // and the next tile's dP is issued before this tile's dQ, so when these warps get here the
-        // latest completed phase can be g - 2: wait for phase g - 1, then g (a parity wait alone
-        // would take phase g - 2 for g)
-        if (g >= 1 && !__all_sync(0xffffffffu, mbar_wait(&sm.g_done, static_cast<uint32_t>(g - 1) & 1u, abort_flag,
-                                                         err, wait_ns)))
-          break;
-        if (!__all_sync(0xffffffffu, mbar_wait(&sm.g_done, static_cast<uint32_t>(g) & 1u, abort_flag, err, wait_ns)))
-          break;
-        tc_fence_after();
-        store_rows(tmem + lane_off + kColAcc, 1.0f / sqrtf(static_cast<float>(kD)),
-                   dQ + (static_cast<size_t>(bb) * H + hh) * static_cast<size_t>(n) * kD, i0,
-                   quarter * 32 + hq * 16 + ((lane & 15) & ~3), n, kh, lane);
-        tc_fence_before();
-      }
+      if (last) pend = true;  // the item's epilogue runs at the top of the next iteration
     }
   }
 
@@ -933,6 +922,10 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
     const float sc = kLog2e / sqrtf(static_cast<float>(kD));
     const uint64_t sc2 = f2_pack(sc, sc);
     MaskT Y = 0, Z = 0;
+    bool pend = false;  // an item's epilogue is pending (item pend_tx, last tile pend_g; g_done completes
+                        // once per tile, and tile pend_g + 1's MMAs wait for these warps, so one
+                        // parity wait is exact)
+    int pend_g = 0, pend_tx = 0;
     for (int g = 0;; ++g) {
       const int st = g % kMaskStages;
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.m_full[st], static_cast<uint32_t>(g / kMaskStages) & 1u,
@@ -940,10 +933,26 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         break;
       const KvStage<MaskT>& ks = sm.m[st];
       const MaskStage<MaskT>& ms = ks.m;
-      if (!ms.valid) break;
+      const bool valid = ms.valid != 0;
       const int kind = ms.kind, last = ms.last, tx = ms.x;
+      // the mask-only work first, while the previous item's last MMAs run
       MaskT lo = 0, hi = 0;
-      if (kind == 0) diag_scan<MaskT, !kCausal, true>(ms, quarter, r, s, &sm.cw[0][threadIdx.x], kElemWarps * 32, lo, hi);
+      if (valid && kind == 0) diag_scan<MaskT, !kCausal, true>(ms, quarter, r, s, &sm.cw[0][threadIdx.x], kElemWarps * 32, lo, hi);
+      if (pend) {
+        pend = false;
+        // the previous item's dV and dK once its last MMAs have completed (dK / sqrt(d))
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.g_done, static_cast<uint32_t>(pend_g) & 1u, abort_flag, err, wait_ns)))
+          break;
+        tc_fence_after();
+        const int BT = prm.B * prm.T;
+        const int gg = pend_tx / BT, bb = (pend_tx % BT) / prm.T, j0 = (pend_tx % prm.T) * kTile;
+        const size_t plane = (static_cast<size_t>(bb) * prm.H_kv + gg) * static_cast<size_t>(n) * kD;
+        const int quad_row = quarter * 32 + hq * 16 + ((lane & 15) & ~3);
+        store_rows(tmem + lane_off + kColDV, 1.0f, dV + plane, j0, quad_row, n, kh, lane);
+        store_rows(tmem + lane_off + kColDK, 1.0f / sqrtf(static_cast<float>(kD)), dK + plane, j0, quad_row, n, kh, lane);
+        tc_fence_before();
+      }
+      if (!valid) break;
       const MaskT Zc = static_cast<MaskT>(Z | ms.bm[0]);
       const MaskT keep_lo = static_cast<MaskT>(FULL & ~(kind == 1 ? Y : lo));
       const MaskT keep_hi = static_cast<MaskT>(FULL & ~(kind == 2 ? Zc : hi));
@@ -1005,18 +1014,10 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.p_full);
-      if (last) {
-        // the item's dV and dK once its last MMAs have completed (dK / sqrt(d))
-        if (!__all_sync(0xffffffffu, mbar_wait(&sm.g_done, static_cast<uint32_t>(g) & 1u, abort_flag, err, wait_ns)))
-          break;
-        tc_fence_after();
-        const int BT = prm.B * prm.T;
-        const int gg = tx / BT, bb = (tx % BT) / prm.T, j0 = (tx % prm.T) * kTile;
-        const size_t plane = (static_cast<size_t>(bb) * prm.H_kv + gg) * static_cast<size_t>(n) * kD;
-        const int quad_row = quarter * 32 + hq * 16 + ((lane & 15) & ~3);
-        store_rows(tmem + lane_off + kColDV, 1.0f, dV + plane, j0, quad_row, n, kh, lane);
-        store_rows(tmem + lane_off + kColDK, 1.0f / sqrtf(static_cast<float>(kD)), dK + plane, j0, quad_row, n, kh, lane);
-        tc_fence_before();
+      if (last) {  // the item's epilogue runs at the top of the next iteration
+        pend = true;
+        pend_g = g;
+        pend_tx = tx;
       }
     }
   }
