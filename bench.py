@@ -113,6 +113,10 @@ class ClockSampler:
                     return
                 time.sleep(self.period)
 
+        # the timed loop's host work (the table draw, the launches) holds the GIL; a short switch
+        # interval lets the sampling thread in every few hundred microseconds
+        self._switch = sys.getswitchinterval()
+        sys.setswitchinterval(0.0002)
         self._thread = threading.Thread(target=loop, daemon=True)
         self._thread.start()
         time.sleep(0.02)
@@ -122,6 +126,7 @@ class ClockSampler:
         if self._thread is not None:
             self._stop.set()
             self._thread.join(timeout=2)
+            sys.setswitchinterval(self._switch)
 
     def summary(self):
         if self.error or not self.samples:
