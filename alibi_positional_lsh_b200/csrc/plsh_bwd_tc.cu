@@ -24,8 +24,8 @@
 // Tensor Memory holds S, dP and the accumulators (dQ; dV and dK): the score MMAs of a tile wait
 // for the previous tile's gradient MMAs to read the elementwise results (one thread's MMAs run in
 // order). An item's epilogue (the accumulators to global memory) runs after the next tile's
-// mask-only work (the diagonal scan), which so overlaps the item's last gradient MMAs. D_i comes
-// from the existing row-dot kernel before both.
+// mask-only work (the diagonal scan), so that the scan overlaps the item's last gradient MMAs.
+// D_i comes from the existing row-dot kernel before both.
 #include <cmath>
 
 #include <cuda.h>
