@@ -229,6 +229,13 @@ PLSH_API int plsh_window_from_table(const double* table_dev, int H, int s, int n
  *   tile_span_dev, bmask_dev   from plsh_window with the same causal flag.
  *   row_sum        [B][H][n] float32 out.
  * Every pointer must be 16-byte aligned.
+ * Range of the scores (bf16, d == 128): the tensor-core kernel scales each
+ * row's exponentials by a running maximum of S taken over every key of the
+ * 32-key chunk pairs it evaluates, weighted or not. If a row's weighted scores
+ * all lie more than about 87 (natural log) below a zero-weight score in those
+ * pairs, its weighted terms underflow: O is NaN and row_sum -inf for that row.
+ * Scores of ordinary attention are far from this (it took Q x 32 on unit
+ * normal inputs to reach it).
  */
 PLSH_API int plsh_attention_fwd(const void* Q, const void* K, const void* V, int dtype, int B, int H,
                        int H_kv, int n, int d, const double* sigma_dev, int s,

@@ -130,6 +130,31 @@ def test_attention_small_full_oracle(B, H, H_kv, n, d, dtype, causal, s, kind):
     PH.assert_close(gpu["O"], gpu["row_sum"], O, R, to, tr, "small")
 
 
+_UNDERFLOW = pytest.mark.xfail(
+    strict=False,
+    reason="known limitation of the fused kernel: its reference maximum is taken over every key of "
+           "a live chunk pair, weighted or not, so a row whose weighted scores all lie more than "
+           "about 87 (natural log) below a zero-weight score in those pairs underflows; with Q x 32 "
+           "row 0 of a causal head (one weighted key beside 31 masked ones) does")
+
+
+@pytest.mark.parametrize("scale,causal", [(8.0, True), pytest.param(32.0, True, marks=_UNDERFLOW),
+                                          pytest.param(32.0, False, marks=_UNDERFLOW)])
+def test_attention_large_scores_full_oracle(scale, causal):
+    """Q scaled by a power of two (exact in bf16): scores spread over tens of log2 units, so a
+    row's maximum rises from tile to tile by more than the kernel's rescale margin. The output
+    must still match the float64 oracle, which works on the same scaled inputs."""
+    B, H, H_kv, n, d, s = 1, 2, 1, 1000, 128, 20
+    q, k, v = _inputs(B, H, H_kv, n, d, torch.bfloat16, 4242 + int(scale))
+    q = (q.float() * scale).to(torch.bfloat16)
+    sig = _sigmas("mixed", H)
+    gpu = PH.run_gpu(B, H, H_kv, n, d, s, causal, sig, 11, q, k, v)
+    assert gpu["errors"] == []
+    O, R = PH.oracle_rows(q, k, v, gpu["table"], causal, None)
+    to, tr = PH.tolerance(torch.bfloat16, v)
+    PH.assert_close(gpu["O"], gpu["row_sum"], O, R, to, tr, f"scores x{scale}")
+
+
 def test_singleton_bins_give_v_and_one_bin_gives_softmax():
     n, d = 500, 128
     q, k, v = _inputs(1, 2, 2, n, d, torch.bfloat16, 9)
