@@ -91,3 +91,20 @@ def test_tensor_core_backward_tiles(causal):
                 rows = rows[rows >= t * 128]
             walked += len({int(r) // 128 for r in rows} | {t})
     assert bench.bwd_tc_tiles(spans, kspans, causal) == (bench.kernel_tiles(spans, causal), walked)
+
+
+def test_profiled_traffic_follows_the_kernel_source(tmp_path, monkeypatch):
+    """The committed DRAM traffic is used only while the attention kernel's source and headers
+    hash to the value recorded beside it; a change to any of them drops it (reported as null)."""
+    srcs = []
+    for name in ("kernel.cu", "a.cuh", "b.h"):
+        p = tmp_path / name
+        p.write_text(f"// {name}\n")
+        srcs.append(str(p))
+    monkeypatch.setattr(bench, "ATTN_KERNEL_SRC", srcs)
+    summary = tmp_path / "summary.md"
+    summary.write_text(f"kernel_source_sha256_16: {bench.kernel_source_hash()}\ntraffic_bytes_per_launch: 12345\n")
+    monkeypatch.setattr(bench, "PROFILE_SUMMARY", str(summary))
+    assert bench.profiled_traffic() == 12345.0
+    (tmp_path / "a.cuh").write_text("// a.cuh, changed\n")
+    assert bench.profiled_traffic() is None
